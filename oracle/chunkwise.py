@@ -1,0 +1,166 @@
+"""Float64 numpy statements of DeltaNet's chunk form, for tiny inputs.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  These functions are a
+second, independent oracle: they follow the algebra of "Linear Attention,
+Visualized" (section "DeltaNet: correcting memory collisions") step by step,
+one (sequence, head) at a time, in the page's row-vector convention:
+S is d_k x d_v, reads are ``k S`` and ``q S``.  Library primitives used as
+steps: matrix products and a triangular solve.
+
+Every function takes K, Q as [n, d_k], V as [n, d_v], beta as [n], S0 as
+[d_k, d_v] (all float64 numpy arrays).
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.linalg import solve_triangular
+
+
+def causal_masks(n: int):
+    """Inclusive causal mask M and its strict part M^- = M - I (section
+    "The triangular correction system")."""
+    M = np.tril(np.ones((n, n)))
+    return M, M - np.eye(n)
+
+
+def full_sequence(Q, K, V, beta, S0=None):
+    """Full-sequence parallel form (subsections "The triangular correction
+    system", "Solving for U" and "Parallel output").
+
+    L = (K K^T) o M^-, (I + B L) U = B V, O = (Q K^T o M) U.  The page starts from
+    S0 = 0; with a nonzero incoming state the prediction gains the term k_t S0,
+    so the right-hand side becomes B (V - K S0), the readout gains Q S0 and the
+    final state is S0 + K^T U (the same substitution the page makes for a chunk
+    in "Correct the incoming state").
+    Returns (O, S_final, U).
+    """
+    n, dk = K.shape
+    dv = V.shape[1]
+    if S0 is None:
+        S0 = np.zeros((dk, dv))
+    M, Mm = causal_masks(n)
+    Bm = np.diag(beta)
+    L = (K @ K.T) * Mm
+    A = np.eye(n) + Bm @ L                      # unit lower triangular
+    R = Bm @ (V - K @ S0)
+    U = solve_triangular(A, R, lower=True, unit_diagonal=True)
+    O = Q @ S0 + ((Q @ K.T) * M) @ U
+    return O, S0 + K.T @ U, U
+
+
+def chunk_factors(Kc, Vc, bc):
+    """Per-chunk factors of the "Complete per-chunk algorithm":
+    L_r = (K_r K_r^T) o M_c^-, (I + B_r L_r) T_r = B_r, W_r = T_r K_r, U_r = T_r V_r.
+    Returns (L, T, W, U)."""
+    c = Kc.shape[0]
+    _, Mm = causal_masks(c)
+    Bm = np.diag(bc)
+    L = (Kc @ Kc.T) * Mm
+    T = solve_triangular(np.eye(c) + Bm @ L, Bm, lower=True, unit_diagonal=True)
+    return L, T, T @ Kc, (T @ Vc if Vc is not None else None)
+
+
+def chunk_step(Qc, Kc, Vc, bc, S):
+    """One chunk of the boundary pass: Z = U - W S, O = Q S + (Q K^T o M_c) Z,
+    S' = S + K^T Z.  Returns (O_chunk, S')."""
+    M, _ = causal_masks(Kc.shape[0])
+    _, _, W, U = chunk_factors(Kc, Vc, bc)
+    Z = U - W @ S
+    O = Qc @ S + ((Qc @ Kc.T) * M) @ Z
+    return O, S + Kc.T @ Z
+
+
+def chunk_bounds(n: int, C: int):
+    """Chunks start at the sequence start; the last one may be shorter (a
+    chunk of any size is exact, subsection "Cost")."""
+    return [(s, min(n, s + C)) for s in range(0, n, C)]
+
+
+def chunkwise(Q, K, V, beta, S0=None, C: int = 64):
+    """The per-chunk algorithm threaded over all chunks from S0.
+    Returns (O, S_final)."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    O = np.zeros((n, dv))
+    for s, e in chunk_bounds(n, C):
+        O[s:e], S = chunk_step(Q[s:e], K[s:e], V[s:e], beta[s:e], S)
+    return O, S
+
+
+def token_transition(k, b):
+    """A_{r,l} = I - beta k^T k (subsection "One chunk as an affine recurrence")."""
+    return np.eye(k.shape[0]) - b * np.outer(k, k)
+
+
+def ordered_product(K, beta):
+    """Lambda[1:n] = A_n ... A_1, multiplied out explicitly (later tokens on the
+    left, since S^(l) = A_l S^(l-1) + X_l)."""
+    P = np.eye(K.shape[1])
+    for t in range(K.shape[0]):
+        P = token_transition(K[t], beta[t]) @ P
+    return P
+
+
+def wy_rows(K, beta):
+    """Rows of W_r built one transition at a time (subsection "Compact the
+    transition product with WY"):
+    w_l = beta_l (k_l - sum_{i<l} (k_l k_i^T) w_i)."""
+    W = np.zeros_like(K)
+    for l in range(K.shape[0]):
+        acc = K[l].copy()
+        for i in range(l):
+            acc -= (K[l] @ K[i]) * W[i]
+        W[l] = beta[l] * acc
+    return W
+
+
+def segment_map(K, V, beta, C: int = 64):
+    """Affine map of a run of chunks: S_end = P S_start + H.
+
+    The pages state the one-chunk case, S_{r+1} = Lambda_r[1:C] S_r + H_r with
+    Lambda_r[1:C] = I - K_r^T W_r and H_r the zero-start local writes.  Composing
+    two affine maps gives (P2, H2) o (P1, H1) = (P2 P1, P2 H1 + H2); a segment is
+    the composition of its chunks, taken in chunk order.
+    Returns (P [d_k, d_k], H [d_k, d_v]).
+    """
+    dk = K.shape[1]
+    dv = V.shape[1]
+    P = np.eye(dk)
+    H = np.zeros((dk, dv))
+    for s, e in chunk_bounds(K.shape[0], C):
+        _, _, W, U = chunk_factors(K[s:e], V[s:e], beta[s:e])
+        Lam = np.eye(dk) - K[s:e].T @ W
+        Hr = K[s:e].T @ U
+        P, H = Lam @ P, Lam @ H + Hr
+    return P, H
+
+
+def context_parallel(Q, K, V, beta, S0=None, C: int = 64, n_segments: int = 2):
+    """Context parallelism over chunk segments ("Context Parallelism for
+    DeltaNet", section 3): each segment summarises itself as (P_g, H_g), a short
+    scan composes the true segment-start states, then every segment reruns its
+    chunks from its own start state.  Exact, so it must equal ``chunkwise``.
+    Returns (O, S_final, starts)."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    chunks = chunk_bounds(n, C)
+    nc = len(chunks)
+    n_segments = max(1, min(n_segments, nc))
+    edges = [round(g * nc / n_segments) for g in range(n_segments + 1)]
+    segs = [(chunks[edges[g]][0], chunks[edges[g + 1] - 1][1]) for g in range(n_segments)]
+    maps = [segment_map(K[s:e], V[s:e], beta[s:e], C) for s, e in segs]
+    starts = [np.zeros((dk, dv)) if S0 is None else S0.copy()]
+    for P, H in maps[:-1]:
+        starts.append(P @ starts[-1] + H)
+    O = np.zeros((n, dv))
+    S = None
+    for (s, e), Sg in zip(segs, starts):
+        O[s:e], S = chunkwise(Q[s:e], K[s:e], V[s:e], beta[s:e], Sg, C)
+    return O, S, starts
+
+
+def linear_attention(Q, K, V):
+    """Causal linear attention, parallel form (Q K^T o M) V."""
+    M, _ = causal_masks(K.shape[0])
+    return ((Q @ K.T) * M) @ V
