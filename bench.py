@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise DeltaNet forward pass on B200.
+
+One step = one deltanet_fwd call over the whole workload (every step of the
+path: WY/UT factors, segment summaries, segment scan, boundary pass with
+output).  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
+d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 beta, zero initial state, fp32
+final state), synthetic seeded inputs.  Inputs (q, k, v: 201 MB) exceed the
+126 MB L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+
+Multi-GPU (torchrun, one process per GPU): the path has no exchange step
+between GPUs, so every rank runs an independent replica of the workload
+(weak scaling); ranks meet only at the barriers around the timed region and
+in the max-over-ranks reduction of the timing.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from deltanet_chunkwise_delta_b200 import workloads as wl  # noqa: E402
+
+METRIC = "DeltaNet fwd tokens/sec and TFLOP/s at 1 B200; fraction of roofline"
+CHUNK = 64
+
+
+# ---- algorithmic counts ------------------------------------------------------
+
+def flops_per_token_head(dk: int, dv: int, C: int = CHUNK) -> float:
+    """Algorithmic FLOPs of the per-chunk algorithm per token-head:
+    L (strict-lower K K^T) C^2 d_k, solve C^3/3, W = T K C^2 d_k, U = T V C^2 d_v,
+    W S 2 C d_k d_v, Q S 2 C d_k d_v, masked Q K^T C^2 d_k, (.) Z C^2 d_v,
+    K^T Z 2 C d_k d_v; divided by C."""
+    per_chunk = 6 * C * dk * dv + C * C * (3 * dk + 2 * dv) + C ** 3 / 3
+    return per_chunk / C
+
+
+def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
+    """q, k, v, o once each, beta once, initial state read if given, final
+    state written."""
+    es = 2 if w.dtype == torch.bfloat16 else 4
+    th = w.tokens * w.H
+    b = th * (es * (2 * w.dk + 2 * w.dv) + 4)
+    st = w.n_seq * w.H * w.dk * w.dv * 4
+    if w.init_state:
+        b += st
+    if with_final:
+        b += st
+    return float(b)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---- clocks ------------------------------------------------------------------
+
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [n for bit, n in sorted(_REASONS.items()) if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---- distributed plumbing ----------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws: int, backend: str):
+    if ws > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, ws: int, device) -> float:
+    if ws <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ---- oracle timing (CPU baseline / reference arm) -----------------------------
+
+def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0):
+    """Runs the float64 oracle on tokens [0, tokens) of batch row b, all heads;
+    returns (seconds, threads)."""
+    import oracle
+    n_threads = os.cpu_count() or 1
+    sl = lambda t: t[b:b + 1, :tokens].contiguous()
+    s0 = None if x["initial_state"] is None else x["initial_state"][b:b + 1].contiguous()
+    t0 = time.perf_counter()
+    oracle.token_recurrence(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]), s0,
+                            n_threads=n_threads)
+    return time.perf_counter() - t0, min(n_threads, w.H)
+
+
+def run_reference(args, w: wl.Workload):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    x = wl.generate(w, seed=0)
+    sample = min(args.ref_tokens, w.T)
+    for i in range(args.warmup):
+        time_oracle(x, w, sample, i % w.B)
+    total = 0.0
+    threads = 1
+    for i in range(args.steps):
+        dt, threads = time_oracle(x, w, sample, i % w.B)
+        total += dt
+    ms = 1e3 * total / args.steps
+    value = sample / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk,
+                   "d_v": w.dv, "chunk": CHUNK,
+                   "sample": f"tokens [0, {sample}) of one batch row, all {w.H} heads, per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{sample} tokens x {w.H} heads per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- our arm -----------------------------------------------------------------
+
+def run_b200(args, w: wl.Workload):
+    import deltanet_chunkwise_delta_b200 as dn
+
+    ws, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(ws, "nccl")
+    dn.load()
+
+    x = wl.generate(w, seed=0)
+    g = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=w.dtype, device=device)
+    fs = torch.empty((w.n_seq, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        dn.deltanet_fwd(g["q"], g["k"], g["v"], g["beta"], g["initial_state"], g["cu_seqlens"],
+                        out=out, final_state=fs, stream=stream)
+
+    step()
+    if dn.get_error(stream) != 0:
+        raise RuntimeError("device reported an error")
+    G, s = dn.last_schedule()
+    launches_per_step = 1 if G == 1 else (3 if G > 1 else 4)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(ws)
+    torch.cuda.synchronize(device)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize(device)
+    barrier(ws)
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, ws, device)
+
+    tokens = w.tokens
+    value = ws * tokens / (ms / 1e3)
+    th = w.tokens * w.H
+    tflops = ws * th * flops_per_token_head(w.dk, w.dv) / (ms / 1e3) / 1e12
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    alg_bytes = algorithmic_bytes(w)
+    achieved = alg_bytes / (ms_local / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
+                "kernel": "k_boundary" if G == 1 else "whole step (summary + scan + boundary)",
+                "algorithmic_bytes_per_launch": alg_bytes}
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: None if t is None else t.pin_memory()
+        hx = {k: pin(v) for k, v in x.items()}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_fs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        d = {k: (torch.empty_like(v, device=device) if isinstance(v, torch.Tensor) else None)
+             for k, v in x.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hx.values() if v is not None)
+        d2h = h_out.numel() * h_out.element_size() + h_fs.numel() * h_fs.element_size()
+
+        def e2e_step():
+            for k, v in hx.items():
+                if v is not None:
+                    d[k].copy_(v, non_blocking=True)
+            dn.deltanet_fwd(d["q"], d["k"], d["v"], d["beta"], d["initial_state"],
+                            d["cu_seqlens"], out=out, final_state=fs, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            h_fs.copy_(fs, non_blocking=True)
+
+        n_e2e = max(3, min(args.steps, 50))
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier(ws)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        barrier(ws)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, ws, device)
+        e2e = {"value": ws * tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        sample = w.T if w.seqlens is None else min(w.T, 4096)
+        rows = w.B if w.seqlens is None else 1
+        total_s, threads = 0.0, 1
+        for b in range(rows):
+            dt, threads = time_oracle(x, w, sample, b)
+            total_s += dt
+        cpu = {"value": rows * sample / total_s, "unit": "tokens/s", "cores": threads,
+               "kind": "oracle",
+               "sample": f"{rows} x {sample} tokens x {w.H} heads (float64 token recurrence)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                   "chunk": CHUNK, "segments_per_chain": G, "chunks_per_segment": s,
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}"},
+        "tflops": tflops,
+        "tflops_unit": "algorithmic TFLOP/s (6Cd^2 + 5C^2d + C^3/3 per chunk-head)",
+        "roofline": roofline,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--config", default="layer_1p3b", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=128,
+                    help="reference arm: tokens of one batch row per step")
+    args = ap.parse_args(argv)
+    w = wl.WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_b200(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+"""ctypes binding of the C ABI in include/deltanet.h.
+
+Argument marshalling only: torch tensors are described as ``dn_tensor``
+structs (pointer, dtype, shape, strides in elements) and handed to the shared
+library.  Every step of the computation runs in the library's CUDA kernels;
+there is no other implementation to fall back to.  If the library is missing
+or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+DN_OK, DN_ERR_INVALID_ARG, DN_ERR_UNSUPPORTED, DN_ERR_ALIAS, DN_ERR_CUDA, \
+    DN_ERR_WORKSPACE, DN_ERR_SEQLENS, DN_ERR_TIMEOUT = range(8)
+DN_F32, DN_BF16, DN_I32 = 0, 1, 2
+
+EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "deltanet_status_string",
+            "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule")
+
+
+class DnTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class DeltaNetError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(path: Optional[str] = None):
+    """Load the shared library (built in-tree by ``build.py``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = path or _build.LIB
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"DeltaNet CUDA library not found at {path}; run "
+                "`python -m deltanet_chunkwise_delta_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER(DnTensor)
+        lib.deltanet_fwd.restype = ctypes.c_int
+        lib.deltanet_fwd.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
+        lib.deltanet_fwd_ex.restype = ctypes.c_int
+        lib.deltanet_fwd_ex.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p,
+                                        ctypes.c_int]
+        lib.deltanet_status_string.restype = ctypes.c_char_p
+        lib.deltanet_status_string.argtypes = [ctypes.c_int]
+        lib.deltanet_get_error.restype = ctypes.c_int
+        lib.deltanet_get_error.argtypes = [ctypes.c_void_p]
+        lib.deltanet_release_workspace.restype = None
+        lib.deltanet_release_workspace.argtypes = []
+        lib.deltanet_last_schedule.restype = None
+        lib.deltanet_last_schedule.argtypes = [ctypes.POINTER(ctypes.c_int),
+                                               ctypes.POINTER(ctypes.c_int)]
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().deltanet_status_string(int(status)).decode()
+
+
+_DT = {torch.float32: DN_F32, torch.bfloat16: DN_BF16, torch.int32: DN_I32}
+
+
+def describe(t: Optional[torch.Tensor]) -> Optional[DnTensor]:
+    """dn_tensor view of a tensor (strides in elements); None stays None."""
+    if t is None:
+        return None
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    if t.dim() > 4:
+        raise ValueError("at most 4 dimensions")
+    d = DnTensor()
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.dtype = _DT[t.dtype]
+    d.ndim = t.dim()
+    for i in range(4):
+        d.shape[i] = t.shape[i] if i < t.dim() else 0
+        d.stride[i] = t.stride(i) if i < t.dim() else 0
+    return d
+
+
+def _ref(d: Optional[DnTensor]):
+    return None if d is None else ctypes.byref(d)
+
+
+def call(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state, stream,
+         seg_chunks: int = 0) -> int:
+    """Raw call: returns the dn_status code (no exception)."""
+    lib = load()
+    ds = [describe(t) for t in (q, k, v, beta, initial_state, cu_seqlens, out, final_state)]
+    args = [_ref(x) for x in ds[:6]] + [int(chunk_size)] + [_ref(x) for x in ds[6:]]
+    if seg_chunks:
+        return lib.deltanet_fwd_ex(*args, stream, int(seg_chunks))
+    return lib.deltanet_fwd(*args, stream)
+
+
+def _stream_handle(device, stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.Tensor,
+                 initial_state: Optional[torch.Tensor] = None,
+                 cu_seqlens: Optional[torch.Tensor] = None, chunk_size: int = 64,
+                 out: Optional[torch.Tensor] = None,
+                 final_state: Optional[torch.Tensor] = None,
+                 output_final_state: bool = True, stream=None, seg_chunks: int = 0):
+    """DeltaNet forward on CUDA tensors through the C ABI.
+
+    Shapes: q, k [B, T, H, d_k]; v [B, T, H, d_v]; beta [B, T, H] fp32;
+    initial_state [N, H, d_k, d_v] fp32 or None; cu_seqlens int32 [N+1] or None.
+    Allocates ``out`` / ``final_state`` when not given.  Returns
+    (out, final_state or None).  Asynchronous on ``stream`` (default: torch's
+    current stream).
+    """
+    if not q.is_cuda:
+        raise ValueError("deltanet_fwd runs on CUDA tensors only")
+    B, T, H, _ = q.shape
+    dk, dv = q.shape[3], v.shape[3]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = call(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
+              _stream_handle(q.device, stream), seg_chunks)
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state
+
+
+def get_error(stream=None, device=None) -> int:
+    """Synchronise the stream and return (and clear) its device-side error flag."""
+    return load().deltanet_get_error(_stream_handle(device, stream))
+
+
+def release_workspace() -> None:
+    load().deltanet_release_workspace()
+
+
+def last_schedule():
+    g, s = ctypes.c_int(0), ctypes.c_int(0)
+    load().deltanet_last_schedule(ctypes.byref(g), ctypes.byref(s))
+    return g.value, s.value

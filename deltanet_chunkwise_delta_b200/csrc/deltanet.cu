@@ -1,0 +1,420 @@
+// Host side of the C ABI declared in include/deltanet.h: argument checks,
+// per-stream workspace, scheduling and kernel launches.  No computation of the
+// method happens on the host.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/deltanet.h"
+#include "dn_chain.cuh"
+#include "dn_common.cuh"
+#include "dn_sched.cuh"
+
+using namespace dn;
+
+namespace {
+
+thread_local int g_last_G = 0, g_last_s = 0;
+
+struct StreamWs {
+    int* flag = nullptr;  // [0] error flag
+    char* buf = nullptr;
+    size_t cap = 0;
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, StreamWs> g_ws;
+std::set<std::pair<int, const void*>> g_attr_done;
+std::map<int, int> g_dev_ok;     // device -> 1 ok, 0 unsupported
+std::map<int, int> g_dev_sms;
+
+int64_t elem_size(int32_t dt) { return dt == DN_F32 ? 4 : dt == DN_BF16 ? 2 : dt == DN_I32 ? 4 : 0; }
+
+bool shape_eq(const dn_tensor* t, int ndim, const int64_t* dims) {
+    if (!t || t->ndim != ndim) return false;
+    for (int i = 0; i < ndim; ++i)
+        if (t->shape[i] != dims[i]) return false;
+    return true;
+}
+
+int64_t numel(const dn_tensor* t) {
+    int64_t n = 1;
+    for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+    return n;
+}
+
+// Byte span [lo, hi) touched by a strided view (non-negative strides only).
+bool span(const dn_tensor* t, uintptr_t& lo, uintptr_t& hi) {
+    lo = hi = 0;
+    if (!t || numel(t) == 0) return true;
+    int64_t last = 0;
+    for (int i = 0; i < t->ndim; ++i) {
+        if (t->stride[i] < 0) return false;
+        last += (t->shape[i] - 1) * t->stride[i];
+    }
+    const int64_t es = elem_size(t->dtype);
+    lo = reinterpret_cast<uintptr_t>(t->data);
+    hi = lo + static_cast<uintptr_t>((last + 1) * es);
+    return true;
+}
+
+bool overlap(const dn_tensor* a, const dn_tensor* b) {
+    uintptr_t a0, a1, b0, b1;
+    span(a, a0, a1);
+    span(b, b0, b1);
+    if (a0 == a1 || b0 == b1) return false;
+    return a0 < b1 && b0 < a1;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// q/k/v/out: [B, T, H, d], stride[3] == 1, 16-byte aligned rows and strides.
+bool token_tensor_ok(const dn_tensor* t) {
+    if (t->stride[3] != 1) return false;
+    const int64_t es = elem_size(t->dtype);
+    if (numel(t) == 0) return true;
+    if (!t->data || !aligned16(t->data)) return false;
+    for (int i = 0; i < 3; ++i)
+        if (t->stride[i] < 0 || (t->stride[i] * es) % 16 != 0) return false;
+    return true;
+}
+
+bool state_tensor_ok(const dn_tensor* t, int64_t dv) {
+    if (t->dtype != DN_F32 || t->stride[3] != 1 || t->stride[2] != dv) return false;
+    if (numel(t) == 0) return true;
+    if (!t->data || !aligned16(t->data)) return false;
+    return t->stride[0] >= 0 && t->stride[1] >= 0 && (t->stride[0] * 4) % 16 == 0 &&
+           (t->stride[1] * 4) % 16 == 0;
+}
+
+dn_status device_check(int& dev, int& sms) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return DN_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev_ok.find(dev);
+    if (it == g_dev_ok.end()) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return DN_ERR_CUDA;
+        g_dev_ok[dev] = (major == 10 && minor == 0) ? 1 : 0;
+        g_dev_sms[dev] = n;
+        it = g_dev_ok.find(dev);
+    }
+    sms = g_dev_sms[dev];
+    return it->second ? DN_OK : DN_ERR_UNSUPPORTED;
+}
+
+template <typename K>
+dn_status set_smem(K* kernel, int dev, int bytes) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto key = std::make_pair(dev, reinterpret_cast<const void*>(kernel));
+    if (g_attr_done.count(key)) return DN_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return DN_ERR_CUDA;
+    g_attr_done.insert(key);
+    return DN_OK;
+}
+
+// Workspace of `bytes` for (dev, stream); grows stream-ordered.
+dn_status get_ws(int dev, cudaStream_t stream, size_t bytes, StreamWs& out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    StreamWs& w = g_ws[std::make_pair(dev, stream)];
+    if (!w.flag) {
+        if (cudaMalloc(&w.flag, 256) != cudaSuccess) {
+            w.flag = nullptr;
+            return DN_ERR_WORKSPACE;
+        }
+        if (cudaMemset(w.flag, 0, 256) != cudaSuccess) return DN_ERR_CUDA;
+    }
+    if (bytes > w.cap) {
+        if (w.buf) cudaFreeAsync(w.buf, stream);
+        w.buf = nullptr;
+        w.cap = 0;
+        size_t want = std::max(bytes, (size_t)1 << 20);
+        if (cudaMallocAsync(reinterpret_cast<void**>(&w.buf), want, stream) != cudaSuccess) {
+            w.buf = nullptr;
+            return DN_ERR_WORKSPACE;
+        }
+        w.cap = want;
+    }
+    out = w;
+    return DN_OK;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Dims {
+    int64_t B, T, H, dk, dv, N;
+    bool varlen;
+};
+
+template <typename E, int DK, int DV, int STAGES>
+dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
+                 const int* cu) {
+    using LC = ChainSmem<E, DK, DV, true, true, STAGES>;
+    using LH = ChainSmem<E, DK, DV, true, false, STAGES>;
+    using LP = ChainSmem<E, DK, DK, false, false, STAGES>;
+    const int smemC = LC::TOTAL;
+    const int smemA = LH::TOTAL > LP::TOTAL ? LH::TOTAL : LP::TOTAL;
+    const int smemS = (DK * (DK + 1) + DK * 16) * 4;
+    auto* kC = k_boundary<E, DK, DV, STAGES>;
+    auto* kA = k_summary<E, DK, DV, STAGES>;
+    auto* kS = k_scan<DK, DV>;
+    dn_status st;
+    if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
+    if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
+    if ((st = set_smem(kS, dev, smemS)) != DN_OK) return st;
+
+    const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
+    const int64_t chains = d.N * d.H;
+    CostModel model;
+    size_t bytes = 0;
+    int64_t slots = 0, nC = 0, nA = 0, nScan = 0;
+    int G = 1, s = 1;
+    if (!d.varlen) {
+        if (forced_s > 0) {
+            s = forced_s;
+        } else {
+            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots);
+            s = ch.s;
+        }
+        G = n_c_max > 0 ? (int)((n_c_max + s - 1) / s) : 1;
+        slots = chains * (G - 1);
+        if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
+        nC = chains * G;
+        nA = G >= 2 ? chains * (2 * G - 3) : 0;
+        nScan = G >= 2 ? chains : 0;
+    } else {
+        if (forced_s > 0) {
+            slots = d.H * ((n_c_max + d.N) / forced_s);
+            if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
+        } else {
+            slots = std::min<int64_t>(kAutoMaxSlots, d.H * (n_c_max + d.N));
+        }
+        nC = chains + slots;
+        nA = 2 * slots;
+        nScan = std::min<int64_t>(chains, slots);
+    }
+    // workspace layout
+    const size_t off_items = 256;
+    const size_t off_A = off_items + up256(nC * sizeof(Item) * (d.varlen ? 1 : 0));
+    const size_t off_S = off_A + up256(nA * sizeof(Item) * (d.varlen ? 1 : 0));
+    const size_t off_nc = off_S + up256(nScan * sizeof(Item) * (d.varlen ? 1 : 0));
+    const size_t off_order = off_nc + up256(d.varlen ? d.N * 4 : 0);
+    const size_t off_offs = off_order + up256(d.varlen ? d.N * 4 : 0);
+    const size_t off_P = off_offs + up256(d.varlen ? d.N * 16 : 0);
+    const size_t off_H = off_P + up256((size_t)slots * DK * DK * 4);
+    const size_t off_SS = off_H + up256((size_t)slots * DK * DV * 4);
+    bytes = off_SS + up256((size_t)slots * DK * DV * 4);
+    StreamWs ws;
+    if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
+    char* base = ws.buf;
+    p.err = ws.flag;
+    p.wsP = reinterpret_cast<float*>(base + off_P);
+    p.wsH = reinterpret_cast<float*>(base + off_H);
+    p.wsS = reinterpret_cast<float*>(base + off_SS);
+    Sched& sc = p.sched;
+    std::memset(&sc, 0, sizeof sc);
+    if (!d.varlen) {
+        sc.list = 0;
+        sc.B = (int)d.B;
+        sc.T = (int)d.T;
+        sc.H = (int)d.H;
+        sc.n_chunks = (int)n_c_max;
+        sc.G = G;
+        sc.s = s;
+        g_last_G = G;
+        g_last_s = s;
+    } else {
+        sc.list = 1;
+        sc.B = 1;
+        sc.T = (int)d.T;
+        sc.H = (int)d.H;
+        sc.itemsC = reinterpret_cast<const Item*>(base + off_items);
+        sc.itemsA = reinterpret_cast<const Item*>(base + off_A);
+        sc.itemsScan = reinterpret_cast<const Item*>(base + off_S);
+        sc.counts = reinterpret_cast<const int*>(base);
+        k_schedule<<<1, 1024, 0, stream>>>(
+            cu, (int)d.N, (int)d.T, (int)d.H, forced_s, forced_s > 0 ? kMaxSlots : kAutoMaxSlots,
+            sms, model, reinterpret_cast<Item*>(base + off_items),
+            reinterpret_cast<Item*>(base + off_A), reinterpret_cast<Item*>(base + off_S),
+            reinterpret_cast<int*>(base), reinterpret_cast<int*>(base + off_nc),
+            reinterpret_cast<int*>(base + off_order), reinterpret_cast<int4*>(base + off_offs),
+            ws.flag);
+        g_last_G = -1;
+        g_last_s = -1;
+    }
+    if (nA > 0) kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p);
+    if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
+    if (nC > 0) kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return DN_ERR_CUDA;
+    return DN_OK;
+}
+
+dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                   const dn_tensor* beta, const dn_tensor* s0, const dn_tensor* cu, int chunk,
+                   dn_tensor* out, dn_tensor* sT, void* stream_ptr, int forced_s) {
+    if (!q || !k || !v || !beta || !out) return DN_ERR_INVALID_ARG;
+    if (q->ndim != 4 || k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return DN_ERR_INVALID_ARG;
+    if (forced_s < 0) return DN_ERR_INVALID_ARG;
+    const int64_t B = q->shape[0], T = q->shape[1], H = q->shape[2], dk = q->shape[3];
+    const int64_t dv = v->shape[3];
+    if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1) return DN_ERR_INVALID_ARG;
+    const int64_t kd[4] = {B, T, H, dk}, vd[4] = {B, T, H, dv}, bd[3] = {B, T, H};
+    if (!shape_eq(k, 4, kd) || !shape_eq(v, 4, vd) || !shape_eq(out, 4, vd) ||
+        !shape_eq(beta, 3, bd))
+        return DN_ERR_INVALID_ARG;
+    const int32_t dt = q->dtype;
+    if ((dt != DN_BF16 && dt != DN_F32) || k->dtype != dt || v->dtype != dt || out->dtype != dt)
+        return DN_ERR_INVALID_ARG;
+    if (beta->dtype != DN_F32) return DN_ERR_INVALID_ARG;
+    if (!token_tensor_ok(q) || !token_tensor_ok(k) || !token_tensor_ok(v) || !token_tensor_ok(out))
+        return DN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (beta->stride[i] < 0) return DN_ERR_INVALID_ARG;
+    if (numel(beta) > 0 && (!beta->data || (reinterpret_cast<uintptr_t>(beta->data) & 3)))
+        return DN_ERR_INVALID_ARG;
+    if (B * T >= (int64_t(1) << 31) || H >= 65536) return DN_ERR_INVALID_ARG;
+
+    int64_t N = B;
+    const bool varlen = cu != nullptr;
+    if (varlen) {
+        if (cu->ndim != 1 || cu->dtype != DN_I32 || cu->shape[0] < 1 || cu->stride[0] != 1 ||
+            !cu->data || (reinterpret_cast<uintptr_t>(cu->data) & 3))
+            return DN_ERR_INVALID_ARG;
+        if (B != 1) return DN_ERR_INVALID_ARG;
+        N = cu->shape[0] - 1;
+        if (N >= (int64_t(1) << 24)) return DN_ERR_INVALID_ARG;
+    }
+    const int64_t sd[4] = {N, H, dk, dv};
+    if (s0 && (!shape_eq(s0, 4, sd) || !state_tensor_ok(s0, dv))) return DN_ERR_INVALID_ARG;
+    if (sT && (!shape_eq(sT, 4, sd) || !state_tensor_ok(sT, dv))) return DN_ERR_INVALID_ARG;
+
+    if (chunk != kChunk) return DN_ERR_UNSUPPORTED;
+    const bool bf16_ok = (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+    const bool f32_ok = dk == 64 && dv == 64;
+    if (dt == DN_BF16 ? !bf16_ok : !f32_ok) return DN_ERR_UNSUPPORTED;
+
+    // aliasing: outputs against inputs and each other
+    const dn_tensor* ins[6] = {q, k, v, beta, s0, cu};
+    for (const dn_tensor* o : {static_cast<const dn_tensor*>(out), static_cast<const dn_tensor*>(sT)}) {
+        if (!o) continue;
+        for (const dn_tensor* in : ins)
+            if (in && overlap(o, in)) return DN_ERR_ALIAS;
+    }
+    if (sT && overlap(out, sT)) return DN_ERR_ALIAS;
+
+    int dev = 0, sms = 0;
+    dn_status st = device_check(dev, sms);
+    if (st != DN_OK) return st;
+    if (N == 0) return DN_OK;
+
+    Params p;
+    std::memset(&p, 0, sizeof p);
+    p.q = q->data; p.k = k->data; p.v = v->data; p.o = out->data;
+    p.beta = static_cast<const float*>(beta->data);
+    p.s0 = s0 && numel(s0) ? static_cast<const float*>(s0->data) : nullptr;
+    p.sT = sT && numel(sT) ? static_cast<float*>(sT->data) : nullptr;
+    p.q_sb = q->stride[0]; p.q_st = q->stride[1]; p.q_sh = q->stride[2];
+    p.k_sb = k->stride[0]; p.k_st = k->stride[1]; p.k_sh = k->stride[2];
+    p.v_sb = v->stride[0]; p.v_st = v->stride[1]; p.v_sh = v->stride[2];
+    p.o_sb = out->stride[0]; p.o_st = out->stride[1]; p.o_sh = out->stride[2];
+    p.b_sb = beta->stride[0]; p.b_st = beta->stride[1]; p.b_sh = beta->stride[2];
+    if (s0) { p.s0_sn = s0->stride[0]; p.s0_sh = s0->stride[1]; }
+    if (sT) { p.sT_sn = sT->stride[0]; p.sT_sh = sT->stride[1]; }
+
+    Dims d{B, T, H, dk, dv, N, varlen};
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    const int* cup = varlen ? static_cast<const int*>(cu->data) : nullptr;
+    if (dt == DN_F32) return launch<float, 64, 64, 1>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 128 && dv == 128)
+        return launch<__nv_bfloat16, 128, 128, 2>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 128 && dv == 64)
+        return launch<__nv_bfloat16, 128, 64, 2>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 64 && dv == 128)
+        return launch<__nv_bfloat16, 64, 128, 2>(p, d, dev, sms, stream, forced_s, cup);
+    return launch<__nv_bfloat16, 64, 64, 2>(p, d, dev, sms, stream, forced_s, cup);
+}
+
+}  // namespace
+
+extern "C" {
+
+dn_status deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                       const dn_tensor* beta, const dn_tensor* initial_state,
+                       const dn_tensor* cu_seqlens, int chunk_size, dn_tensor* out,
+                       dn_tensor* final_state, void* stream) {
+    return fwd_impl(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, 0);
+}
+
+dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                          const dn_tensor* beta, const dn_tensor* initial_state,
+                          const dn_tensor* cu_seqlens, int chunk_size, dn_tensor* out,
+                          dn_tensor* final_state, void* stream, int seg_chunks) {
+    return fwd_impl(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, seg_chunks);
+}
+
+const char* deltanet_status_string(dn_status s) {
+    switch (s) {
+        case DN_OK: return "DN_OK";
+        case DN_ERR_INVALID_ARG: return "DN_ERR_INVALID_ARG: bad shape, dtype, stride, alignment or pointer";
+        case DN_ERR_UNSUPPORTED: return "DN_ERR_UNSUPPORTED: chunk size, head dims or device not supported";
+        case DN_ERR_ALIAS: return "DN_ERR_ALIAS: an output overlaps an input or another output";
+        case DN_ERR_CUDA: return "DN_ERR_CUDA: CUDA runtime or launch error";
+        case DN_ERR_WORKSPACE: return "DN_ERR_WORKSPACE: workspace allocation failed or limit exceeded";
+        case DN_ERR_SEQLENS: return "DN_ERR_SEQLENS: invalid cu_seqlens contents";
+        case DN_ERR_TIMEOUT: return "DN_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown dn_status";
+}
+
+dn_status deltanet_get_error(void* stream_ptr) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DN_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return DN_ERR_CUDA;
+    int* flag = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_ws.find(std::make_pair(dev, stream));
+        if (it == g_ws.end() || !it->second.flag) return DN_OK;
+        flag = it->second.flag;
+    }
+    int h = 0;
+    if (cudaMemcpy(&h, flag, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DN_ERR_CUDA;
+    if (h != 0 && cudaMemset(flag, 0, sizeof h) != cudaSuccess) return DN_ERR_CUDA;
+    if (h == kErrSeqlens) return DN_ERR_SEQLENS;
+    if (h == kErrTimeout) return DN_ERR_TIMEOUT;
+    return DN_OK;
+}
+
+void deltanet_release_workspace(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto& kv : g_ws) {
+        cudaSetDevice(kv.first.first);
+        cudaDeviceSynchronize();
+        if (kv.second.buf) cudaFree(kv.second.buf);
+        if (kv.second.flag) cudaFree(kv.second.flag);
+    }
+    g_ws.clear();
+    cudaSetDevice(cur);
+}
+
+void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment) {
+    if (segments_per_chain) *segments_per_chain = g_last_G;
+    if (chunks_per_segment) *chunks_per_segment = g_last_s;
+}
+
+}  // extern "C"

@@ -1,0 +1,452 @@
+// One CTA threads the chunk state through a run of chunks of one (sequence, head).
+//
+// Per chunk r ("Linear Attention, Visualized", DeltaNet, "Complete per-chunk
+// algorithm"), with B_r = diag(beta_r):
+//   L_r = (K_r K_r^T) o M_c^-           strict-lower Gram matrix
+//   (I + B_r L_r) T_r = B_r             UT triangular solve (blocked, fp32)
+//   W_r = T_r K_r,  U_r = T_r V_r        WY / UT factors
+//   Z_r = U_r - W_r S_r                  corrected writes
+//   O_r = Q_r S_r + (Q_r K_r^T o M_c) Z_r
+//   S_{r+1} = S_r + K_r^T Z_r
+// The same loop with other start states and without output produces the
+// segment maps used for context parallelism (see SegMode): the zero-start
+// local writes H (V present, S_0 = 0) and the transition product P (no V,
+// S_0 = I, so each chunk applies I - K_r^T W_r, subsection "Compact the
+// transition product with WY").
+//
+// The state stays in registers (fp32) for the whole run; W, U, Z, T and the
+// masked scores never leave shared memory.  Only q, k, v, beta are read and o
+// written per chunk.  Loads of chunk r+1 are issued before chunk r is computed.
+#pragma once
+
+#include "dn_common.cuh"
+#include "dn_warp_gemm.cuh"
+
+namespace dn {
+
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES>
+struct ChainSmem {
+    static constexpr int ES = sizeof(E);
+    static constexpr int Q_BYTES = kChunk * DK * ES;
+    static constexpr int K_BYTES = kChunk * DK * ES;
+    static constexpr int V_BYTES = kChunk * NX * ES;
+    static constexpr int SOLVE_LD = 65;  // fp32 solve tiles, padded against bank conflicts
+    static constexpr int SOLVE_BYTES = (2 * kChunk * SOLVE_LD + 3 * 256) * 4;
+    static constexpr int O_BYTES = HAS_Q ? kChunk * NX * ES : 0;
+    static constexpr int UNION_BYTES = SOLVE_BYTES > O_BYTES ? SOLVE_BYTES : O_BYTES;
+
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + (HAS_Q ? STAGES * Q_BYTES : 0);
+    static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
+    static constexpr int OFF_BETA = OFF_V + (HAS_V ? STAGES * V_BYTES : 0);
+    static constexpr int OFF_SOLVE = OFF_BETA + STAGES * kChunk * 4;
+    static constexpr int OFF_T = align_up(OFF_SOLVE + UNION_BYTES, 128);
+    static constexpr int OFF_W = OFF_T + kChunk * kChunk * ES;
+    static constexpr int OFF_X = OFF_W + kChunk * DK * ES;
+    static constexpr int OFF_Z = OFF_X + DK * NX * ES;
+    static constexpr int OFF_P = OFF_Z + kChunk * NX * ES;
+    static constexpr int TOTAL = OFF_P + (HAS_Q ? kChunk * kChunk * ES : 0);
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+                 "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src),
+                 "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+// Copy a 64-row tile (row stride `st` elements in global memory) into a
+// swizzled shared tile of width D; rows >= rows_valid are zero-filled.
+template <typename E, int D>
+__device__ __forceinline__ void load_tile(E* dst, const E* src, int64_t st, int rows_valid) {
+    constexpr int V = 16 / sizeof(E);
+    constexpr int CPR = D / V;
+    for (int idx = threadIdx.x; idx < kChunk * CPR; idx += kThreads) {
+        const int r = idx / CPR, c = idx % CPR;
+        const bool ok = r < rows_valid;
+        const E* s = ok ? src + r * st + c * V : src;
+        cp_async16(smem_addr(dst + Swz<E>::template off<D>(r, c * V)), s, ok ? 16 : 0);
+    }
+}
+
+template <typename E>
+__device__ __forceinline__ E to_e(float x);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_e<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ float to_e<float>(float x) {
+    return x;
+}
+
+// Blocked solve of (I + A) N = I for the strictly lower A (= B L, 64 x 64, fp32,
+// row stride 65), followed by T = N diag(beta) written to a swizzled tile.
+// Diagonal 16 x 16 blocks by forward substitution, one column per thread;
+// off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order of i - j.
+template <typename E>
+__device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
+                                         const float* beta, E* Ts) {
+    constexpr int LD = 65;
+    const int tid = threadIdx.x;
+    if (tid < 64) {
+        const int blk = tid >> 4, c = tid & 15;
+        const float* Ab = Af + (16 * blk) * LD + 16 * blk;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float a = (i == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) a = fmaf(-Ab[i * LD + j], x[j], a);
+            x[i] = a;
+        }
+        float* Nb = Nf + (16 * blk) * LD + 16 * blk;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Nb[i * LD + c] = x[i];
+    } else {
+        // zero the strictly upper blocks: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
+            const int p = e >> 8;
+            const int bi = p < 3 ? 0 : (p < 5 ? 1 : 2);
+            const int bj = p < 3 ? p + 1 : (p < 5 ? p - 1 : 3);
+            const int ri = (e >> 4) & 15, cj = e & 15;
+            Nf[(16 * bi + ri) * LD + 16 * bj + cj] = 0.f;
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int npairs = 4 - d;
+        for (int e = tid; e < npairs * 256; e += kThreads) {
+            const int p = e >> 8, i = d + p, j = p, ri = (e >> 4) & 15, cj = e & 15;
+            float acc = 0.f;
+            for (int kb = j; kb < i; ++kb) {
+                const float* Ar = Af + (16 * i + ri) * LD + 16 * kb;
+                const float* Nc = Nf + (16 * kb) * LD + 16 * j + cj;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc = fmaf(Ar[m], Nc[m * LD], acc);
+            }
+            Xt[p * 256 + ri * 16 + cj] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < npairs * 256; e += kThreads) {
+            const int p = e >> 8, i = d + p, j = p, ri = (e >> 4) & 15, cj = e & 15;
+            const float* Nr = Nf + (16 * i + ri) * LD + 16 * i;
+            float acc = 0.f;
+            for (int m = 0; m <= ri; ++m) acc = fmaf(Nr[m], Xt[p * 256 + m * 16 + cj], acc);
+            Nf[(16 * i + ri) * LD + 16 * j + cj] = -acc;
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+        const int i = e >> 6, j = e & 63;
+        const float val = j <= i ? Nf[i * LD + j] * beta[j] : 0.f;
+        Ts[Swz<E>::template off<kChunk>(i, j)] = to_e<E>(val);
+    }
+}
+
+// Runs one work item.  mode selects start state, output and destination.
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES>
+__device__ __forceinline__ void run_segment(const Params& p, const Item& it, int mode,
+                                            char* smem) {
+    using L = ChainSmem<E, DK, NX, HAS_V, HAS_Q, STAGES>;
+    using SW = Swz<E>;
+    constexpr int MT_S = DK / 64;  // 16-row tiles of the state per warp
+    constexpr int NT_X = NX / 16;  // 8-column tiles per warp (NX / 2 columns)
+    constexpr int NT_W = DK / 16;
+
+    E* Qs = reinterpret_cast<E*>(smem + L::OFF_Q);
+    E* Ks = reinterpret_cast<E*>(smem + L::OFF_K);
+    E* Vs = reinterpret_cast<E*>(smem + L::OFF_V);
+    float* betas = reinterpret_cast<float*>(smem + L::OFF_BETA);
+    float* Af = reinterpret_cast<float*>(smem + L::OFF_SOLVE);
+    float* Nf = Af + kChunk * L::SOLVE_LD;
+    float* Xt = Nf + kChunk * L::SOLVE_LD;
+    E* Os = reinterpret_cast<E*>(smem + L::OFF_SOLVE);  // aliases the solve tiles
+    E* Ts = reinterpret_cast<E*>(smem + L::OFF_T);
+    E* Ws = reinterpret_cast<E*>(smem + L::OFF_W);
+    E* Xb = reinterpret_cast<E*>(smem + L::OFF_X);
+    E* Zs = reinterpret_cast<E*>(smem + L::OFF_Z);
+    E* Ps = reinterpret_cast<E*>(smem + L::OFF_P);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int mt = warp & 3, nh = warp >> 2;
+    const int s_r0 = (DK / 4) * mt;
+    const int x_c0 = (NX / 2) * nh;
+
+    // ---- start state and destination
+    const float* x_in = nullptr;
+    float* x_out = nullptr;
+    bool identity = false;
+    const float* s0 = p.s0 ? p.s0 + it.seq * p.s0_sn + it.head * p.s0_sh : nullptr;
+    if (mode == kModeOut) {
+        x_in = it.g == 0 ? s0 : p.wsS + (int64_t)(it.slot + it.g - 1) * DK * NX;
+        if (it.g == it.G - 1 && p.sT) x_out = p.sT + it.seq * p.sT_sn + it.head * p.sT_sh;
+    } else if (mode == kModeEnd) {
+        x_in = s0;
+        x_out = p.wsH + (int64_t)it.slot * DK * NX;
+    } else if (mode == kModeH) {
+        x_out = p.wsH + (int64_t)(it.slot + it.g) * DK * NX;
+    } else {
+        identity = true;
+        x_out = p.wsP + (int64_t)(it.slot + it.g) * DK * NX;
+    }
+
+    float s[MT_S][NT_X][4];
+#pragma unroll
+    for (int m = 0; m < MT_S; ++m)
+#pragma unroll
+        for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = s_r0 + 16 * m + g8 + 8 * h;
+                const int c = x_c0 + 8 * nt + 2 * t4;
+                float2 v2 = make_float2(0.f, 0.f);
+                if (x_in) {
+                    v2 = *reinterpret_cast<const float2*>(x_in + r * NX + c);
+                } else if (identity) {
+                    v2.x = (r == c) ? 1.f : 0.f;
+                    v2.y = (r == c + 1) ? 1.f : 0.f;
+                }
+                s[m][nt][2 * h] = v2.x;
+                s[m][nt][2 * h + 1] = v2.y;
+            }
+
+    const E* qg = static_cast<const E*>(p.q) + it.b * p.q_sb + it.head * p.q_sh;
+    const E* kg = static_cast<const E*>(p.k) + it.b * p.k_sb + it.head * p.k_sh;
+    const E* vg = static_cast<const E*>(p.v) + it.b * p.v_sb + it.head * p.v_sh;
+    E* og = static_cast<E*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
+    const float* bg = p.beta + it.b * p.b_sb + it.head * p.b_sh;
+
+    const int ntok = it.tok1 - it.tok0;
+    const int nchunks = (ntok + kChunk - 1) / kChunk;
+
+    auto issue_load = [&](int r, int stg) {
+        const int t0 = it.tok0 + r * kChunk;
+        const int rows = min(kChunk, it.tok1 - t0);
+        if (HAS_Q) load_tile<E, DK>(Qs + stg * (L::Q_BYTES / L::ES), qg + t0 * p.q_st, p.q_st, rows);
+        load_tile<E, DK>(Ks + stg * (L::K_BYTES / L::ES), kg + t0 * p.k_st, p.k_st, rows);
+        if (HAS_V) load_tile<E, NX>(Vs + stg * (L::V_BYTES / L::ES), vg + t0 * p.v_st, p.v_st, rows);
+        if (tid < kChunk) {
+            const bool ok = tid < rows;
+            cp_async4(smem_addr(betas + stg * kChunk + tid), ok ? bg + (t0 + tid) * p.b_st : bg,
+                      ok ? 4 : 0);
+        }
+        cp_async_commit();
+    };
+
+    if (STAGES == 2 && nchunks > 0) issue_load(0, 0);
+
+#pragma unroll 1
+    for (int r = 0; r < nchunks; ++r) {
+        const int stg = STAGES == 2 ? (r & 1) : 0;
+        if (STAGES == 2) {
+            if (r + 1 < nchunks) {
+                issue_load(r + 1, stg ^ 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+        } else {
+            issue_load(r, 0);
+            cp_async_wait<0>();
+        }
+        const E* Qc = Qs + stg * (L::Q_BYTES / L::ES);
+        const E* Kc = Ks + stg * (L::K_BYTES / L::ES);
+        const E* Vc = Vs + stg * (L::V_BYTES / L::ES);
+        const float* bc = betas + stg * kChunk;
+
+        // (a) state -> operand copy
+#pragma unroll
+        for (int m = 0; m < MT_S; ++m) store_frag<NT_X, NX>(Xb, s_r0 + 16 * m, x_c0, s[m], 1.f);
+        __syncthreads();
+
+        // (b) A = B L (strict lower, fp32) and, with output, P = (Q K^T) o M_c
+        {
+            float acc[4][4];
+            zero_frag(acc);
+            warp_gemm<DK, 4, DK, false, DK, false>(acc, Kc, 16 * mt, Kc, 32 * nh);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int row = 16 * mt + g8 + 8 * (e >> 1);
+                    const int col = 32 * nh + 8 * nt + 2 * t4 + (e & 1);
+                    Af[row * L::SOLVE_LD + col] = col < row ? bc[row] * acc[nt][e] : 0.f;
+                }
+            if (HAS_Q) {
+                zero_frag(acc);
+                warp_gemm<DK, 4, DK, false, DK, false>(acc, Qc, 16 * mt, Kc, 32 * nh);
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int row = 16 * mt + g8 + 8 * (e >> 1);
+                        const int col = 32 * nh + 8 * nt + 2 * t4 + (e & 1);
+                        if (col > row) acc[nt][e] = 0.f;
+                    }
+                store_frag<4, kChunk>(Ps, 16 * mt, 32 * nh, acc, 1.f);
+            }
+        }
+        __syncthreads();
+
+        // (c) T = (I + B L)^{-1} B
+        ut_solve<E>(Af, Nf, Xt, bc, Ts);
+        __syncthreads();
+
+        // (d) -W = -T K (stored negated), U = T V (kept in registers as Z's start)
+        float z[NT_X][4];
+        zero_frag(z);
+        {
+            float w[NT_W][4];
+            zero_frag(w);
+            warp_gemm<kChunk, NT_W, kChunk, false, DK, true>(w, Ts, 16 * mt, Kc, nh * (DK / 2));
+            store_frag<NT_W, DK>(Ws, 16 * mt, nh * (DK / 2), w, -1.f);
+            if (HAS_V) warp_gemm<kChunk, NT_X, kChunk, false, NX, true>(z, Ts, 16 * mt, Vc, x_c0);
+        }
+        __syncthreads();
+
+        // (e) Z = U - W S ; O = Q S
+        warp_gemm<DK, NT_X, DK, false, NX, true>(z, Ws, 16 * mt, Xb, x_c0);
+        float o[NT_X][4];
+        if constexpr (HAS_Q) {
+            zero_frag(o);
+            warp_gemm<DK, NT_X, DK, false, NX, true>(o, Qc, 16 * mt, Xb, x_c0);
+        }
+        store_frag<NT_X, NX>(Zs, 16 * mt, x_c0, z, 1.f);
+        __syncthreads();
+
+        // (f) O += (Q K^T o M_c) Z
+        if constexpr (HAS_Q) {
+            warp_gemm<kChunk, NT_X, kChunk, false, NX, true>(o, Ps, 16 * mt, Zs, x_c0);
+            store_frag<NT_X, NX>(Os, 16 * mt, x_c0, o, 1.f);
+        }
+        // (g) S += K^T Z
+#pragma unroll
+        for (int m = 0; m < MT_S; ++m)
+            warp_gemm<kChunk, NT_X, DK, true, NX, true>(s[m], Kc, s_r0 + 16 * m, Zs, x_c0);
+        __syncthreads();
+
+        // (h) O tile -> global
+        if (HAS_Q) {
+            constexpr int V = 16 / sizeof(E);
+            constexpr int CPR = NX / V;
+            const int t0 = it.tok0 + r * kChunk;
+            const int rows = min(kChunk, it.tok1 - t0);
+            for (int idx = tid; idx < kChunk * CPR; idx += kThreads) {
+                const int rr = idx / CPR, c = idx % CPR;
+                if (rr < rows)
+                    *reinterpret_cast<int4*>(og + (t0 + rr) * p.o_st + c * V) =
+                        *reinterpret_cast<const int4*>(Os + SW::template off<NX>(rr, c * V));
+            }
+        }
+    }
+
+    if (x_out) {
+#pragma unroll
+        for (int m = 0; m < MT_S; ++m)
+#pragma unroll
+            for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = s_r0 + 16 * m + g8 + 8 * h;
+                    const int c = x_c0 + 8 * nt + 2 * t4;
+                    *reinterpret_cast<float2*>(x_out + r * NX + c) =
+                        make_float2(s[m][nt][2 * h], s[m][nt][2 * h + 1]);
+                }
+    }
+}
+
+template <typename E, int DK, int DV, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) k_boundary(Params p) {
+    extern __shared__ __align__(128) char smem[];
+    const int n = count_C(p.sched);
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const Item it = item_C(p.sched, i);
+        run_segment<E, DK, DV, true, true, STAGES>(p, it, kModeOut, smem);
+        __syncthreads();
+    }
+}
+
+template <typename E, int DK, int DV, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
+    extern __shared__ __align__(128) char smem[];
+    const int n = count_A(p.sched);
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        int mode;
+        const Item it = item_A(p.sched, i, mode);
+        if (mode == kModeP)
+            run_segment<E, DK, DK, false, false, STAGES>(p, it, mode, smem);
+        else
+            run_segment<E, DK, DV, true, false, STAGES>(p, it, mode, smem);
+        __syncthreads();
+    }
+}
+
+// Segment scan: start(g+1) = P_g start(g) + H_g, start(1) = end state of
+// segment 0.  fp32; one CTA per (chain, 16 columns of the state).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads) k_scan(Params p) {
+    extern __shared__ __align__(16) float fsm[];
+    constexpr int PLD = DK + 1;
+    constexpr int NCOL = 16;
+    constexpr int GROUPS = kThreads / DK;       // column groups
+    constexpr int CPT = NCOL / GROUPS;          // columns per thread
+    float* Pm = fsm;                            // DK x PLD
+    float* Sm = Pm + DK * PLD;                  // DK x NCOL
+    const int tid = threadIdx.x;
+    const int a = tid % DK, cg = tid / DK;
+    const int c0 = blockIdx.y * NCOL;
+    const int n = count_scan(p.sched);
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+        const Item it = item_scan(p.sched, i);
+        const float* E0 = p.wsH + (int64_t)it.slot * DK * DV;
+        float* out0 = p.wsS + (int64_t)it.slot * DK * DV;
+        for (int e = tid; e < DK * NCOL; e += kThreads) {
+            const int r = e / NCOL, c = e % NCOL;
+            const float x = E0[r * DV + c0 + c];
+            Sm[e] = x;
+            out0[r * DV + c0 + c] = x;
+        }
+        for (int g = 1; g + 1 < it.G; ++g) {
+            __syncthreads();
+            const float* Pg = p.wsP + (int64_t)(it.slot + g) * DK * DK;
+            for (int e = tid; e < DK * DK / 4; e += kThreads) {
+                const float4 x = reinterpret_cast<const float4*>(Pg)[e];
+                const int r = (4 * e) / DK, c = (4 * e) % DK;
+                float* d = Pm + r * PLD + c;
+                d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+            }
+            __syncthreads();
+            const float* Hg = p.wsH + (int64_t)(it.slot + g) * DK * DV;
+            float acc[CPT];
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) acc[j] = Hg[a * DV + c0 + cg * CPT + j];
+            for (int b = 0; b < DK; ++b) {
+                const float pab = Pm[a * PLD + b];
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) acc[j] = fmaf(pab, Sm[b * NCOL + cg * CPT + j], acc[j]);
+            }
+            __syncthreads();
+            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                Sm[a * NCOL + cg * CPT + j] = acc[j];
+                outg[a * DV + c0 + cg * CPT + j] = acc[j];
+            }
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace dn

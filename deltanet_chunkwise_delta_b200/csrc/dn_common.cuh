@@ -1,0 +1,137 @@
+// Shared definitions of the chunkwise DeltaNet kernels (sm_100a).
+//
+// Notation follows "Linear Attention, Visualized" (DeltaNet section), row-vector
+// convention: a chunk holds C = 64 tokens; K_r, Q_r are C x d_k, V_r is C x d_v;
+// the state S is d_k x d_v and is read as k S / q S.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace dn {
+
+constexpr int kChunk = 64;       // C
+constexpr int kThreads = 256;    // 8 warps per CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxSlots = 4096;  // segment-map slots (P, H, start state) per call
+constexpr int kAutoMaxSlots = 592;  // slots the automatic schedule may use (4 x 148)
+
+// Device error flag values (match dn_status).
+constexpr int kErrSeqlens = 6;
+constexpr int kErrTimeout = 7;
+
+// A unit of work: one run of whole chunks of one (sequence, head) chain.
+//   b       batch row holding the tokens (0 for packed varlen input)
+//   seq     sequence index n (state row)
+//   head    head index h
+//   tok0/1  token range [tok0, tok1) within batch row b
+//   g, G    segment index and segment count of the chain
+//   slot    first workspace slot of the chain (segments 0..G-2 use slot+g)
+//   mode    see SegMode
+struct Item {
+    int b, seq, head, tok0, tok1, g, G, slot;
+};
+
+enum SegMode : int {
+    kModeOut = 0,    // boundary pass with output: start state -> O, end state
+    kModeEnd = 1,    // first segment: end state from the true initial state (no output)
+    kModeH = 2,      // zero-start local writes H_g of a segment
+    kModeP = 3,      // transition product P_g of a segment (state is d_k x d_k, starts at I)
+};
+
+// How work items are enumerated.
+//  dense:  B x H chains of n_chunks chunks each, G segments of s chunks.
+//  list:   items written by the device scheduler (packed varlen input).
+struct Sched {
+    int list;           // 0 = dense, 1 = list
+    int B, T, H;        // dense shape
+    int n_chunks, G, s; // dense segmentation
+    const Item* itemsC;     // list: boundary-pass items
+    const Item* itemsA;     // list: summary items; Item.g carries mode in bits 16+
+    const Item* itemsScan;  // list: one per chain with G >= 2
+    const int* counts;      // list: [nC, nA, nScan]
+};
+
+struct Params {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    const float* beta;
+    const float* s0;     // may be null
+    float* sT;           // may be null
+    int64_t q_sb, q_st, q_sh;
+    int64_t k_sb, k_st, k_sh;
+    int64_t v_sb, v_st, v_sh;
+    int64_t o_sb, o_st, o_sh;
+    int64_t b_sb, b_st, b_sh;
+    int64_t s0_sn, s0_sh;
+    int64_t sT_sn, sT_sh;
+    float* wsP;          // [slots][d_k][d_k]
+    float* wsH;          // [slots][d_k][d_v]
+    float* wsS;          // [slots][d_k][d_v] start states of segments 1..G-1
+    int* err;            // device error flag
+    Sched sched;
+};
+
+// ---- schedule decoding --------------------------------------------------------
+
+__device__ __forceinline__ void dense_chain_item(const Sched& s, int chain, int g, Item& it) {
+    it.b = chain / s.H;
+    it.seq = it.b;
+    it.head = chain % s.H;
+    it.G = s.G;
+    it.g = g;
+    it.tok0 = g * s.s * kChunk;
+    int e = (g + 1) * s.s * kChunk;
+    it.tok1 = e < s.T ? e : s.T;
+    if (g == s.G - 1) it.tok1 = s.T;
+    it.slot = chain * (s.G - 1);
+}
+
+__device__ __forceinline__ int count_C(const Sched& s) {
+    return s.list ? s.counts[0] : s.B * s.H * s.G;
+}
+__device__ __forceinline__ int count_A(const Sched& s) {
+    return s.list ? s.counts[1] : (s.G >= 2 ? s.B * s.H * (2 * s.G - 3) : 0);
+}
+__device__ __forceinline__ int count_scan(const Sched& s) {
+    return s.list ? s.counts[2] : (s.G >= 2 ? s.B * s.H : 0);
+}
+
+__device__ __forceinline__ Item item_C(const Sched& s, int i) {
+    Item it;
+    if (s.list) return s.itemsC[i];
+    dense_chain_item(s, i / s.G, i % s.G, it);
+    return it;
+}
+
+// Summary items: per chain, [End(g=0), H(1), P(1), H(2), P(2), ..., H(G-2), P(G-2)].
+__device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
+    Item it;
+    if (s.list) {
+        it = s.itemsA[i];
+        mode = it.g >> 16;
+        it.g &= 0xffff;
+        return it;
+    }
+    const int per = 2 * s.G - 3;
+    const int chain = i / per, r = i % per;
+    if (r == 0) {
+        mode = kModeEnd;
+        dense_chain_item(s, chain, 0, it);
+    } else {
+        mode = ((r - 1) & 1) ? kModeP : kModeH;
+        dense_chain_item(s, chain, 1 + (r - 1) / 2, it);
+    }
+    return it;
+}
+
+__device__ __forceinline__ Item item_scan(const Sched& s, int i) {
+    Item it;
+    if (s.list) return s.itemsScan[i];
+    dense_chain_item(s, i, 0, it);
+    return it;
+}
+
+}  // namespace dn

@@ -1,0 +1,254 @@
+// Segmentation of (sequence, head) chains into runs of chunks.
+//
+// A chain of n_c chunks is cut into G = ceil(n_c / s) runs of s chunks (the
+// last one shorter).  Run 0 starts from the true initial state; the others need
+// the maps (P_g, H_g) of every run before them ("Context Parallelism for
+// DeltaNet", section 3: the chunk update is affine in the incoming state, so
+// runs compose).  Work per call:
+//   summary pass   run 0: end state; runs 1..G-2: H_g and P_g (two items)
+//   segment scan   start states of runs 1..G-1
+//   boundary pass  every run from its start state: outputs, final state
+// The run length s minimises a simple model of the call's duration:
+//   c * max(min(s, longest chain), chunk-heads / slots)      boundary pass
+// + a * max(s, summary chunk-heads / slots)                  summary pass
+// + scan * (G_max - 1)                                       segment scan
+// with costs per chunk relative to one boundary-pass chunk.
+#pragma once
+
+#include "dn_common.cuh"
+
+namespace dn {
+
+struct CostModel {
+    float c = 1.0f;      // boundary pass, per chunk
+    float a = 0.65f;     // summary pass, per chunk (no output, no Q)
+    float scan = 0.4f;   // one step of the segment scan
+};
+
+struct SegChoice {
+    int s;
+    float cost;
+};
+
+// Cost of run length s for `chains` chains of equal length n_c (dense input).
+__host__ __device__ inline float dense_cost(const CostModel& m, int chains, int n_c, int s,
+                                            int slots) {
+    const int G = n_c > 0 ? (n_c + s - 1) / s : 1;
+    const double work = (double)chains * n_c;
+    float tC = m.c * fmaxf((float)min(s, n_c), (float)(work / slots));
+    float tA = 0.f;
+    if (G >= 2) tA = m.a * fmaxf((float)s, (float)((double)chains * (2 * G - 3) * s / slots));
+    return tC + tA + m.scan * (G - 1);
+}
+
+inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots,
+                              int max_slots) {
+    SegChoice best{n_c > 0 ? n_c : 1, 3.0e38f};
+    if (n_c <= 0) return {1, 0.f};
+    for (int G = 1; G <= 256 && G <= n_c; ++G) {
+        const int s = (n_c + G - 1) / G;
+        const int Gs = (n_c + s - 1) / s;
+        if ((long long)chains * (Gs - 1) > max_slots) break;
+        const float cst = dense_cost(m, chains, n_c, s, slots);
+        if (cst < best.cost) best = {s, cst};
+    }
+    return best;
+}
+
+// Device scheduler for packed variable-length input (one CTA of 1024 threads).
+// Validates cu_seqlens, picks s (unless forced), orders sequences longest
+// first and writes the three item lists and their counts.
+// Scratch: nc[N], order[N], offs[N][4].
+__global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, int N, int T,
+                                                   int H, int forced_s, int max_slots,
+                                                   int slots, CostModel m, Item* itemsC,
+                                                   Item* itemsA, Item* itemsScan, int* counts,
+                                                   int* nc, int* order, int4* offs, int* err) {
+    __shared__ int s_err, s_lmax;
+    __shared__ unsigned long long s_total;
+    __shared__ float s_cost[64];
+    __shared__ int s_s;
+    __shared__ int4 s_warp[32];
+    __shared__ int4 s_carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        s_err = 0;
+        s_lmax = 0;
+        s_total = 0;
+        s_carry = make_int4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    if (N > 0 && tid == 0 && (cu[0] != 0 || cu[N] != T)) s_err = 1;
+    for (int n = tid; n < N; n += blockDim.x) {
+        const int a = cu[n], e = cu[n + 1];
+        if (e < a || a < 0 || e > T) atomicOr(&s_err, 1);
+        const int L = e > a ? e - a : 0;
+        const int c = (L + kChunk - 1) / kChunk;
+        nc[n] = c;
+        atomicMax(&s_lmax, c);
+        atomicAdd(&s_total, (unsigned long long)c);
+    }
+    __syncthreads();
+    if (s_err) {
+        if (tid == 0) {
+            counts[0] = counts[1] = counts[2] = 0;
+            atomicExch(err, kErrSeqlens);
+        }
+        return;
+    }
+    const int lmax = s_lmax;
+
+    // ---- run length
+    if (forced_s > 0) {
+        if (tid == 0) s_s = forced_s;
+    } else {
+        for (int k = warp; k < 64; k += 32) {
+            const int s = lmax > 0 ? (lmax + k) / (k + 1) : 1;
+            long long extra = 0, wA = 0;
+            int gmax = 1;
+            for (int n = lane; n < N; n += 32) {
+                const int c = nc[n];
+                const int G = c > 0 ? (c + s - 1) / s : 1;
+                extra += G - 1;
+                if (G >= 2) wA += 2 * G - 3;
+                gmax = max(gmax, G);
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                extra += __shfl_xor_sync(0xffffffffu, extra, o);
+                wA += __shfl_xor_sync(0xffffffffu, wA, o);
+                gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+            }
+            if (lane == 0) {
+                float cst = 3.0e38f;
+                if ((long long)H * extra <= max_slots) {
+                    const double work = (double)H * (double)s_total;
+                    cst = m.c * fmaxf((float)min(s, max(lmax, 1)), (float)(work / slots));
+                    if (wA > 0)
+                        cst += m.a * fmaxf((float)s, (float)((double)H * wA * s / slots));
+                    cst += m.scan * (gmax - 1);
+                }
+                s_cost[k] = cst;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int best = 0;
+            for (int k = 1; k < 64; ++k)
+                if (s_cost[k] < s_cost[best]) best = k;
+            s_s = lmax > 0 ? (lmax + best) / (best + 1) : 1;
+        }
+    }
+    __syncthreads();
+    const int s = s_s;
+
+    // ---- order sequences longest first (stable); identity order for very large N
+    for (int n = tid; n < N; n += blockDim.x) {
+        if (N <= 4096) {
+            const int c = nc[n];
+            int rank = 0;
+            for (int j = 0; j < N; ++j) {
+                const int cj = nc[j];
+                rank += (cj > c) || (cj == c && j < n);
+            }
+            order[rank] = n;
+        } else {
+            order[n] = n;
+        }
+    }
+    __syncthreads();
+
+    // ---- exclusive prefix sums over ordered sequences: (C items, A items, scan items, slots)
+    for (int base = 0; base < N; base += blockDim.x) {
+        const int pos = base + tid;
+        int4 v = make_int4(0, 0, 0, 0);
+        if (pos < N) {
+            const int c = nc[order[pos]];
+            const int G = c > 0 ? (c + s - 1) / s : 1;
+            v = make_int4(H * G, G >= 2 ? H * (2 * G - 3) : 0, G >= 2 ? H : 0, H * (G - 1));
+        }
+        int4 inc = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, inc.x, o);
+            const int y = __shfl_up_sync(0xffffffffu, inc.y, o);
+            const int z = __shfl_up_sync(0xffffffffu, inc.z, o);
+            const int w = __shfl_up_sync(0xffffffffu, inc.w, o);
+            if (lane >= o) { inc.x += x; inc.y += y; inc.z += z; inc.w += w; }
+        }
+        if (lane == 31) s_warp[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int4 t = s_warp[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, t.x, o);
+                const int y = __shfl_up_sync(0xffffffffu, t.y, o);
+                const int z = __shfl_up_sync(0xffffffffu, t.z, o);
+                const int w = __shfl_up_sync(0xffffffffu, t.w, o);
+                if (lane >= o) { t.x += x; t.y += y; t.z += z; t.w += w; }
+            }
+            s_warp[lane] = t;  // inclusive over warps
+        }
+        __syncthreads();
+        int4 before = s_carry;
+        if (warp > 0) {
+            const int4 pw = s_warp[warp - 1];
+            before.x += pw.x; before.y += pw.y; before.z += pw.z; before.w += pw.w;
+        }
+        if (pos < N)
+            offs[pos] = make_int4(before.x + inc.x - v.x, before.y + inc.y - v.y,
+                                  before.z + inc.z - v.z, before.w + inc.w - v.w);
+        __syncthreads();
+        if (tid == blockDim.x - 1) {
+            const int4 tot = s_warp[31];
+            s_carry = make_int4(s_carry.x + tot.x, s_carry.y + tot.y, s_carry.z + tot.z,
+                                s_carry.w + tot.w);
+        }
+        __syncthreads();
+    }
+
+    // ---- emit items
+    for (int pos = tid; pos < N; pos += blockDim.x) {
+        const int n = order[pos];
+        const int c = nc[n];
+        const int G = c > 0 ? (c + s - 1) / s : 1;
+        const int4 o = offs[pos];
+        const int a = cu[n], e = cu[n + 1];
+        for (int h = 0; h < H; ++h) {
+            const int slot = o.w + h * (G - 1);
+            for (int g = 0; g < G; ++g) {
+                Item it;
+                it.b = 0;
+                it.seq = n;
+                it.head = h;
+                it.tok0 = a + g * s * kChunk;
+                it.tok1 = (g == G - 1) ? e : min(e, a + (g + 1) * s * kChunk);
+                it.g = g;
+                it.G = G;
+                it.slot = slot;
+                itemsC[o.x + h * G + g] = it;
+                if (G >= 2 && g + 1 < G) {
+                    const int abase = o.y + h * (2 * G - 3);
+                    if (g == 0) {
+                        Item x = it;
+                        x.g = 0 | (kModeEnd << 16);
+                        itemsA[abase] = x;
+                    } else {
+                        Item x = it;
+                        x.g = g | (kModeH << 16);
+                        itemsA[abase + 1 + 2 * (g - 1)] = x;
+                        x.g = g | (kModeP << 16);
+                        itemsA[abase + 2 + 2 * (g - 1)] = x;
+                    }
+                }
+                if (G >= 2 && g == 0) itemsScan[o.z + h] = it;
+            }
+        }
+    }
+    if (tid == 0) {
+        // totals = carry after the last tile
+        counts[0] = s_carry.x;
+        counts[1] = s_carry.y;
+        counts[2] = s_carry.z;
+    }
+}
+
+}  // namespace dn

@@ -1,0 +1,131 @@
+/*
+ * deltanet.h -- C ABI of the B200 (sm_100a) chunkwise DeltaNet forward pass.
+ *
+ * The operation ("Linear Attention, Visualized", section "DeltaNet: correcting
+ * memory collisions"; "Context Parallelism for DeltaNet", section 2): for every
+ * sequence n and head h, starting from S = initial_state[n, h] (or zero),
+ *
+ *     vhat_t = k_t S,  u_t = beta_t (v_t - vhat_t),  S <- S + k_t^T u_t,  o_t = q_t S
+ *
+ * in the row-vector convention, S being d_k x d_v ("Recurrent form").  This is
+ * S_t = S_{t-1}(I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t with the
+ * state transposed.  The library evaluates it chunk by chunk (chunk C = 64)
+ * through the WY/UT factors of the "Complete per-chunk algorithm"
+ * (L = (K K^T) o M^-, (I + B L) T = B, W = T K, U = T V, Z = U - W S,
+ * O = Q S + (Q K^T o M) Z, S' = S + K^T Z), and splits each sequence's chain of
+ * chunk states across the GPU's SMs by composing the affine maps
+ * S_end = P S_start + H of runs of chunks ("One chunk as an affine recurrence";
+ * "Context Parallelism for DeltaNet", section 3).  No query scaling is applied.
+ *
+ * Tensors are passed as descriptors of device memory (dn_tensor).  Strides are
+ * in ELEMENTS.  Every call is asynchronous on the given CUDA stream.
+ */
+#ifndef DELTANET_H_
+#define DELTANET_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DN_OK = 0,
+    DN_ERR_INVALID_ARG = 1,   /* bad shape, dtype, stride, alignment or NULL pointer */
+    DN_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (chunk size,
+                                 head dims, device other than sm_100) */
+    DN_ERR_ALIAS = 3,         /* an output overlaps an input or another output */
+    DN_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+    DN_ERR_WORKSPACE = 5,     /* workspace allocation failed */
+    DN_ERR_SEQLENS = 6,       /* cu_seqlens content invalid (reported by deltanet_get_error) */
+    DN_ERR_TIMEOUT = 7        /* a bounded device-side wait gave up (reported by deltanet_get_error) */
+} dn_status;
+
+typedef enum { DN_F32 = 0, DN_BF16 = 1, DN_I32 = 2 } dn_dtype;
+
+/* A strided view of device memory.  shape/stride entries beyond ndim are ignored. */
+typedef struct {
+    void* data;
+    int32_t dtype;        /* dn_dtype */
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];    /* in elements */
+} dn_tensor;
+
+/*
+ * deltanet_fwd -- DeltaNet forward pass over a batch.
+ *
+ *   q, k          [B, T, H, d_k]   bf16 or fp32 (the same dtype for q, k, v, out)
+ *   v             [B, T, H, d_v]
+ *   beta          [B, T, H]        fp32, any finite values (the pages use 0 < beta <= 1)
+ *   initial_state [N, H, d_k, d_v] fp32, or NULL for zeros
+ *   cu_seqlens    int32 [N + 1] device array, or NULL.  With it, B must be 1 and
+ *                 sequence n covers tokens cu[n] .. cu[n+1]-1 (cu[0] = 0,
+ *                 cu[N] = T, non-decreasing; zero-length sequences allowed).
+ *                 Without it N = B and each batch row is one sequence.
+ *   chunk_size    must be 64 (others: DN_ERR_UNSUPPORTED)
+ *   out           [B, T, H, d_v], dtype of q; fully overwritten (bf16 rounded to
+ *                 nearest-even from the fp32 accumulator)
+ *   final_state   [N, H, d_k, d_v] fp32, or NULL (not produced)
+ *   stream        cudaStream_t (NULL = legacy default stream)
+ *
+ * Supported head dims: bf16 d_k, d_v in {64, 128}; fp32 d_k = d_v = 64.
+ * Layout rules: the last dimension of every tensor has stride 1; q/k/v/out base
+ * addresses and their B/T/H strides are multiples of 16 bytes; states have
+ * stride[3] = 1 and stride[2] = d_v, with 16-byte aligned N/H strides and base.
+ * The caller owns every buffer; the library only reads the inputs.  Any byte
+ * overlap between an output and an input or the other output returns
+ * DN_ERR_ALIAS (final_state may not alias initial_state).
+ *
+ * Returns DN_OK once all kernels are enqueued on `stream`.  Argument errors are
+ * reported synchronously and nothing is launched.  Errors found on the device
+ * (invalid cu_seqlens contents, a bounded wait that ran out) are recorded in a
+ * per-stream flag read by deltanet_get_error; in that case out/final_state are
+ * unspecified.  Reentrant: calls on different streams use separate workspaces.
+ */
+dn_status deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                       const dn_tensor* beta, const dn_tensor* initial_state,
+                       const dn_tensor* cu_seqlens, int chunk_size,
+                       dn_tensor* out, dn_tensor* final_state, void* stream);
+
+/*
+ * deltanet_fwd_ex -- deltanet_fwd with a scheduling override.
+ * seg_chunks > 0 forces every sequence to be split into runs of seg_chunks
+ * chunks (the last run of each sequence may be shorter), each run on its own
+ * CTA, composed through the segment maps; 0 lets the library choose.  The
+ * result is the same up to rounding for every value (the composition is
+ * exact), which the tests exercise.  Returns DN_ERR_WORKSPACE if the forced
+ * split needs more segment slots than the library's limit (4096).
+ */
+dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                          const dn_tensor* beta, const dn_tensor* initial_state,
+                          const dn_tensor* cu_seqlens, int chunk_size,
+                          dn_tensor* out, dn_tensor* final_state, void* stream,
+                          int seg_chunks);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* deltanet_status_string(dn_status status);
+
+/*
+ * deltanet_get_error -- synchronises `stream`, then returns and clears the
+ * device-side error flag of the calls made on it (DN_OK, DN_ERR_SEQLENS or
+ * DN_ERR_TIMEOUT), or DN_ERR_CUDA if the stream itself reports an error.
+ */
+dn_status deltanet_get_error(void* stream);
+
+/* Frees every cached workspace (synchronises the device first). */
+void deltanet_release_workspace(void);
+
+/*
+ * deltanet_last_schedule -- the segmentation chosen by the last successful
+ * call on this thread for dense (cu_seqlens == NULL) batches: segments per
+ * sequence-head chain and chunks per segment.  Varlen batches are scheduled on
+ * the device and report -1 for both.  For tests and benchmarks.
+ */
+void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTANET_H_ */

@@ -1,0 +1,133 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+declared in include/deltanet.h, and rejects bad arguments before touching a
+GPU (these calls never reach the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from deltanet_chunkwise_delta_b200 import _lib as L
+from deltanet_chunkwise_delta_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "deltanet.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(deltanet_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(L.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = L.status_string(code)
+        assert s.startswith("DN_")
+    assert "unknown" in L.status_string(99)
+
+
+def desc(shape, dtype=L.DN_BF16, data=0x10000, strides=None):
+    d = L.DnTensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if strides is None:
+        strides, acc = [], 1
+        for s in reversed(shape):
+            strides.insert(0, acc)
+            acc *= s
+    for i in range(4):
+        d.shape[i] = shape[i] if i < len(shape) else 0
+        d.stride[i] = strides[i] if i < len(shape) else 0
+    return d
+
+
+def call(lib, q, k, v, beta, s0=None, cu=None, chunk=64, out=None, sT=None):
+    r = lambda x: None if x is None else ctypes.byref(x)
+    return lib.deltanet_fwd(r(q), r(k), r(v), r(beta), r(s0), r(cu), chunk, r(out), r(sT), None)
+
+
+def good(B=2, T=100, H=3, dk=128, dv=64, dtype=L.DN_BF16):
+    base = 0x100000000
+    es = 2 if dtype == L.DN_BF16 else 4
+    q = desc([B, T, H, dk], dtype, base)
+    k = desc([B, T, H, dk], dtype, base + 1 * 2**28)
+    v = desc([B, T, H, dv], dtype, base + 2 * 2**28)
+    beta = desc([B, T, H], L.DN_F32, base + 3 * 2**28)
+    out = desc([B, T, H, dv], dtype, base + 4 * 2**28)
+    s0 = desc([B, H, dk, dv], L.DN_F32, base + 5 * 2**28)
+    sT = desc([B, H, dk, dv], L.DN_F32, base + 6 * 2**28)
+    return q, k, v, beta, s0, out, sT
+
+
+def test_rejects_null_and_bad_shapes(lib):
+    q, k, v, beta, s0, out, sT = good()
+    assert call(lib, None, k, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+    assert call(lib, q, k, v, beta, out=None) == L.DN_ERR_INVALID_ARG
+    kb = desc([2, 100, 3, 64], L.DN_BF16, 0x200000000)
+    assert call(lib, q, kb, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+    bb = desc([2, 100, 4], L.DN_F32, 0x300000000)
+    assert call(lib, q, k, v, bb, out=out) == L.DN_ERR_INVALID_ARG
+    s_bad = desc([2, 3, 64, 64], L.DN_F32, 0x500000000)
+    assert call(lib, q, k, v, beta, s0=s_bad, out=out) == L.DN_ERR_INVALID_ARG
+
+
+def test_rejects_dtype_stride_alignment(lib):
+    q, k, v, beta, s0, out, sT = good()
+    kf = good(dtype=L.DN_F32)[1]
+    assert call(lib, q, kf, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+    bb = good()[3]
+    bb.dtype = L.DN_BF16
+    assert call(lib, q, k, v, bb, out=out) == L.DN_ERR_INVALID_ARG
+    qs = good()[0]
+    qs.stride[3] = 2
+    assert call(lib, qs, k, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+    qa = good()[0]
+    qa.data = qa.data + 2
+    assert call(lib, qa, k, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+    qh = good()[0]
+    qh.stride[2] = 129            # 258-byte head stride: not a multiple of 16
+    assert call(lib, qh, k, v, beta, out=out) == L.DN_ERR_INVALID_ARG
+
+
+def test_rejects_unsupported(lib):
+    q, k, v, beta, s0, out, sT = good()
+    assert call(lib, q, k, v, beta, out=out, chunk=32) == L.DN_ERR_UNSUPPORTED
+    q2, k2, v2, b2, _, o2, _ = good(dk=96)
+    assert call(lib, q2, k2, v2, b2, out=o2) == L.DN_ERR_UNSUPPORTED
+    q3, k3, v3, b3, _, o3, _ = good(dk=128, dv=128, dtype=L.DN_F32)
+    assert call(lib, q3, k3, v3, b3, out=o3) == L.DN_ERR_UNSUPPORTED
+
+
+def test_rejects_aliasing(lib):
+    q, k, v, beta, s0, out, sT = good()
+    o_on_q = desc([2, 100, 3, 64], L.DN_BF16, q.data + 4096)
+    assert call(lib, q, k, v, beta, out=o_on_q) == L.DN_ERR_ALIAS
+    same = desc([2, 3, 128, 64], L.DN_F32, s0.data)
+    assert call(lib, q, k, v, beta, s0=s0, out=out, sT=same) == L.DN_ERR_ALIAS
+    sT_on_out = desc([2, 3, 128, 64], L.DN_F32, out.data)
+    assert call(lib, q, k, v, beta, out=out, sT=sT_on_out) == L.DN_ERR_ALIAS
+
+
+def test_rejects_bad_varlen_descriptors(lib):
+    q, k, v, beta, s0, out, sT = good()          # B = 2
+    cu = desc([3], L.DN_I32, 0x700000000)
+    assert call(lib, q, k, v, beta, cu=cu, out=out) == L.DN_ERR_INVALID_ARG
+    q1, k1, v1, b1, _, o1, _ = good(B=1)
+    cu_f = desc([3], L.DN_F32, 0x700000000)
+    assert call(lib, q1, k1, v1, b1, cu=cu_f, out=o1) == L.DN_ERR_INVALID_ARG
+    s_wrong_n = desc([1, 3, 128, 64], L.DN_F32, 0x500000000)   # N = 2 from cu
+    assert call(lib, q1, k1, v1, b1, s0=s_wrong_n, cu=cu, out=o1) == L.DN_ERR_INVALID_ARG
