@@ -9,12 +9,14 @@
 #include <map>
 #include <mutex>
 #include <set>
+#include <type_traits>
 #include <utility>
 
 #include "../../include/deltanet.h"
 #include "dn_chain.cuh"
 #include "dn_common.cuh"
 #include "dn_sched.cuh"
+#include "dn_tc.cuh"
 
 using namespace dn;
 
@@ -151,6 +153,43 @@ dn_status get_ws(int dev, cudaStream_t stream, size_t bytes, StreamWs& out) {
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// TMA map of a bf16 [B, T, H, 128] tensor (element strides sb, st, sh): boxes of
+// 64 tokens x 64 channels of one head, 128-byte swizzle, zero fill past T.
+dn_status make_token_map(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t H,
+                         int64_t sb, int64_t st, int64_t sh) {
+    std::memset(m, 0, sizeof *m);
+    if (B * T == 0) return DN_OK;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return DN_ERR_CUDA;
+    cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)sh * 2, (cuuint64_t)st * 2, (cuuint64_t)(sb > 0 ? sb : T * st) * 2};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DN_OK : DN_ERR_UNSUPPORTED;
+}
+
 struct Dims {
     int64_t B, T, H, dk, dv, N;
     bool varlen;
@@ -159,6 +198,8 @@ struct Dims {
 template <typename E, int DK, int DV, int STAGES>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
+    // bf16 with d_k = d_v = 128 runs on the tensor-core (tcgen05) chain kernel
+    constexpr bool kTc = std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
     using LC = ChainSmem<E, DK, DV, true, true, STAGES>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES>;
@@ -168,10 +209,24 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kC = k_boundary<E, DK, DV, STAGES>;
     auto* kA = k_summary<E, DK, DV, STAGES>;
     auto* kS = k_scan<DK, DV>;
+    auto* kCt = tc::k_tc_chain<true>;
+    auto* kAt = tc::k_tc_chain<false>;
     dn_status st;
-    if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
-    if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
+    if (kTc) {
+        if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
+        if ((st = set_smem(kAt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
+    } else {
+        if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
+        if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
+    }
     if ((st = set_smem(kS, dev, smemS)) != DN_OK) return st;
+    CUtensorMap tq, tk, tv;
+    if (kTc) {
+        const int64_t Bq = d.varlen ? 1 : d.B;
+        if ((st = make_token_map(&tq, p.q, Bq, d.T, d.H, p.q_sb, p.q_st, p.q_sh)) != DN_OK) return st;
+        if ((st = make_token_map(&tk, p.k, Bq, d.T, d.H, p.k_sb, p.k_st, p.k_sh)) != DN_OK) return st;
+        if ((st = make_token_map(&tv, p.v, Bq, d.T, d.H, p.v_sb, p.v_st, p.v_sh)) != DN_OK) return st;
+    }
 
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
     const int64_t chains = d.N * d.H;
@@ -252,9 +307,15 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         g_last_G = -1;
         g_last_s = -1;
     }
-    if (nA > 0) kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p);
-    if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
-    if (nC > 0) kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p);
+    if (kTc) {
+        if (nA > 0) kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
+        if (nC > 0) kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    } else {
+        if (nA > 0) kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p);
+        if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
+        if (nC > 0) kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p);
+    }
     if (cudaGetLastError() != cudaSuccess) return DN_ERR_CUDA;
     return DN_OK;
 }
