@@ -15,6 +15,7 @@
 #include "../../include/deltanet.h"
 #include "dn_chain.cuh"
 #include "dn_common.cuh"
+#include "dn_prep.cuh"
 #include "dn_sched.cuh"
 #include "dn_tc.cuh"
 
@@ -211,10 +212,13 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kS = k_scan<DK, DV>;
     auto* kCt = tc::k_tc_chain<true>;
     auto* kAt = tc::k_tc_chain<false>;
+    auto* kPrep = k_ut_prep<128>;
+    constexpr int smemPrep = PrepSmem<128>::TOTAL;
     dn_status st;
     if (kTc) {
         if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
         if ((st = set_smem(kAt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
+        if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
     } else {
         if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
         if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
@@ -265,10 +269,14 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     const size_t off_nc = off_S + up256(nScan * sizeof(Item) * (d.varlen ? 1 : 0));
     const size_t off_order = off_nc + up256(d.varlen ? d.N * 4 : 0);
     const size_t off_offs = off_order + up256(d.varlen ? d.N * 4 : 0);
-    const size_t off_P = off_offs + up256(d.varlen ? d.N * 16 : 0);
+    const size_t off_cum = off_offs + up256(d.varlen ? d.N * 16 : 0);
+    const size_t off_P = off_cum + up256(d.varlen ? (d.N + 1) * 4 : 0);
     const size_t off_H = off_P + up256((size_t)slots * DK * DK * 4);
     const size_t off_SS = off_H + up256((size_t)slots * DK * DV * 4);
-    bytes = off_SS + up256((size_t)slots * DK * DV * 4);
+    // UT factors of every (chunk, head): chunks <= ceil(T / C) per row (+1 per sequence)
+    const int64_t chunk_ub = d.varlen ? n_c_max + d.N : d.B * n_c_max;
+    const size_t off_T = off_SS + up256((size_t)slots * DK * DV * 4);
+    bytes = off_T + (kTc ? (size_t)chunk_ub * d.H * 8192 : 0);
     StreamWs ws;
     if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
     char* base = ws.buf;
@@ -276,6 +284,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     p.wsP = reinterpret_cast<float*>(base + off_P);
     p.wsH = reinterpret_cast<float*>(base + off_H);
     p.wsS = reinterpret_cast<float*>(base + off_SS);
+    p.wsT = reinterpret_cast<uint8_t*>(base + off_T);
     Sched& sc = p.sched;
     std::memset(&sc, 0, sizeof sc);
     if (!d.varlen) {
@@ -297,17 +306,25 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         sc.itemsA = reinterpret_cast<const Item*>(base + off_A);
         sc.itemsScan = reinterpret_cast<const Item*>(base + off_S);
         sc.counts = reinterpret_cast<const int*>(base);
+        sc.cumchunks = reinterpret_cast<const int*>(base + off_cum);
+        sc.cu = cu;
+        sc.N = (int)d.N;
         k_schedule<<<1, 1024, 0, stream>>>(
             cu, (int)d.N, (int)d.T, (int)d.H, forced_s, forced_s > 0 ? kMaxSlots : kAutoMaxSlots,
             sms, model, reinterpret_cast<Item*>(base + off_items),
             reinterpret_cast<Item*>(base + off_A), reinterpret_cast<Item*>(base + off_S),
             reinterpret_cast<int*>(base), reinterpret_cast<int*>(base + off_nc),
             reinterpret_cast<int*>(base + off_order), reinterpret_cast<int4*>(base + off_offs),
-            ws.flag);
+            reinterpret_cast<int*>(base + off_cum), ws.flag);
         g_last_G = -1;
         g_last_s = -1;
     }
     if (kTc) {
+        const int64_t units = chunk_ub * d.H;
+        if (units > 0) {
+            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * 8);
+            kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(p);
+        }
         if (nA > 0) kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
         if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
         if (nC > 0) kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -472,6 +489,12 @@ void deltanet_release_workspace(void) {
     g_ws.clear();
     cudaSetDevice(cur);
 }
+
+#ifdef DN_TRACE
+int dn_trace_copy(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, tc::g_dn_trace, sizeof(tc::g_dn_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment) {
     if (segments_per_chain) *segments_per_chain = g_last_G;

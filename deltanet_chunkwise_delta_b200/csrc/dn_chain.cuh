@@ -66,11 +66,11 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // Copy a 64-row tile (row stride `st` elements in global memory) into a
 // swizzled shared tile of width D; rows >= rows_valid are zero-filled.
-template <typename E, int D>
+template <typename E, int D, int NT = kThreads>
 __device__ __forceinline__ void load_tile(E* dst, const E* src, int64_t st, int rows_valid) {
     constexpr int V = 16 / sizeof(E);
     constexpr int CPR = D / V;
-    for (int idx = threadIdx.x; idx < kChunk * CPR; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < kChunk * CPR; idx += NT) {
         const int r = idx / CPR, c = idx % CPR;
         const bool ok = r < rows_valid;
         const E* s = ok ? src + r * st + c * V : src;
@@ -93,7 +93,7 @@ __device__ __forceinline__ float to_e<float>(float x) {
 // row stride 65), followed by T = N diag(beta) written to a swizzled tile.
 // Diagonal 16 x 16 blocks by forward substitution, one column per thread;
 // off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order of i - j.
-template <typename E>
+template <typename E, int NT = kThreads>
 __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
                                          const float* beta, E* Ts) {
     constexpr int LD = 65;
@@ -114,7 +114,7 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
         for (int i = 0; i < 16; ++i) Nb[i * LD + c] = x[i];
     } else {
         // zero the strictly upper blocks: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
             const int p = e >> 8;
             const int bi = p < 3 ? 0 : (p < 5 ? 1 : 2);
             const int bj = p < 3 ? p + 1 : (p < 5 ? p - 1 : 3);
@@ -126,7 +126,7 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
 #pragma unroll 1
     for (int d = 1; d < 4; ++d) {
         const int npairs = 4 - d;
-        for (int e = tid; e < npairs * 256; e += kThreads) {
+        for (int e = tid; e < npairs * 256; e += NT) {
             const int p = e >> 8, i = d + p, j = p, ri = (e >> 4) & 15, cj = e & 15;
             float acc = 0.f;
             for (int kb = j; kb < i; ++kb) {
@@ -138,7 +138,7 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
             Xt[p * 256 + ri * 16 + cj] = acc;
         }
         __syncthreads();
-        for (int e = tid; e < npairs * 256; e += kThreads) {
+        for (int e = tid; e < npairs * 256; e += NT) {
             const int p = e >> 8, i = d + p, j = p, ri = (e >> 4) & 15, cj = e & 15;
             const float* Nr = Nf + (16 * i + ri) * LD + 16 * i;
             float acc = 0.f;
@@ -147,7 +147,7 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
         }
         __syncthreads();
     }
-    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+    for (int e = tid; e < kChunk * kChunk; e += NT) {
         const int i = e >> 6, j = e & 63;
         const float val = j <= i ? Nf[i * LD + j] * beta[j] : 0.f;
         Ts[Swz<E>::template off<kChunk>(i, j)] = to_e<E>(val);

@@ -27,9 +27,10 @@ constexpr int kErrTimeout = 7;
 //   tok0/1  token range [tok0, tok1) within batch row b
 //   g, G    segment index and segment count of the chain
 //   slot    first workspace slot of the chain (segments 0..G-2 use slot+g)
-//   mode    see SegMode
+//   cbase   global index of the run's first chunk (chunks are numbered per
+//           sequence in order, all heads sharing one number)
 struct Item {
-    int b, seq, head, tok0, tok1, g, G, slot;
+    int b, seq, head, tok0, tok1, g, G, slot, cbase;
 };
 
 enum SegMode : int {
@@ -49,7 +50,10 @@ struct Sched {
     const Item* itemsC;     // list: boundary-pass items
     const Item* itemsA;     // list: summary items; Item.g carries mode in bits 16+
     const Item* itemsScan;  // list: one per chain with G >= 2
-    const int* counts;      // list: [nC, nA, nScan]
+    const int* counts;      // list: [nC, nA, nScan, total chunks]
+    const int* cumchunks;   // list: [N + 1] first global chunk index of each sequence
+    const int* cu;          // list: cu_seqlens [N + 1]
+    int N;                  // list: number of sequences
 };
 
 struct Params {
@@ -70,6 +74,7 @@ struct Params {
     float* wsP;          // [slots][d_k][d_k]
     float* wsH;          // [slots][d_k][d_v]
     float* wsS;          // [slots][d_k][d_v] start states of segments 1..G-1
+    uint8_t* wsT;        // [chunks * H] UT factors T (bf16 64 x 64, 128-byte swizzled rows)
     int* err;            // device error flag
     Sched sched;
 };
@@ -87,6 +92,7 @@ __device__ __forceinline__ void dense_chain_item(const Sched& s, int chain, int 
     it.tok1 = e < s.T ? e : s.T;
     if (g == s.G - 1) it.tok1 = s.T;
     it.slot = chain * (s.G - 1);
+    it.cbase = it.b * s.n_chunks + g * s.s;
 }
 
 __device__ __forceinline__ int count_C(const Sched& s) {
@@ -125,6 +131,30 @@ __device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
         dense_chain_item(s, chain, 1 + (r - 1) / 2, it);
     }
     return it;
+}
+
+// Chunk-head units of the UT pre-pass: (global chunk, head).
+__device__ __forceinline__ int count_chunks(const Sched& s) {
+    return s.list ? s.counts[3] : s.B * s.n_chunks;
+}
+
+// Token range and batch row of global chunk `id`.
+__device__ __forceinline__ void chunk_range(const Sched& s, int id, int& b, int& t0, int& t1) {
+    if (!s.list) {
+        b = id / s.n_chunks;
+        t0 = (id % s.n_chunks) * kChunk;
+        t1 = min(s.T, t0 + kChunk);
+        return;
+    }
+    int lo = 0, hi = s.N;  // largest n with cumchunks[n] <= id
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s.cumchunks[mid] <= id) lo = mid;
+        else hi = mid;
+    }
+    b = 0;
+    t0 = s.cu[lo] + (id - s.cumchunks[lo]) * kChunk;
+    t1 = min(s.cu[lo + 1], t0 + kChunk);
 }
 
 __device__ __forceinline__ Item item_scan(const Sched& s, int i) {

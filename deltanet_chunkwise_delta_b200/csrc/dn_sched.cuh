@@ -58,12 +58,15 @@ inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots
 // Device scheduler for packed variable-length input (one CTA of 1024 threads).
 // Validates cu_seqlens, picks s (unless forced), orders sequences longest
 // first and writes the three item lists and their counts.
+// Also numbers the chunks of all sequences in input order (cumchunks[N + 1],
+// counts[3] = total) for the UT pre-pass.
 // Scratch: nc[N], order[N], offs[N][4].
 __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, int N, int T,
                                                    int H, int forced_s, int max_slots,
                                                    int slots, CostModel m, Item* itemsC,
                                                    Item* itemsA, Item* itemsScan, int* counts,
-                                                   int* nc, int* order, int4* offs, int* err) {
+                                                   int* nc, int* order, int4* offs, int* cumchunks,
+                                                   int* err) {
     __shared__ int s_err, s_lmax;
     __shared__ unsigned long long s_total;
     __shared__ float s_cost[64];
@@ -91,12 +94,45 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
     __syncthreads();
     if (s_err) {
         if (tid == 0) {
-            counts[0] = counts[1] = counts[2] = 0;
+            counts[0] = counts[1] = counts[2] = counts[3] = 0;
             atomicExch(err, kErrSeqlens);
         }
         return;
     }
     const int lmax = s_lmax;
+
+    // ---- cumchunks: exclusive prefix of nc in input order
+    for (int base = 0; base < N; base += blockDim.x) {
+        const int pos = base + tid;
+        const int v = pos < N ? nc[pos] : 0;
+        int inc = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += x;
+        }
+        if (lane == 31) s_warp[warp].x = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int t = s_warp[lane].x;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += x;
+            }
+            s_warp[lane].x = t;
+        }
+        __syncthreads();
+        const int before = s_carry.x + (warp > 0 ? s_warp[warp - 1].x : 0);
+        if (pos < N) cumchunks[pos] = before + inc - v;
+        __syncthreads();
+        if (tid == blockDim.x - 1) s_carry.x += s_warp[31].x;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        cumchunks[N] = s_carry.x;
+        counts[3] = s_carry.x;
+        s_carry.x = 0;
+    }
+    __syncthreads();
 
     // ---- run length
     if (forced_s > 0) {
@@ -224,6 +260,7 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
                 it.g = g;
                 it.G = G;
                 it.slot = slot;
+                it.cbase = cumchunks[n] + g * s;
                 itemsC[o.x + h * G + g] = it;
                 if (G >= 2 && g + 1 < G) {
                     const int abase = o.y + h * (2 * G - 3);
