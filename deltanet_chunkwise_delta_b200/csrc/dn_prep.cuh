@@ -33,8 +33,9 @@ constexpr int kBlkFloats = 16 * kBlkLd;
 template <int DK>
 struct PrepSmem {
     static constexpr int K_BYTES = kChunk * DK * 2;
-    static constexpr int OFF_A = K_BYTES;
-    static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;
+    static constexpr int A_BYTES = 10 * kBlkFloats * 4;
+    static constexpr int OFF_A = 0;  // the A blocks replace K once the Gram matrix is in registers
+    static constexpr int OFF_N = (K_BYTES > A_BYTES ? K_BYTES : A_BYTES);
     static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;
     static constexpr int OFF_BETA = OFF_X + 4 * kBlkFloats * 4;
     static constexpr int TOTAL = OFF_BETA + kChunk * 4;
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_ut_prep(Params p) {
             float acc[8][4];
             zero_frag(acc);
             warp_gemm<DK, 8, DK, false, DK, false>(acc, Ks, 16 * warp, Ks, 0);
+            __syncthreads();  // K is no longer read: its space now holds A
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const int bj = nt >> 1;
