@@ -22,7 +22,8 @@ DN_OK, DN_ERR_INVALID_ARG, DN_ERR_UNSUPPORTED, DN_ERR_ALIAS, DN_ERR_CUDA, \
 DN_F32, DN_BF16, DN_I32 = 0, 1, 2
 
 EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "deltanet_status_string",
-            "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule")
+            "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
+            "deltanet_fwd_noalloc")
 
 
 class DnTensor(ctypes.Structure):
@@ -62,6 +63,8 @@ def load(path: Optional[str] = None):
         lib.deltanet_fwd_ex.restype = ctypes.c_int
         lib.deltanet_fwd_ex.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p,
                                         ctypes.c_int]
+        lib.deltanet_fwd_noalloc.restype = ctypes.c_int
+        lib.deltanet_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
         lib.deltanet_status_string.restype = ctypes.c_char_p
         lib.deltanet_status_string.argtypes = [ctypes.c_int]
         lib.deltanet_get_error.restype = ctypes.c_int
@@ -146,6 +149,27 @@ def deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.
         final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     st = call(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
               _stream_handle(q.device, stream), seg_chunks)
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state
+
+
+def deltanet_fwd_noalloc(q, k, v, beta, initial_state=None, chunk_size: int = 64, out=None,
+                         final_state=None, stream=None):
+    """The forward pass through the entry point that allocates no device memory
+    (for callers that cannot allocate; see include/deltanet.h).  Dense bf16
+    batches with d_k = d_v = 128 only.  ``out`` and ``final_state`` are allocated
+    here with torch when not given: the C call itself allocates nothing."""
+    B, T, H, _ = q.shape
+    if out is None:
+        out = torch.empty((B, T, H, v.shape[3]), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((B, H, q.shape[3], v.shape[3]), dtype=torch.float32,
+                                  device=q.device)
+    ds = [describe(t) for t in (q, k, v, beta, initial_state, out, final_state)]
+    st = load().deltanet_fwd_noalloc(*[_ref(x) for x in ds[:5]], int(chunk_size),
+                                     *[_ref(x) for x in ds[5:]],
+                                     _stream_handle(q.device, stream))
     if st != DN_OK:
         raise DeltaNetError(st, status_string(st))
     return out, final_state

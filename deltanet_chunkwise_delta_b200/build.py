@@ -1,8 +1,8 @@
 """Builds the sm_100a shared library behind the C ABI (include/deltanet.h).
 
-``python -m deltanet_chunkwise_delta_b200.build`` compiles
-``csrc/deltanet.cu`` with nvcc into ``_build/libdeltanet_b200.so`` inside the
-package directory, so the library travels with the source tree.
+``python -m deltanet_chunkwise_delta_b200.build`` compiles ``csrc/deltanet.cu``
+and ``csrc/deltanet_noalloc.cu`` with nvcc into ``_build/libdeltanet_b200.so``
+inside the package directory, so the library travels with the source tree.
 """
 from __future__ import annotations
 
@@ -13,7 +13,7 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "deltanet.cu")
+SRCS = [os.path.join(PKG, "csrc", "deltanet.cu"), os.path.join(PKG, "csrc", "deltanet_noalloc.cu")]
 LIB = os.path.join(PKG, "_build", "libdeltanet_b200.so")
 
 NVCC_FLAGS = [
@@ -42,7 +42,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(os.path.dirname(LIB), exist_ok=True)
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, SRC]
+    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, *SRCS]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)

@@ -103,6 +103,35 @@ dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tenso
                           dn_tensor* out, dn_tensor* final_state, void* stream,
                           int seg_chunks);
 
+/*
+ * deltanet_fwd_noalloc -- the forward pass without any device allocation.
+ * (No counterpart on the pages: this is a deployment variant of deltanet_fwd.)
+ *
+ * For callers that cannot call cudaMalloc: code running where the allocator
+ * must not be entered (host callbacks, plugins inside another runtime's
+ * allocator, graph-recording runtimes that forbid allocation) or processes
+ * whose device memory is capped and owned by someone else.  deltanet_fwd may
+ * grow a cached workspace with cudaMallocAsync; this call never allocates.
+ * Its scratch (the per-chunk UT factors and an error word) is one fixed
+ * 48 MiB + 256 B __device__ array that every GPU loading the library holds
+ * until the process exits.
+ *
+ * Arguments as deltanet_fwd, without cu_seqlens.  Supported: dense batches,
+ * bf16 q/k/v/out, d_k = d_v = 128, chunk_size 64, and
+ * B * ceil(T / 64) * H <= 6144 (chunk, head) pairs; larger problems return
+ * DN_ERR_WORKSPACE, other shapes or dtypes DN_ERR_UNSUPPORTED / _INVALID_ARG.
+ * Outputs must not overlap inputs (not checked here).  Each (sequence, head)
+ * runs as one run of chunks (no split across SMs).
+ * The first call on a device looks up the array's device address and sets
+ * kernel attributes; make it before any stream capture.  All calls share the
+ * array, which keeps the last call's contents, so calls that overlap on the
+ * GPU race with each other; serialise them (one stream, or events).
+ */
+dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                               const dn_tensor* beta, const dn_tensor* initial_state,
+                               int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                               void* stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* deltanet_status_string(dn_status status);
 
