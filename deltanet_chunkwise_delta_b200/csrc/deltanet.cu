@@ -494,6 +494,9 @@ void deltanet_release_workspace(void) {
 int dn_trace_copy(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, tc::g_dn_trace, sizeof(tc::g_dn_trace)) == cudaSuccess ? 0 : 1;
 }
+int dn_trace_copy_prep(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_dn_trace_prep, sizeof(g_dn_trace_prep)) == cudaSuccess ? 0 : 1;
+}
 #endif
 
 void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment) {

@@ -13,12 +13,14 @@
 // S^T (d_v lanes x d_k columns, fp32) lives in tensor memory for the whole run;
 // a bf16 copy in shared memory feeds the next chunk's products.
 //
-// Warp roles (480 threads):
+// Warp roles (512 threads):
 //   warps 0-7   chain epilogue: Z^T -> bf16, S^T -> bf16, O -> global
-//   warps 8-11  chunk-parallel epilogue: G -> P; W^T -> W
-//   warp 12     issues the state-chain products (Z, O, S updates), one thread
-//   warp 13     issues the TMA loads of q, k, v and the bulk copy of T, one thread
+//   warps 8-11  chunk-parallel epilogue: W^T -> bf16 rows; G -> P
+//   warp 12     issues the state-chain products (Z, O, S updates), one thread;
+//               owns the tensor-memory allocation
+//   warp 13     TMA loads of q, k (3-stage ring), one thread
 //   warp 14     issues the chunk-parallel products (G, W^T, U^T), one thread
+//   warp 15     TMA loads of v and bulk copies of T (2-stage ring), one thread
 // The two issuers run independently, so the chunk-parallel work of chunk
 // r+1 overlaps the state chain of chunk r.  Buffers that outlive one chunk
 // are double-buffered with one "free" barrier per buffer.  Every wait on an
@@ -35,21 +37,25 @@ namespace tc {
 using namespace sm100;
 
 constexpr int D = 128;
-constexpr int kThreadsTc = 480;
+constexpr int kThreadsTc = 512;
 constexpr int kChainMmaWarp = 12;
 constexpr int kTmaWarp = 13;
 constexpr int kParMmaWarp = 14;
+constexpr int kTmaBWarp = 15;
 
 // shared memory (byte offsets from a 1024-aligned base)
-// stage: [Q|K] for d 0-63, [Q|K] for d 64-127, V (2 x 8 KB), T (8 KB)
-constexpr int ST_V = 32768, ST_T = 49152;
-constexpr int STAGE_BYTES = 57344;
-constexpr int OFF_WB = 2 * STAGE_BYTES;       // 2 x W^T rows (d_k rows of 64 tokens)
-constexpr int OFF_PB = OFF_WB + 2 * 16384;
-constexpr int OFF_ZB = OFF_PB + 2 * 8192;
-constexpr int OFF_SBF = OFF_ZB + 16384;
+//   ring A (q, k): 3 stages of [Q d0-63 | K d0-63 | Q d64-127 | K d64-127]
+//   ring B (v, T): 2 stages of [V d0-63 | V d64-127 | T]
+constexpr int NA = 3, NB = 2;
+constexpr int A_STAGE = 32768;
+constexpr int OFF_B = NA * A_STAGE;
+constexpr int B_STAGE = 24576, B_T = 16384;
+constexpr int OFF_WB = OFF_B + NB * B_STAGE;   // W^T rows (d_k rows of 64 tokens)
+constexpr int OFF_PB = OFF_WB + 16384;         // P rows
+constexpr int OFF_ZB = OFF_PB + 8192;          // Z^T rows
+constexpr int OFF_SBF = OFF_ZB + 16384;        // S^T rows, bf16
 constexpr int OFF_BAR = OFF_SBF + 32768;
-constexpr int NBAR = 22;
+constexpr int NBAR = 26;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_USED = OFF_MISC + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -58,30 +64,31 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // tensor-memory columns (512 allocated): S^T, O^T, 2 x U^T/Z^T, 2 x W^T, G
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_ZU = 192, TM_WT = 320, TM_G = 448;
 
-// Barriers named "+buf" come in pairs, one per buffer (chunk parity); a
-// waiter on such a barrier waits for its (r / 2)-th completion.
+// Barriers of a ring or of a double buffer come one per slot; a waiter on slot
+// s for chunk r waits for that slot's (r / slots)-th completion.
 enum : int {
-    B_FULL = 0,     // +buf: TMA landed
-    B_EMPTY = 2,    // +buf: stage consumed by both issuers
-    B_GFULL = 4,    // G ready in TMEM
-    B_GFREE = 5,    // G read out (P written)
-    B_WUFULL = 6,   // +buf: W^T, U^T ready in TMEM
-    B_WFULL = 8,    // +buf: W^T (bf16) written to shared memory, TMEM copy read
-    B_C1A = 10,     // Z^T = U^T - S^T W^T complete
-    B_ZFULL = 11,   // Z^T (bf16) written
-    B_SFULL = 12,   // S^T updated
-    B_OFULL = 13,   // O^T complete
-    B_SBF = 14,     // bf16 copy of S^T written
-    B_OFREE = 15,   // O^T read out
-    B_PFREE = 16,   // +buf: P consumed
-    B_ZFREE = 18,   // +buf: U^T / Z^T columns read out
-    B_WFREE = 20,   // +buf: W^T (bf16) consumed
+    B_FULLA = 0,     // +3: q, k of a stage landed
+    B_EMPTYA = 3,    // +3: stage of ring A consumed by both issuers
+    B_FULLB = 6,     // +2: v, T landed
+    B_EMPTYB = 8,    // +2: stage of ring B consumed
+    B_GFULL = 10,    // G ready in TMEM
+    B_GFREE = 11,    // G read out (P written)
+    B_WUFULL = 12,   // +2: W^T, U^T ready in TMEM
+    B_WFULL = 14,    // W^T rows written to shared memory
+    B_C1A = 15,      // Z^T = U^T - S^T W^T complete
+    B_ZFULL = 16,    // Z^T (bf16) written
+    B_SFULL = 17,    // S^T updated
+    B_OFULL = 18,    // O^T complete (P consumed)
+    B_SBF = 19,      // bf16 copy of S^T written
+    B_OFREE = 20,    // O^T read out
+    B_ZFREE = 21,    // +2: U^T / Z^T columns read out
+    B_WTFREE = 23,   // +2: W^T columns read out
 };
 
 // Optional timeline of CTA 0 (build with -DDN_TRACE): globaltimer stamps per
 // chunk and pipeline event, read back with dn_trace_copy().
 #ifdef DN_TRACE
-__device__ unsigned long long g_dn_trace[64 * 32];
+static __device__ unsigned long long g_dn_trace[64 * 32];
 #define DN_TR(cond, r, slot)                                                          \
     do {                                                                              \
         if ((cond) && blockIdx.x == 0 && (r) < 64 && (threadIdx.x & 31) == 0)          \
@@ -131,17 +138,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        for (int s = 0; s < NA; ++s) {
+            mbar_init(&bars[B_FULLA + s], 1);
+            mbar_init(&bars[B_EMPTYA + s], 2);
+        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[B_FULL + s], 1);
-            mbar_init(&bars[B_EMPTY + s], 2);
-            mbar_init(&bars[B_PFREE + s], 1);
-            mbar_init(&bars[B_ZFREE + s], 256);
+            mbar_init(&bars[B_FULLB + s], 1);
+            mbar_init(&bars[B_EMPTYB + s], 1);
             mbar_init(&bars[B_WUFULL + s], 1);
-            mbar_init(&bars[B_WFULL + s], 128);
-            mbar_init(&bars[B_WFREE + s], 1);
+            mbar_init(&bars[B_ZFREE + s], 256);
+            mbar_init(&bars[B_WTFREE + s], 128);
         }
         mbar_init(&bars[B_GFULL], 1);
         mbar_init(&bars[B_GFREE], 64);
+        mbar_init(&bars[B_WFULL], 128);
         mbar_init(&bars[B_C1A], 1);
         mbar_init(&bars[B_ZFULL], 256);
         mbar_init(&bars[B_SFULL], 1);
@@ -182,31 +192,50 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
 
     if (warp == kTmaWarp) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ ring A: q, k
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = (HAS_Q ? 16384u : 0u) + 16384u + (has_v ? 16384u : 0u) + 8192u;
+            const uint32_t bytes = (HAS_Q ? 16384u : 0u) + 16384u;
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
-                const int s = r & 1;
-                if (r >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((r >> 1) - 1) & 1, abort_flag)) break;
-                mbar_expect_tx(&bars[B_FULL + s], bytes);
-                uint8_t* st = smem + s * STAGE_BYTES;
+                const int s = r % NA;
+                if (r >= NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / NA) - 1) & 1, abort_flag)) break;
+                mbar_expect_tx(&bars[B_FULLA + s], bytes);
+                uint8_t* st = smem + s * A_STAGE;
                 const int t0 = it.tok0 + r * kChunk;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
-                    if (HAS_Q) tma_load_4d(st + a * 16384, &tq, &bars[B_FULL + s], a * 64, it.head, t0, it.b);
-                    tma_load_4d(st + a * 16384 + 8192, &tk, &bars[B_FULL + s], a * 64, it.head, t0, it.b);
-                    if (has_v)
-                        tma_load_4d(st + ST_V + a * 8192, &tv, &bars[B_FULL + s], a * 64, it.head, t0, it.b);
+                    if (HAS_Q) tma_load_4d(st + a * 16384, &tq, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
+                    tma_load_4d(st + a * 16384 + 8192, &tk, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
                 }
-                bulk_load(st + ST_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * 8192, 8192,
-                          &bars[B_FULL + s]);
                 issued = r + 1;
                 DN_TR(true, r, 24);
             }
             // the last loads issued must have landed before the CTA may exit
+            for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
+                mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, abort_flag, 200000000ull);
+        }
+    } else if (warp == kTmaBWarp) {
+        // ------------------------------------------------------------ ring B: v, T
+        if (lane == 0 && nch > 0) {
+            const uint32_t bytes = (has_v ? 16384u : 0u) + 8192u;
+            int issued = 0;
+            for (int r = 0; r < nch; ++r) {
+                const int s = r & 1;
+                if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
+                mbar_expect_tx(&bars[B_FULLB + s], bytes);
+                uint8_t* st = smem + OFF_B + s * B_STAGE;
+                const int t0 = it.tok0 + r * kChunk;
+                if (has_v) {
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
+                }
+                bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * 8192, 8192,
+                          &bars[B_FULLB + s]);
+                issued = r + 1;
+            }
             for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
-                mbar_wait(&bars[B_FULL + (r & 1)], (r >> 1) & 1, abort_flag, 200000000ull);
+                mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, abort_flag, 200000000ull);
         }
     } else if (warp == kParMmaWarp) {
         // ------------------------------------------------------------ chunk-parallel products
@@ -215,42 +244,45 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t i_g = idesc_bf16(128, 64, false, false);
             const uint32_t i_tt = idesc_bf16(128, 64, true, false);
             // descriptors at offset 0; per-step offsets are added in 16-byte units
-            const uint64_t dQK = sdesc(sb, 16, 1024);             // K-major [Q;K] / K rows
-            const uint64_t dKT = sdesc(sb + 8192, 16384, 1024);   // K^T, MN-major
-            const uint64_t dVT = sdesc(sb + ST_V, 8192, 1024);    // V^T, MN-major
-            const uint64_t dT = sdesc(sb + ST_T, 16, 1024);       // T^T, K-major
+            const uint64_t dQK = sdesc(sb, 16, 1024);                  // K-major [Q;K] / K rows
+            const uint64_t dKT = sdesc(sb + 8192, 16384, 1024);        // K^T, MN-major
+            const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
+            const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
             for (int r = 0; r < nch; ++r) {
-                const int s = r & 1;
-                const uint64_t st = (uint64_t)((s * STAGE_BYTES) >> 4);
-                if (!mbar_wait(&bars[B_FULL + s], (r >> 1) & 1, abort_flag)) break;
+                const int sa = r % NA, s = r & 1;
+                const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
+                const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
+                if (!mbar_wait(&bars[B_FULLA + sa], (r / NA) & 1, abort_flag)) break;
                 if (HAS_Q) {
                     // G = [Q; K] K^T (only the query rows are used: P)
                     if (r >= 1 && !mbar_wait(&bars[B_GFREE], (r - 1) & 1, abort_flag)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const uint64_t o = st + (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
+                        const uint64_t o = sta + (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
                         umma_bf16(tmem + TM_G, dQK + o, dQK + o + (8192 >> 4), i_g, j > 0);
                     }
                     umma_commit(&bars[B_GFULL]);
                 }
                 // W^T = K^T T^T, U^T = V^T T^T once this parity's W^T and U^T columns are free
-                if (r >= 2 && (!mbar_wait(&bars[B_WFULL + s], ((r >> 1) - 1) & 1, abort_flag) ||
+                if (!mbar_wait(&bars[B_FULLB + s], (r >> 1) & 1, abort_flag)) break;
+                if (r >= 2 && (!mbar_wait(&bars[B_WTFREE + s], ((r >> 1) - 1) & 1, abort_flag) ||
                                !mbar_wait(&bars[B_ZFREE + s], ((r >> 1) - 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    umma_bf16(tmem + TM_WT + s * 64, dKT + st + (uint64_t)((j * 2048) >> 4),
-                              dT + st + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                    umma_bf16(tmem + TM_WT + s * 64, dKT + sta + (uint64_t)((j * 2048) >> 4),
+                              dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 if (has_v) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        umma_bf16(tmem + TM_ZU + (r & 1) * 64, dVT + st + (uint64_t)((j * 2048) >> 4),
-                                  dT + st + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                        umma_bf16(tmem + TM_ZU + s * 64, dVT + stb + (uint64_t)((j * 2048) >> 4),
+                                  dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 }
                 umma_commit(&bars[B_WUFULL + s]);
-                umma_commit(&bars[B_EMPTY + s]);
+                umma_commit(&bars[B_EMPTYB + s]);
+                umma_commit(&bars[B_EMPTYA + sa]);
                 DN_TR(true, r, 5);
             }
         }
@@ -269,22 +301,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint64_t dK = sdesc(sb + 8192, 16384, 1024);   // K, MN-major
             const uint64_t dP = sdesc(sb + OFF_PB, 16, 1024);    // P^T, K-major
             for (int r = 0; r < nch; ++r) {
-                const int s = r & 1;
-                const uint64_t st = (uint64_t)((s * STAGE_BYTES) >> 4);
+                const int sa = r % NA, s = r & 1;
+                const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
                 DN_TR(true, r, 0);
-                if (!mbar_wait(&bars[B_WFULL + s], (r >> 1) & 1, abort_flag) ||
+                if (!mbar_wait(&bars[B_WFULL], r & 1, abort_flag) ||
                     !mbar_wait(&bars[B_SBF], r & 1, abort_flag)) break;
                 tc_fence_after();
                 // Z^T = U^T - S^T W^T
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint64_t o = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
-                    const uint64_t wo = (uint64_t)((s * 16384 + j * 2048) >> 4);
-                    umma_bf16(tmem + TM_ZU + (r & 1) * 64, dS + o, dW + wo, i_c1a,
+                    const uint64_t wo = (uint64_t)((j * 2048) >> 4);
+                    umma_bf16(tmem + TM_ZU + s * 64, dS + o, dW + wo, i_c1a,
                               has_v ? 1u : (j > 0 ? 1u : 0u));
                 }
                 umma_commit(&bars[B_C1A]);
-                umma_commit(&bars[B_WFREE + s]);
                 DN_TR(true, r, 1);
                 if (HAS_Q) {
                     if (!mbar_wait(&bars[B_OFREE], r & 1, abort_flag)) break;
@@ -293,7 +324,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const uint64_t o = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
-                        umma_bf16(tmem + TM_O, dS + o, dQ + st + o, i_c1b, j > 0);
+                        umma_bf16(tmem + TM_O, dS + o, dQ + sta + o, i_c1b, j > 0);
                     }
                 }
                 DN_TR(true, r, 2);
@@ -303,19 +334,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     umma_bf16(tmem + TM_S, dZ + (uint64_t)((j * 32) >> 4),
-                              dK + st + (uint64_t)((j * 2048) >> 4), i_c3, 1u);
+                              dK + sta + (uint64_t)((j * 2048) >> 4), i_c3, 1u);
                 umma_commit(&bars[B_SFULL]);
                 if (HAS_Q) {
                     // O^T += Z^T P^T
-                    const uint64_t pb = (uint64_t)(((r & 1) * 8192) >> 4);
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         umma_bf16(tmem + TM_O, dZ + (uint64_t)((j * 32) >> 4),
-                                  dP + pb + (uint64_t)((j * 32) >> 4), i_c2, 1u);
+                                  dP + (uint64_t)((j * 32) >> 4), i_c2, 1u);
                     umma_commit(&bars[B_OFULL]);
-                    umma_commit(&bars[B_PFREE + (r & 1)]);
                 }
-                umma_commit(&bars[B_EMPTY + s]);
+                umma_commit(&bars[B_EMPTYA + sa]);
                 DN_TR(true, r, 4);
             }
         }
@@ -324,40 +353,42 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const int q = warp - 8;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         for (int r = 0; r < nch; ++r) {
-            if (HAS_Q && q < 2) {
-                // query rows of G: P = (Q K^T) o M_c (inclusive), bf16, rows i
-                if (r >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_PFREE + (r & 1)], ((r >> 1) - 1) & 1, abort_flag))) break;
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_GFULL], r & 1, abort_flag))) break;
-                DN_TR(q == 0, r, 8);
-                tc_fence_after();
-                const int i = 32 * q + lane;
-                uint8_t* pb = smem + OFF_PB + (r & 1) * 8192;
-                uint32_t v[64];
-                tmem_ld64(tmem + lane_base + TM_G, v);
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj)
-                    if (jj > i) v[jj] = 0u;
-                st_row_bf16<64>(pb, i, 0, v);
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bars[B_GFREE]);
-                DN_TR(q == 0, r, 9);
-            }
-            // W^T (TMEM, d_k lanes) -> bf16 rows of 64 tokens (an MN-major operand)
             const int s = r & 1;
-            if (r >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_WFREE + s], ((r >> 1) - 1) & 1, abort_flag))) break;
+            // W^T (TMEM, d_k lanes) -> bf16 rows of 64 tokens (an MN-major operand),
+            // once the previous W^T rows are consumed
+            if (r >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_C1A], (r - 1) & 1, abort_flag))) break;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_WUFULL + s], (r >> 1) & 1, abort_flag))) break;
             DN_TR(q == 0, r, 13);
             tc_fence_after();
             {
                 uint32_t v[64];
                 tmem_ld64(tmem + lane_base + TM_WT + s * 64, v);
-                st_row_bf16<64>(Wb + s * 16384, 32 * q + lane, 0, v);
+                tc_fence_before();
+                mbar_arrive(&bars[B_WTFREE + s]);
+                st_row_bf16<64>(Wb, 32 * q + lane, 0, v);
             }
             fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[B_WFULL + s]);
+            mbar_arrive(&bars[B_WFULL]);
             DN_TR(q == 0, r, 14);
+            if (HAS_Q && q < 2) {
+                // query rows of G: P = (Q K^T) o M_c (inclusive), bf16 rows i, once the
+                // previous P is consumed
+                if (r >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL], (r - 1) & 1, abort_flag))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_GFULL], r & 1, abort_flag))) break;
+                DN_TR(q == 0, r, 8);
+                tc_fence_after();
+                const int i = 32 * q + lane;
+                uint32_t v[64];
+                tmem_ld64(tmem + lane_base + TM_G, v);
+                tc_fence_before();
+                mbar_arrive(&bars[B_GFREE]);
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj)
+                    if (jj > i) v[jj] = 0u;
+                st_row_bf16<64>(smem + OFF_PB, i, 0, v);
+                fence_async_smem();
+                DN_TR(q == 0, r, 9);
+            }
         }
     } else {
         // ------------------------------------------------------------ chain epilogue
@@ -389,19 +420,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (HAS_Q) mbar_arrive(&bars[B_OFREE]);
         __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
         for (int r = 0; r < nch; ++r) {
+            const int s = r & 1;
             // Z^T -> bf16 operand
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1A], r & 1, abort_flag))) break;
             DN_TR(warp == 0, r, 16);
             tc_fence_after();
             {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_base + TM_ZU + (r & 1) * 64 + 32 * h, v);
+                tmem_ld32(tmem + lane_base + TM_ZU + s * 64 + 32 * h, v);
                 st_row_bf16<32>(Zb, d, 32 * h, v);
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_ZFULL]);
-            mbar_arrive(&bars[B_ZFREE + (r & 1)]);
+            mbar_arrive(&bars[B_ZFREE + s]);
             DN_TR(warp == 0, r, 17);
             // S^T -> bf16 operand (and fp32 out after the last chunk)
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL], r & 1, abort_flag))) break;
