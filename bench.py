@@ -63,6 +63,34 @@ def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
     return float(b)
 
 
+def kernel_source_digest() -> str:
+    """Digest of the CUDA sources, so that a stored ncu traffic figure is only
+    used for the kernels it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "deltanet_chunkwise_delta_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per launch of the boundary kernel from the committed ncu
+    summary of this workload, if it was taken on the current sources."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"k_tc_chain_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_src = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    m_val = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_src or not m_val or m_src.group(1) != kernel_source_digest():
+        return None
+    return int(m_val.group(1))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -231,9 +259,15 @@ def run_b200(args, w: wl.Workload):
     if dn.get_error(stream) != 0:
         raise RuntimeError("device reported an error")
     G, s = dn.last_schedule()
-    launches_per_step = 1 if G == 1 else (3 if G > 1 else 4)
+    launches_per_step = dn.last_launches()
     for _ in range(args.warmup):
         step()
+    # one event pair per timed step around the boundary-pass (output) kernel
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in kev:
+        a.record(stream)
+        b.record(stream)
     torch.cuda.synchronize(device)
     barrier(ws)
     torch.cuda.synchronize(device)
@@ -241,14 +275,17 @@ def run_b200(args, w: wl.Workload):
     ev1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         ev0.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
+            dn.set_kernel_events(*kev[i])
             step()
         ev1.record(stream)
         ev1.synchronize()
+    dn.set_kernel_events()
     torch.cuda.synchronize(device)
     barrier(ws)
     ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms_local, ws, device)
+    kernel_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
 
     tokens = w.tokens
     value = ws * tokens / (ms / 1e3)
@@ -256,11 +293,25 @@ def run_b200(args, w: wl.Workload):
     tflops = ws * th * flops_per_token_head(w.dk, w.dv) / (ms / 1e3) / 1e12
     hbm_peak, tc_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(w)
-    achieved = alg_bytes / (ms_local / 1e3) / 1e9
+    # the boundary (output) kernel moves q, k, v, o and the states; beta is read by the
+    # UT pre-pass
+    kernel_bytes = alg_bytes - 4.0 * w.tokens * w.H
+    achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9
+    tc_kernel = w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
-                "kernel": "k_boundary" if G == 1 else "whole step (summary + scan + boundary)",
-                "algorithmic_bytes_per_launch": alg_bytes}
+                "frac": achieved / hbm_peak,
+                "traffic": stored_traffic(w.name) if tc_kernel else None,
+                "peak_kind": peak_kind,
+                "kernel": "k_tc_chain<true> (boundary pass)" if tc_kernel else "k_boundary",
+                "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": kernel_bytes}
+    # the whole path against its roofline: slower of FLOPs at the bf16 peak and bytes at HBM
+    t_roof = max(th * flops_per_token_head(w.dk, w.dv) / (tc_peak * 1e12),
+                 alg_bytes / (hbm_peak * 1e9))
+    roofline_step = {"bound": "hbm" if alg_bytes / hbm_peak > th * flops_per_token_head(w.dk, w.dv) / tc_peak / 1e3 else "tensor",
+                     "roofline_ms": t_roof * 1e3, "step_ms": ms_local,
+                     "frac": t_roof * 1e3 / ms_local, "algorithmic_bytes": alg_bytes,
+                     "algorithmic_flops": th * flops_per_token_head(w.dk, w.dv),
+                     "peaks": {"hbm_gbs": hbm_peak, "bf16_tflops": tc_peak, "kind": peak_kind}}
 
     # end to end through the public call with host buffers
     e2e = None
@@ -323,6 +374,7 @@ def run_b200(args, w: wl.Workload):
         "tflops": tflops,
         "tflops_unit": "algorithmic TFLOP/s (6Cd^2 + 5C^2d + C^3/3 per chunk-head)",
         "roofline": roofline,
+        "roofline_step": roofline_step,
         "clocks": clk.summary(),
         "e2e": e2e,
         "cpu_baseline": cpu,

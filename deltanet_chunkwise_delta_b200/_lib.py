@@ -23,7 +23,7 @@ DN_F32, DN_BF16, DN_I32 = 0, 1, 2
 
 EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
-            "deltanet_fwd_noalloc")
+            "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events")
 
 
 class DnTensor(ctypes.Structure):
@@ -71,6 +71,10 @@ def load(path: Optional[str] = None):
         lib.deltanet_get_error.argtypes = [ctypes.c_void_p]
         lib.deltanet_release_workspace.restype = None
         lib.deltanet_release_workspace.argtypes = []
+        lib.deltanet_last_launches.restype = ctypes.c_int
+        lib.deltanet_last_launches.argtypes = []
+        lib.deltanet_set_kernel_events.restype = None
+        lib.deltanet_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
         lib.deltanet_last_schedule.restype = None
         lib.deltanet_last_schedule.argtypes = [ctypes.POINTER(ctypes.c_int),
                                                ctypes.POINTER(ctypes.c_int)]
@@ -182,6 +186,18 @@ def get_error(stream=None, device=None) -> int:
 
 def release_workspace() -> None:
     load().deltanet_release_workspace()
+
+
+def last_launches() -> int:
+    return load().deltanet_last_launches()
+
+
+def set_kernel_events(start=None, stop=None) -> None:
+    """Bracket the boundary-pass kernel of following calls with two
+    torch.cuda.Event objects (enable_timing=True, already recorded once so that
+    their handles exist); call with no arguments to stop."""
+    load().deltanet_set_kernel_events(start.cuda_event if start is not None else None,
+                                      stop.cuda_event if stop is not None else None)
 
 
 def last_schedule():

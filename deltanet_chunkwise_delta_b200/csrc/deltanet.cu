@@ -23,7 +23,8 @@ using namespace dn;
 
 namespace {
 
-thread_local int g_last_G = 0, g_last_s = 0;
+thread_local int g_last_G = 0, g_last_s = 0, g_last_launches = 0;
+thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
 
 struct StreamWs {
     int* flag = nullptr;  // [0] error flag
@@ -319,20 +320,27 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         g_last_G = -1;
         g_last_s = -1;
     }
+    int launches = d.varlen ? 1 : 0;
     if (kTc) {
         const int64_t units = chunk_ub * d.H;
         if (units > 0) {
             const int grid = (int)std::min<int64_t>(units, (int64_t)sms * 8);
             kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(p);
+            ++launches;
         }
-        if (nA > 0) kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-        if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
-        if (nC > 0) kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        if (nA > 0) { kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p); ++launches; }
+        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p); ++launches; }
+        if (g_ev_start) cudaEventRecord(g_ev_start, stream);
+        if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p); ++launches; }
+        if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
     } else {
-        if (nA > 0) kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p);
-        if (nScan > 0) kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p);
-        if (nC > 0) kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p);
+        if (nA > 0) { kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p); ++launches; }
+        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p); ++launches; }
+        if (g_ev_start) cudaEventRecord(g_ev_start, stream);
+        if (nC > 0) { kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p); ++launches; }
+        if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
     }
+    g_last_launches = launches;
     if (cudaGetLastError() != cudaSuccess) return DN_ERR_CUDA;
     return DN_OK;
 }
@@ -502,6 +510,13 @@ int dn_trace_copy_prep(unsigned long long* host) {
 void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment) {
     if (segments_per_chain) *segments_per_chain = g_last_G;
     if (chunks_per_segment) *chunks_per_segment = g_last_s;
+}
+
+int deltanet_last_launches(void) { return g_last_launches; }
+
+void deltanet_set_kernel_events(void* start_event, void* stop_event) {
+    g_ev_start = static_cast<cudaEvent_t>(start_event);
+    g_ev_stop = static_cast<cudaEvent_t>(stop_event);
 }
 
 }  // extern "C"

@@ -153,6 +153,19 @@ void deltanet_release_workspace(void);
  */
 void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment);
 
+/* Number of kernels the last successful call on this thread enqueued. */
+int deltanet_last_launches(void);
+
+/*
+ * deltanet_set_kernel_events -- profiling hook.  While set (non-NULL), every
+ * deltanet_fwd / deltanet_fwd_ex call on this thread records start_event on
+ * its stream right before launching the boundary-pass kernel (the output
+ * kernel, which dominates the call) and stop_event right after it, so that
+ * cudaEventElapsedTime gives that kernel's device time.  The caller owns the
+ * events (cudaEvent_t, created with timing enabled); pass NULL, NULL to stop.
+ */
+void deltanet_set_kernel_events(void* start_event, void* stop_event);
+
 #ifdef __cplusplus
 }
 #endif
