@@ -213,8 +213,8 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kS = k_scan<DK, DV>;
     auto* kCt = tc::k_tc_chain<true>;
     auto* kAt = tc::k_tc_chain<false>;
-    auto* kPrep = k_ut_prep<128>;
-    constexpr int smemPrep = PrepSmem<128>::TOTAL;
+    auto* kPrep = k_ut_prep;
+    constexpr int smemPrep = PrepSmem::TOTAL;
     dn_status st;
     if (kTc) {
         if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
@@ -225,12 +225,13 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
     }
     if ((st = set_smem(kS, dev, smemS)) != DN_OK) return st;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (kTc) {
         const int64_t Bq = d.varlen ? 1 : d.B;
         if ((st = make_token_map(&tq, p.q, Bq, d.T, d.H, p.q_sb, p.q_st, p.q_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tk, p.k, Bq, d.T, d.H, p.k_sb, p.k_st, p.k_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tv, p.v, Bq, d.T, d.H, p.v_sb, p.v_st, p.v_sh)) != DN_OK) return st;
+        if ((st = make_token_map(&to, p.o, Bq, d.T, d.H, p.o_sb, p.o_st, p.o_sh)) != DN_OK) return st;
     }
 
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
@@ -277,7 +278,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     // UT factors of every (chunk, head): chunks <= ceil(T / C) per row (+1 per sequence)
     const int64_t chunk_ub = d.varlen ? n_c_max + d.N : d.B * n_c_max;
     const size_t off_T = off_SS + up256((size_t)slots * DK * DV * 4);
-    bytes = off_T + (kTc ? (size_t)chunk_ub * d.H * 8192 : 0);
+    bytes = off_T + (kTc ? (size_t)chunk_ub * d.H * kUnitBytes : 0);
     StreamWs ws;
     if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
     char* base = ws.buf;
@@ -324,14 +325,14 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     if (kTc) {
         const int64_t units = chunk_ub * d.H;
         if (units > 0) {
-            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * 8);
-            kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(p);
+            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * kPrepCtasPerSm);
+            kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
             ++launches;
         }
-        if (nA > 0) { kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p); ++launches; }
+        if (nA > 0) { kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, tq, p); ++launches; }
         if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p); ++launches; }
         if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-        if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, p); ++launches; }
+        if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
         if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
     } else {
         if (nA > 0) { kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p); ++launches; }

@@ -7,7 +7,7 @@
 // records, or a memory-capped process whose allocator is owned by someone
 // else.  deltanet_fwd caches a per-stream workspace that it may grow with
 // cudaMallocAsync; this entry point never allocates.  Its only scratch (the
-// per-chunk UT factors T, and an error word) lives in one fixed-size
+// per-chunk factors T and P, and an error word) lives in one fixed-size
 // __device__ array below, which every GPU that loads the library holds until
 // the process exits.
 //
@@ -36,9 +36,9 @@
 
 namespace {
 
-constexpr int kNoAllocMaxUnits = 6144;                 // (chunk, head) pairs
+constexpr int kNoAllocMaxUnits = 3072;                 // (chunk, head) pairs
 constexpr size_t kNoAllocFlagBytes = 256;              // error word + padding
-constexpr size_t kNoAllocScratchBytes = kNoAllocFlagBytes + (size_t)kNoAllocMaxUnits * 8192;  // 48 MiB + 256 B
+constexpr size_t kNoAllocScratchBytes = kNoAllocFlagBytes + (size_t)kNoAllocMaxUnits * dn::kUnitBytes;  // 48 MiB + 256 B
 
 // In host code this name is only a host-side stand-in for the device array;
 // kernels receive the address returned by cudaGetSymbolAddress.
@@ -92,8 +92,8 @@ dn_status na_setup(int dev, unsigned char** scratch) {
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DN_ERR_CUDA;
     if (cudaFuncSetAttribute(dn::tc::k_tc_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::tc::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(dn::k_ut_prep<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             dn::PrepSmem<128>::TOTAL) != cudaSuccess)
+        cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dn::PrepSmem::TOTAL) != cudaSuccess)
         return DN_ERR_CUDA;
     g_na_scratch[dev] = static_cast<unsigned char*>(ptr);
     *scratch = static_cast<unsigned char*>(ptr);
@@ -174,9 +174,9 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     sc.G = 1;
     sc.s = (int)n_c;
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!na_map(&tq, q->data, B, T, H, q->stride) || !na_map(&tk, k->data, B, T, H, k->stride) ||
-        !na_map(&tv, v->data, B, T, H, v->stride))
+        !na_map(&tv, v->data, B, T, H, v->stride) || !na_map(&to, out->data, B, T, H, out->stride))
         return DN_ERR_UNSUPPORTED;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
@@ -185,9 +185,20 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DN_ERR_CUDA;
     const int64_t units = B * n_c * H;
-    const int grid = (int)(units < (int64_t)sms * 8 ? units : (int64_t)sms * 8);
-    dn::k_ut_prep<128><<<grid, dn::kPrepThreads, dn::PrepSmem<128>::TOTAL, stream>>>(p);
+    const int64_t cap = (int64_t)sms * dn::kPrepCtasPerSm;
+    const int grid = (int)(units < cap ? units : cap);
+    dn::k_ut_prep<<<grid, dn::kPrepThreads, dn::PrepSmem::TOTAL, stream>>>(tq, tk, p);
     dn::tc::k_tc_chain<true><<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
-        tq, tk, tv, p);
+        tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
+
+#ifdef DN_TRACE
+// Timeline readers for this translation unit's copies of the trace arrays.
+extern "C" int dn_trace_copy_na(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, dn::tc::g_dn_trace, sizeof(dn::tc::g_dn_trace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int dn_trace_copy_prep_na(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, dn::g_dn_trace_prep, sizeof(dn::g_dn_trace_prep)) == cudaSuccess ? 0 : 1;
+}
+#endif

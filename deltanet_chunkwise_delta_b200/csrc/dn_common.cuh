@@ -14,6 +14,8 @@ constexpr int kChunk = 64;       // C
 constexpr int kThreads = 256;    // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 4096;  // segment-map slots (P, H, start state) per call
+// workspace bytes per (chunk, head) written by the UT pre-pass: T tile, then P tile
+constexpr int kUnitBytes = 16384;
 constexpr int kAutoMaxSlots = 592;  // slots the automatic schedule may use (4 x 148)
 
 // Device error flag values (match dn_status).

@@ -1,22 +1,26 @@
-// UT pre-pass: the chunk-local factor of every (chunk, head), computed once.
+// UT pre-pass: the chunk-local factors of every (chunk, head), computed once.
 //
 // "Context Parallelism for DeltaNet", section 2, step 1: the WY factors of a
 // chunk depend only on that chunk's keys and step sizes, so every chunk can be
 // processed in parallel.  Per (chunk r, head) this kernel forms
+//   G_r = [Q_r; K_r] K_r^T                 (one tcgen05 product, M = 128)
 //   L_r = (K_r K_r^T) o M_c^-,    T_r = (I + B_r L_r)^{-1} B_r
+//   P_r = (Q_r K_r^T) o M_c               (inclusive causal mask)
 // ("Linear Attention, Visualized", DeltaNet, "Complete per-chunk algorithm")
-// and stores T_r as a bf16 64 x 64 tile whose rows are 128 bytes with the
-// 128-byte swizzle, i.e. exactly the shared-memory layout in which the chain
-// kernel uses T^T as a tensor-core operand (it copies the tile in with one
-// bulk copy).  W_r = T_r K_r and U_r = T_r V_r are formed later, on the
-// tensor cores, next to the state chain.
+// and stores T_r and P_r as two bf16 64 x 64 tiles (16 KB per unit, T first)
+// whose rows are 128 bytes with the 128-byte swizzle: exactly the
+// shared-memory layout in which the chain kernel uses T^T and P^T as
+// tensor-core operands (it copies each tile in with one bulk copy).
+// W_r = T_r K_r and U_r = T_r V_r are formed later, next to the state chain.
 //
 // The 64 x 64 solve is blocked in 16 x 16 blocks: N = (I + A)^{-1} with
 // A = B L; each diagonal block by forward substitution (one warp per block,
 // one column per lane, fp32), then N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj in
 // order of i - j with tf32 mma.sync, and T = N B.
-// One CTA of 4 warps per (chunk, head) at a time, several CTAs per SM, so the
-// latency of the solve is hidden by parallelism across chunks.
+// One CTA of 4 warps per (chunk, head) at a time, three CTAs per SM, so the
+// latency of the solve is hidden by parallelism across chunks.  The q/k tile
+// of the next unit is loaded by TMA as soon as this unit's product has read
+// the current one.
 #pragma once
 
 #include "dn_chain.cuh"
@@ -43,20 +47,23 @@ static __device__ unsigned long long g_dn_trace_prep[16 * 8];
 #endif
 
 constexpr int kPrepThreads = 128;
+constexpr int kPrepCtasPerSm = 3;
 constexpr int kBlkLd = 20;  // fp32 16 x 16 blocks, 16-byte aligned rows
 constexpr int kBlkFloats = 16 * kBlkLd;
 
-template <int DK>
+// Shared memory of the pre-pass (byte offsets from a 1024-aligned base).
 struct PrepSmem {
-    static constexpr int K_BYTES = kChunk * DK * 2;  // one K tile; the A blocks reuse it
-    static constexpr int A_BYTES = 10 * kBlkFloats * 4;
-    static_assert(A_BYTES <= K_BYTES, "A blocks must fit in a K tile");
-    static constexpr int OFF_K = 0;                  // 2 K tiles (double buffer)
-    static constexpr int OFF_N = 2 * K_BYTES;
-    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;
-    static constexpr int OFF_BETA = OFF_X + 6 * kBlkFloats * 4;
-    static constexpr int TOTAL = OFF_BETA + 2 * kChunk * 4;
+    static constexpr int OFF_QK = 0;                              // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127]
+    static constexpr int OFF_A = 32768;                           // 10 blocks of A = B L
+    static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N
+    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 6 staging blocks
+    static constexpr int OFF_BETA = OFF_X + 6 * kBlkFloats * 4;   // 2 x 64 step sizes
+    static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE
+    static constexpr int OFF_MISC = OFF_BAR + 16;                 // TMEM address, abort flag
+    static constexpr int USED = OFF_MISC + 16;
+    static constexpr int TOTAL = USED + 1024;                     // slack for 1024-byte alignment
 };
+static_assert(PrepSmem::TOTAL * kPrepCtasPerSm <= 227 * 1024, "pre-pass shared memory");
 
 __device__ __forceinline__ int blk_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
 
@@ -108,83 +115,142 @@ __device__ __forceinline__ void ld_blk(float (&acc)[2][4], const float* C) {
     }
 }
 
-template <int DK>
-__global__ void __launch_bounds__(kPrepThreads, 4) k_ut_prep(Params p) {
-    using L = PrepSmem<DK>;
-    extern __shared__ __align__(128) char smem[];
+static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
+    k_ut_prep(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
+    using L = PrepSmem;
+    extern __shared__ uint8_t prep_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(prep_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float* Ablk = reinterpret_cast<float*>(smem + L::OFF_A);
     float* Nblk = reinterpret_cast<float*>(smem + L::OFF_N);
     float* Xs = reinterpret_cast<float*>(smem + L::OFF_X);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);  // [0] FULL, [1] GDONE
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g8 = lane >> 2, t4 = lane & 3;
     const int H = p.sched.H;
     const int units = count_chunks(p.sched) * H;
+    if ((int)blockIdx.x >= units) return;
 
-    // K tile and step sizes of unit u into buffer `buf` (cp.async; one group)
-    auto issue = [&](int u, int buf) {
+    if (tid == 0) {
+        sm100::mbar_init(&bars[0], 1);
+        sm100::mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        sm100::mbar_fence_init();
+    }
+    if (warp == 0) {
+        sm100::tmem_alloc(tmem_slot, 64);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // q/k tile of unit u (TMA, thread 0) and its step sizes into beta buffer `bb`
+    // (cp.async, zero past the chunk's last token, which zeroes T's rows and
+    // columns there; one group)
+    auto issue = [&](int u, int bb) {
         const int id = u / H, head = u % H;
         int b, t0, t1;
         chunk_range(p.sched, id, b, t0, t1);
-        const int rows = t1 - t0;
-        const __nv_bfloat16* kg =
-            static_cast<const __nv_bfloat16*>(p.k) + b * p.k_sb + head * p.k_sh + (int64_t)t0 * p.k_st;
-        load_tile<__nv_bfloat16, DK, kPrepThreads>(
-            reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K + buf * L::K_BYTES), kg, p.k_st, rows);
+        if (tid == 0) {
+            sm100::mbar_expect_tx(&bars[0], 32768u);
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                sm100::tma_load_4d(smem + L::OFF_QK + a * 16384, &tq, &bars[0], a * 64, head, t0, b);
+                sm100::tma_load_4d(smem + L::OFF_QK + a * 16384 + 8192, &tk, &bars[0], a * 64, head, t0, b);
+            }
+        }
         if (tid < kChunk) {
-            const bool ok = tid < rows;
+            const bool ok = tid < t1 - t0;
             const float* src = p.beta + b * p.b_sb + (int64_t)(t0 + (ok ? tid : 0)) * p.b_st + head * p.b_sh;
-            cp_async4(smem_addr(smem + L::OFF_BETA + (buf * kChunk + tid) * 4), src, ok ? 4 : 0);
+            cp_async4(smem_addr(smem + L::OFF_BETA + (bb * kChunk + tid) * 4), src, ok ? 4 : 0);
         }
         cp_async_commit();
     };
 
-    int buf = 0, it_ = 0;
-    if ((int)blockIdx.x < units) issue(blockIdx.x, 0);
-    for (int u = blockIdx.x; u < units; u += gridDim.x, buf ^= 1, ++it_) {
+    const uint32_t i_g = sm100::idesc_bf16(128, 64, false, false);
+    const uint64_t dQK = sm100::sdesc(sm100::saddr(smem + L::OFF_QK), 16, 1024);
+    bool in_flight = true;
+    issue(blockIdx.x, 0);
+    int it_ = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it_) {
+        const int bb = it_ & 1;
         DN_TRP(it_, 0);
+        const bool got = sm100::mbar_wait(&bars[0], it_ & 1, abort_flag);
+        cp_async_wait<0>();
+        if (__syncthreads_or(!got)) break;
+        in_flight = false;
+        DN_TRP(it_, 1);
+        // G = [Q; K] K^T into 64 tensor-memory columns: lanes 0-63 Q K^T, 64-127 K K^T
+        if (tid == 0) {
+            sm100::tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint64_t o = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
+                sm100::umma_bf16(tmem, dQK + o, dQK + o + (8192 >> 4), i_g, j > 0);
+            }
+            sm100::umma_commit(&bars[1]);
+        }
+        const bool gdone = sm100::mbar_wait(&bars[1], it_ & 1, abort_flag);
+        if (__syncthreads_or(!gdone)) break;
+        sm100::tc_fence_after();
+        // the product has read the q/k tile: load the next unit's
         const int un = u + gridDim.x;
         if (un < units) {
-            issue(un, buf ^ 1);  // prefetch the next unit while this one is computed
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+            issue(un, bb ^ 1);
+            in_flight = true;
         }
-        __syncthreads();
-        DN_TRP(it_, 1);
-        __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem + L::OFF_K + buf * L::K_BYTES);
-        float* Ablk = reinterpret_cast<float*>(Ks);
-        const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + buf * kChunk;
-
-        // A = B L, blocked: warp w owns rows 16w .. 16w + 15 (row block w) and only the
-        // column blocks 0 .. w.  Diagonal blocks are stored transposed (column-major)
-        // for the column sweeps of the solve; the others row-major for the MMAs.
+        const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + bb * kChunk;
         {
-            float acc[8][4];
-            zero_frag(acc);
-            switch (warp) {
-                case 0: warp_gemm<DK, 2, DK, false, DK, false>(*reinterpret_cast<float(*)[2][4]>(acc), Ks, 0, Ks, 0); break;
-                case 1: warp_gemm<DK, 4, DK, false, DK, false>(*reinterpret_cast<float(*)[4][4]>(acc), Ks, 16, Ks, 0); break;
-                case 2: warp_gemm<DK, 6, DK, false, DK, false>(*reinterpret_cast<float(*)[6][4]>(acc), Ks, 32, Ks, 0); break;
-                default: warp_gemm<DK, 8, DK, false, DK, false>(acc, Ks, 48, Ks, 0); break;
-            }
-            const float b_lo = betas[16 * warp + g8], b_hi = betas[16 * warp + g8 + 8];
-            __syncthreads();  // K is no longer read: its space now holds A
+            const int i = 32 * (warp & 1) + lane;  // row of Q K^T (warps 0, 1) or K K^T (warps 2, 3)
+            uint32_t v[64];
+            sm100::tmem_ld64(tmem + ((uint32_t)(32 * warp) << 16), v);
+            if (warp >= 2) {
+                // A = B L, blocked: row i of block row bi; blocks left of the diagonal
+                // row-major, the diagonal block transposed (for the column sweeps)
+                const int bi = i >> 4, ri = i & 15;
+                const float bta = betas[i];
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int bj = nt >> 1;
-                if (bj <= warp) {
-                    float* blk = Ablk + blk_index(warp, bj) * kBlkFloats;
+                for (int bj = 0; bj < 4; ++bj) {
+                    if (bj > bi) continue;
+                    float* blk = Ablk + blk_index(bi, bj) * kBlkFloats;
+                    if (bj < bi) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int row = 16 * warp + g8 + 8 * (e >> 1);
-                        const int col = 8 * nt + 2 * t4 + (e & 1);
-                        const float val = col < row ? ((e >> 1) ? b_hi : b_lo) * acc[nt][e] : 0.f;
-                        if (bj == warp) blk[(col & 15) * kBlkLd + (row & 15)] = val;
-                        else blk[(row & 15) * kBlkLd + (col & 15)] = val;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            float4 f;
+                            f.x = bta * __uint_as_float(v[16 * bj + 4 * q4 + 0]);
+                            f.y = bta * __uint_as_float(v[16 * bj + 4 * q4 + 1]);
+                            f.z = bta * __uint_as_float(v[16 * bj + 4 * q4 + 2]);
+                            f.w = bta * __uint_as_float(v[16 * bj + 4 * q4 + 3]);
+                            *reinterpret_cast<float4*>(blk + ri * kBlkLd + 4 * q4) = f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            blk[c * kBlkLd + ri] = c < ri ? bta * __uint_as_float(v[16 * bj + c]) : 0.f;
                     }
+                }
+            } else {
+                // P = (Q K^T) o M_c, inclusive: bf16 row i of the unit's P tile
+                uint8_t* pg = p.wsT + (size_t)u * kUnitBytes + 8192;
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = (8 * c8 + e <= i) ? __uint_as_float(v[8 * c8 + e]) : 0.f;
+                    uint4 w;
+                    w.x = sm100::pack_bf16(x[0], x[1]);
+                    w.y = sm100::pack_bf16(x[2], x[3]);
+                    w.z = sm100::pack_bf16(x[4], x[5]);
+                    w.w = sm100::pack_bf16(x[6], x[7]);
+                    *reinterpret_cast<uint4*>(pg + sm100::swz128(i, 8 * c8)) = w;
                 }
             }
         }
+        sm100::tc_fence_before();
         __syncthreads();
         DN_TRP(it_, 2);
         // diagonal block `warp` of N = (I + A)^{-1}: one column per lane (lanes 16-31
@@ -271,7 +337,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) k_ut_prep(Params p) {
         // T = N diag(beta) -> bf16 tile (128-byte rows, 128-byte swizzle) in global memory
         {
             const int i = tid >> 1, hh = tid & 1, bi = i >> 4;
-            uint8_t* tg = p.wsT + (size_t)u * 8192;
+            uint8_t* tg = p.wsT + (size_t)u * kUnitBytes;
             float bj32[32];
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
@@ -303,6 +369,19 @@ __global__ void __launch_bounds__(kPrepThreads, 4) k_ut_prep(Params p) {
         }
         __syncthreads();
     }
+    // a load issued for a unit this CTA then gave up on must land before exit
+    if (in_flight) {
+        volatile int drain = 0;
+        sm100::mbar_wait(&bars[0], it_ & 1, &drain, 200000000ull);
+    }
+    cp_async_wait<0>();
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, 64);
+    }
+    if (tid == 0 && *abort_flag) atomicExch(p.err, kErrTimeout);
 }
 
 }  // namespace dn

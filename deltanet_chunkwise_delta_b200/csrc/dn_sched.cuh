@@ -8,11 +8,12 @@
 //   summary pass   run 0: end state; runs 1..G-2: H_g and P_g (two items)
 //   segment scan   start states of runs 1..G-1
 //   boundary pass  every run from its start state: outputs, final state
-// The run length s minimises a simple model of the call's duration:
-//   c * max(min(s, longest chain), chunk-heads / slots)      boundary pass
-// + a * max(s, summary chunk-heads / slots)                  summary pass
-// + scan * (G_max - 1)                                       segment scan
-// with costs per chunk relative to one boundary-pass chunk.
+// The run length s minimises a simple model of the call's duration, with
+// costs per chunk relative to one boundary-pass chunk and one CTA per SM:
+//   dense input (equal runs):  c * s * waves(runs) + a * s * waves(summary items)
+//                              + scan * (G - 1),  waves(n) = ceil(n / SMs)
+//   packed input (unequal):    c * max(min(s, longest chain), chunk-heads / SMs)
+//                              + a * max(s, summary chunk-heads / SMs) + scan * (G_max - 1)
 #pragma once
 
 #include "dn_common.cuh"
@@ -22,7 +23,7 @@ namespace dn {
 struct CostModel {
     float c = 1.0f;      // boundary pass, per chunk
     float a = 0.65f;     // summary pass, per chunk (no output, no Q)
-    float scan = 0.4f;   // one step of the segment scan
+    float scan = 3.0f;   // one step of the segment scan
 };
 
 struct SegChoice {
@@ -34,11 +35,11 @@ struct SegChoice {
 __host__ __device__ inline float dense_cost(const CostModel& m, int chains, int n_c, int s,
                                             int slots) {
     const int G = n_c > 0 ? (n_c + s - 1) / s : 1;
-    const double work = (double)chains * n_c;
-    float tC = m.c * fmaxf((float)min(s, n_c), (float)(work / slots));
-    float tA = 0.f;
-    if (G >= 2) tA = m.a * fmaxf((float)s, (float)((double)chains * (2 * G - 3) * s / slots));
-    return tC + tA + m.scan * (G - 1);
+    const long long runs = (long long)chains * G;
+    const long long summ = G >= 2 ? (long long)chains * (2 * G - 3) : 0;
+    const float wC = (float)((runs + slots - 1) / slots);
+    const float wA = (float)((summ + slots - 1) / slots);
+    return m.c * min(s, n_c) * wC + m.a * s * wA + m.scan * (G - 1);
 }
 
 inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots,

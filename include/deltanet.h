@@ -118,7 +118,7 @@ dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tenso
  *
  * Arguments as deltanet_fwd, without cu_seqlens.  Supported: dense batches,
  * bf16 q/k/v/out, d_k = d_v = 128, chunk_size 64, and
- * B * ceil(T / 64) * H <= 6144 (chunk, head) pairs; larger problems return
+ * B * ceil(T / 64) * H <= 3072 (chunk, head) pairs; larger problems return
  * DN_ERR_WORKSPACE, other shapes or dtypes DN_ERR_UNSUPPORTED / _INVALID_ARG.
  * Outputs must not overlap inputs (not checked here).  Each (sequence, head)
  * runs as one run of chunks (no split across SMs).

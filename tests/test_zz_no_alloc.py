@@ -45,8 +45,8 @@ def test_noalloc_matches_allocating_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    q = torch.zeros((1, 64 * 6145, 1, 128), dtype=torch.bfloat16, device=DEV)
-    b = torch.zeros((1, 64 * 6145, 1), device=DEV)
+    q = torch.zeros((1, 64 * 3073, 1, 128), dtype=torch.bfloat16, device=DEV)
+    b = torch.zeros((1, 64 * 3073, 1), device=DEV)
     with pytest.raises(dn.DeltaNetError) as e:
         _lib.deltanet_fwd_noalloc(q, q, q, b)
     assert e.value.status == _lib.DN_ERR_WORKSPACE
