@@ -227,6 +227,58 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         : "memory");
 }
 
+// 16 lanes x 8 columns starting at taddr (lane, column), in the mma fragment
+// layout: thread t receives rows t/4 and t/4 + 8, columns 2 (t % 4) and + 1:
+//   r[0] (t/4, 2(t%4)), r[1] (t/4, 2(t%4)+1), r[2] (t/4+8, 2(t%4)), r[3] (t/4+8, 2(t%4)+1).
+// Does not wait: follow with tmem_wait_ld() before using the registers.
+__device__ __forceinline__ void tmem_ld16x256(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Four 8 x 8 bf16 matrices, each given in the mma fragment layout (thread t holds
+// row t/4, columns 2 (t%4), +1 of every matrix), stored transposed: row j of
+// matrix i goes to the 16 bytes at the address supplied by thread 8 i + j.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr_row, uint32_t r0, uint32_t r1, uint32_t r2,
+                                                  uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr_row),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
+// Zeroes 32 consecutive 32-bit TMEM columns of this thread's lane; waits for completion.
+__device__ __forceinline__ void tmem_zero32(uint32_t taddr) {
+    asm volatile(
+        "{\n .reg .b32 z;\n mov.b32 z, 0;\n"
+        " tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z,z};\n"
+        " tcgen05.wait::st.sync.aligned;\n}\n" ::"r"(taddr)
+        : "memory");
+}
+// Waits for four phases, testing all four back to back first.
+__device__ __forceinline__ bool mbar_wait4(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, uint64_t* c,
+                                           uint32_t pc, uint64_t* d, uint32_t pd, volatile int* abort) {
+    const bool ra = mbar_try_wait(a, pa);
+    const bool rb = mbar_try_wait(b, pb);
+    const bool rc = mbar_try_wait(c, pc);
+    const bool rd = mbar_try_wait(d, pd);
+    if (ra && rb && rc && rd) return true;
+    return (ra || mbar_wait(a, pa, abort)) && (rb || mbar_wait(b, pb, abort)) && (rc || mbar_wait(c, pc, abort)) &&
+           (rd || mbar_wait(d, pd, abort));
+}
+// Waits for three phases, testing all three back to back first.
+__device__ __forceinline__ bool mbar_wait3(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, uint64_t* c,
+                                           uint32_t pc, volatile int* abort) {
+    const bool ra = mbar_try_wait(a, pa);
+    const bool rb = mbar_try_wait(b, pb);
+    const bool rc = mbar_try_wait(c, pc);
+    if (ra && rb && rc) return true;
+    return (ra || mbar_wait(a, pa, abort)) && (rb || mbar_wait(b, pb, abort)) && (rc || mbar_wait(c, pc, abort));
+}
+
 // 16 consecutive 32-bit TMEM columns of this thread's lane; waits for completion.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
