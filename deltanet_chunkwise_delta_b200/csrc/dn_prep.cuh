@@ -10,7 +10,9 @@
 // and stores T_r and P_r as two bf16 64 x 64 tiles (16 KB per unit, T first)
 // whose rows are 128 bytes with the 128-byte swizzle: exactly the
 // shared-memory layout in which the chain kernel uses T^T and P^T as
-// tensor-core operands (it copies each tile in with one bulk copy).
+// tensor-core operands (it copies each tile in with one bulk copy).  Both tiles
+// are built in shared memory (in scratch space that is free at that point of
+// the unit) and written out with one bulk copy each.
 // W_r = T_r K_r and U_r = T_r V_r are formed later, next to the state chain.
 //
 // The 64 x 64 solve is blocked in 16 x 16 blocks: N = (I + A)^{-1} with
@@ -56,8 +58,8 @@ struct PrepSmem {
     static constexpr int OFF_QK = 0;                              // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127]
     static constexpr int OFF_A = 32768;                           // 10 blocks of A = B L
     static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N
-    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 6 staging blocks
-    static constexpr int OFF_BETA = OFF_X + 6 * kBlkFloats * 4;   // 2 x 64 step sizes
+    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 6 staging blocks; P tile staging
+    static constexpr int OFF_BETA = OFF_X + 8192;                 // 2 x 64 step sizes
     static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE
     static constexpr int OFF_MISC = OFF_BAR + 16;                 // TMEM address, abort flag
     static constexpr int USED = OFF_MISC + 16;
@@ -181,6 +183,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         DN_TRP(it_, 0);
         const bool got = sm100::mbar_wait(&bars[0], it_ & 1, abort_flag);
         cp_async_wait<0>();
+        if (tid == 0) sm100::bulk_wait_read0();  // the previous T copy has read the A blocks
         if (__syncthreads_or(!got)) break;
         in_flight = false;
         DN_TRP(it_, 1);
@@ -234,8 +237,9 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                     }
                 }
             } else {
-                // P = (Q K^T) o M_c, inclusive: bf16 row i of the unit's P tile
-                uint8_t* pg = p.wsT + (size_t)u * kUnitBytes + 8192;
+                // P = (Q K^T) o M_c, inclusive: bf16 row i of the unit's P tile, staged in
+                // the X blocks (free until the off-diagonal solve)
+                uint8_t* ps = smem + L::OFF_X;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
                     float x[8];
@@ -246,12 +250,17 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                     w.y = sm100::pack_bf16(x[2], x[3]);
                     w.z = sm100::pack_bf16(x[4], x[5]);
                     w.w = sm100::pack_bf16(x[6], x[7]);
-                    *reinterpret_cast<uint4*>(pg + sm100::swz128(i, 8 * c8)) = w;
+                    *reinterpret_cast<uint4*>(ps + sm100::swz128(i, 8 * c8)) = w;
                 }
+                sm100::fence_async_smem();
             }
         }
         sm100::tc_fence_before();
         __syncthreads();
+        if (tid == 0) {
+            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes + 8192, smem + L::OFF_X, 8192);
+            sm100::bulk_commit();
+        }
         DN_TRP(it_, 2);
         // diagonal block `warp` of N = (I + A)^{-1}: one column per lane (lanes 16-31
         // repeat 0-15), right-looking: once x_j is final it updates every later row.
@@ -288,6 +297,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                 for (int i = 0; i < 16; ++i) Nb[i * kBlkLd + c] = x[i];
             }
         }
+        if (tid == 0) sm100::bulk_wait_read0();  // the P copy has read the X blocks
         __syncthreads();
         DN_TRP(it_, 3);
         // off-diagonal blocks N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj; the products that
@@ -334,10 +344,11 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             __syncthreads();
         }
         DN_TRP(it_, 4);
-        // T = N diag(beta) -> bf16 tile (128-byte rows, 128-byte swizzle) in global memory
+        // T = N diag(beta) -> bf16 tile (128-byte rows, 128-byte swizzle), built in the
+        // A blocks (no longer read) and copied out in one piece
         {
             const int i = tid >> 1, hh = tid & 1, bi = i >> 4;
-            uint8_t* tg = p.wsT + (size_t)u * kUnitBytes;
+            uint8_t* tg = smem + L::OFF_A;
             float bj32[32];
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
@@ -366,8 +377,13 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                 w.w = sm100::pack_bf16(vals[6], vals[7]);
                 *reinterpret_cast<uint4*>(tg + sm100::swz128(i, j0)) = w;
             }
+            sm100::fence_async_smem();
         }
         __syncthreads();
+        if (tid == 0) {
+            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes, smem + L::OFF_A, 8192);
+            sm100::bulk_commit();
+        }
     }
     // a load issued for a unit this CTA then gave up on must land before exit
     if (in_flight) {
@@ -375,6 +391,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         sm100::mbar_wait(&bars[0], it_ & 1, &drain, 200000000ull);
     }
     cp_async_wait<0>();
+    if (tid == 0) sm100::bulk_wait0();  // the tile copies are complete
     sm100::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
