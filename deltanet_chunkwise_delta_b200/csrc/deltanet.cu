@@ -207,7 +207,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     using LP = ChainSmem<E, DK, DK, false, false, STAGES>;
     const int smemC = LC::TOTAL;
     const int smemA = LH::TOTAL > LP::TOTAL ? LH::TOTAL : LP::TOTAL;
-    const int smemS = (DK * (DK + 1) + DK * 16) * 4;
+    const int smemS = scan_smem_bytes<DK>();
     auto* kC = k_boundary<E, DK, DV, STAGES>;
     auto* kA = k_summary<E, DK, DV, STAGES>;
     auto* kS = k_scan<DK, DV>;
@@ -330,13 +330,13 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             ++launches;
         }
         if (nA > 0) { kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, tq, p); ++launches; }
-        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p); ++launches; }
+        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / kScanCols), kThreads, smemS, stream>>>(p); ++launches; }
         if (g_ev_start) cudaEventRecord(g_ev_start, stream);
         if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
         if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
     } else {
         if (nA > 0) { kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p); ++launches; }
-        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / 16), kThreads, smemS, stream>>>(p); ++launches; }
+        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / kScanCols), kThreads, smemS, stream>>>(p); ++launches; }
         if (g_ev_start) cudaEventRecord(g_ev_start, stream);
         if (nC > 0) { kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p); ++launches; }
         if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);

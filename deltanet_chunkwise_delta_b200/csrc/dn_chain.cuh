@@ -394,57 +394,85 @@ __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
 }
 
 // Segment scan: start(g+1) = P_g start(g) + H_g, start(1) = end state of
-// segment 0.  fp32; one CTA per (chain, 16 columns of the state).
+// segment 0.  fp32; one CTA per (chain, kScanCols columns of the state).  P_{g+1}
+// and the CTA's columns of H_{g+1} are prefetched (cp.async, second buffer) while
+// step g is computed; rows of P are padded by 4 floats so that a warp reading 32
+// rows as float4 hits 8 distinct 16-byte bank groups per access.
+constexpr int kScanCols = 8;
+template <int DK>
+__host__ __device__ constexpr int scan_smem_bytes() {
+    return (2 * DK * (DK + 4) + 3 * DK * kScanCols) * 4;
+}
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads) k_scan(Params p) {
     extern __shared__ __align__(16) float fsm[];
-    constexpr int PLD = DK + 1;
-    constexpr int NCOL = 16;
-    constexpr int GROUPS = kThreads / DK;       // column groups
-    constexpr int CPT = NCOL / GROUPS;          // columns per thread
-    float* Pm = fsm;                            // DK x PLD
-    float* Sm = Pm + DK * PLD;                  // DK x NCOL
+    constexpr int LD = DK + 4;
+    constexpr int GROUPS = kThreads / DK;       // column groups (threads per row)
+    constexpr int CPT = kScanCols / GROUPS;     // columns per thread
+    static_assert(CPT == 2 || CPT == 4, "columns per thread");
+    float* Pm[2] = {fsm, fsm + DK * LD};        // DK x LD, two buffers
+    float* Sm = fsm + 2 * DK * LD;              // DK x kScanCols
+    float* Hm[2] = {Sm + DK * kScanCols, Sm + 2 * DK * kScanCols};  // DK x kScanCols, two buffers
     const int tid = threadIdx.x;
     const int a = tid % DK, cg = tid / DK;
-    const int c0 = blockIdx.y * NCOL;
+    const int c0 = blockIdx.y * kScanCols;
     const int n = count_scan(p.sched);
+    // P_g and H_g's columns into buffers g % 2 (one cp.async group; an empty group
+    // past the last step)
+    auto prefetch = [&](const Item& it, int g) {
+        if (g + 1 < it.G) {
+            const float* Pg = p.wsP + (int64_t)(it.slot + g) * DK * DK;
+            float* dst = Pm[g & 1];
+            for (int e = tid; e < DK * DK / 4; e += kThreads) {
+                const int r = (4 * e) / DK, c = (4 * e) % DK;
+                cp_async16(smem_addr(dst + r * LD + c), Pg + 4 * e, 16);
+            }
+            const float* Hg = p.wsH + (int64_t)(it.slot + g) * DK * DV + c0;
+            for (int e = tid; e < DK * kScanCols / 4; e += kThreads) {
+                const int r = (4 * e) / kScanCols, c = (4 * e) % kScanCols;
+                cp_async16(smem_addr(Hm[g & 1] + 4 * e), Hg + r * DV + c, 16);
+            }
+        }
+        cp_async_commit();
+    };
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
         const Item it = item_scan(p.sched, i);
         const float* E0 = p.wsH + (int64_t)it.slot * DK * DV;
         float* out0 = p.wsS + (int64_t)it.slot * DK * DV;
-        for (int e = tid; e < DK * NCOL; e += kThreads) {
-            const int r = e / NCOL, c = e % NCOL;
+        prefetch(it, 1);
+        for (int e = tid; e < DK * kScanCols; e += kThreads) {
+            const int r = e / kScanCols, c = e % kScanCols;
             const float x = E0[r * DV + c0 + c];
             Sm[e] = x;
             out0[r * DV + c0 + c] = x;
         }
         for (int g = 1; g + 1 < it.G; ++g) {
+            prefetch(it, g + 1);
+            cp_async_wait<1>();  // P_g has landed
             __syncthreads();
-            const float* Pg = p.wsP + (int64_t)(it.slot + g) * DK * DK;
-            for (int e = tid; e < DK * DK / 4; e += kThreads) {
-                const float4 x = reinterpret_cast<const float4*>(Pg)[e];
-                const int r = (4 * e) / DK, c = (4 * e) % DK;
-                float* d = Pm + r * PLD + c;
-                d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
-            }
-            __syncthreads();
-            const float* Hg = p.wsH + (int64_t)(it.slot + g) * DK * DV;
             float acc[CPT];
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) acc[j] = Hg[a * DV + c0 + cg * CPT + j];
-            for (int b = 0; b < DK; ++b) {
-                const float pab = Pm[a * PLD + b];
+            for (int j = 0; j < CPT; ++j) acc[j] = Hm[g & 1][a * kScanCols + cg * CPT + j];
+            const float* prow = Pm[g & 1] + a * LD;
+            const float* scol = Sm + cg * CPT;
+#pragma unroll 4
+            for (int b = 0; b < DK; b += 4) {
+                const float4 pv = *reinterpret_cast<const float4*>(prow + b);
+                const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
-                for (int j = 0; j < CPT; ++j) acc[j] = fmaf(pab, Sm[b * NCOL + cg * CPT + j], acc[j]);
+                for (int e = 0; e < 4; ++e)
+#pragma unroll
+                    for (int j = 0; j < CPT; ++j) acc[j] = fmaf(pe[e], scol[(b + e) * kScanCols + j], acc[j]);
             }
-            __syncthreads();
-            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV;
+            __syncthreads();  // every thread has read S(g) and P_g
+            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV + a * DV + c0 + cg * CPT;
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
-                Sm[a * NCOL + cg * CPT + j] = acc[j];
-                outg[a * DV + c0 + cg * CPT + j] = acc[j];
+                Sm[a * kScanCols + cg * CPT + j] = acc[j];
+                outg[j] = acc[j];
             }
         }
+        cp_async_wait<0>();
         __syncthreads();
     }
 }

@@ -23,7 +23,7 @@ namespace dn {
 struct CostModel {
     float c = 1.0f;      // boundary pass, per chunk
     float a = 0.65f;     // summary pass, per chunk (no output, no Q)
-    float scan = 3.0f;   // one step of the segment scan
+    float scan = 2.0f;   // one step of the segment scan
 };
 
 struct SegChoice {
