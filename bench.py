@@ -63,13 +63,17 @@ def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
     return float(b)
 
 
+# Sources the tensor-core boundary kernel is compiled from.
+BOUNDARY_KERNEL_SOURCES = ("dn_common.cuh", "dn_sm100.cuh", "dn_tc.cuh")
+
+
 def kernel_source_digest() -> str:
-    """Digest of the CUDA sources, so that a stored ncu traffic figure is only
-    used for the kernels it was measured on."""
+    """Digest of the boundary kernel's CUDA sources, so that a stored ncu
+    traffic figure is only used for the kernel it was measured on."""
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "deltanet_chunkwise_delta_b200", "csrc")
-    for name in sorted(os.listdir(src)):
+    for name in BOUNDARY_KERNEL_SOURCES:
         with open(os.path.join(src, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
