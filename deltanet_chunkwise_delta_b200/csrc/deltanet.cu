@@ -18,6 +18,7 @@
 #include "dn_prep.cuh"
 #include "dn_sched.cuh"
 #include "dn_tc.cuh"
+#include "dn_tc_sum.cuh"
 
 using namespace dn;
 
@@ -207,24 +208,30 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     using LP = ChainSmem<E, DK, DK, false, false, STAGES>;
     const int smemC = LC::TOTAL;
     const int smemA = LH::TOTAL > LP::TOTAL ? LH::TOTAL : LP::TOTAL;
-    const int smemS = scan_smem_bytes<DK>();
+    const int smemS8 = scan_smem_bytes<DK, 8>(), smemS16 = scan_smem_bytes<DK, 16>();
     auto* kC = k_boundary<E, DK, DV, STAGES>;
     auto* kA = k_summary<E, DK, DV, STAGES>;
-    auto* kS = k_scan<DK, DV>;
+    auto* kS8 = k_scan<DK, DV, 8>;
+    auto* kS16 = k_scan<DK, DV, 16>;
     auto* kCt = tc::k_tc_chain<true>;
-    auto* kAt = tc::k_tc_chain<false>;
+    auto* kAt = tcs::k_tc_summary;
     auto* kPrep = k_ut_prep;
     constexpr int smemPrep = PrepSmem::TOTAL;
     dn_status st;
     if (kTc) {
         if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
-        if ((st = set_smem(kAt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
+        if ((st = set_smem(kAt, dev, tcs::SMEM_BYTES)) != DN_OK) return st;
         if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
+        // several pre-pass CTAs share an SM: ask for the largest shared-memory carveout
+        if (cudaFuncSetAttribute(kPrep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            return DN_ERR_CUDA;
     } else {
         if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
         if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
     }
-    if ((st = set_smem(kS, dev, smemS)) != DN_OK) return st;
+    if ((st = set_smem(kS8, dev, smemS8)) != DN_OK) return st;
+    if ((st = set_smem(kS16, dev, smemS16)) != DN_OK) return st;
     CUtensorMap tq, tk, tv, to;
     if (kTc) {
         const int64_t Bq = d.varlen ? 1 : d.B;
@@ -251,7 +258,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         slots = chains * (G - 1);
         if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
         nC = chains * G;
-        nA = G >= 2 ? chains * (2 * G - 3) : 0;
+        nA = G >= 2 ? chains * (G - 1) : 0;
         nScan = G >= 2 ? chains : 0;
     } else {
         if (forced_s > 0) {
@@ -261,7 +268,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             slots = std::min<int64_t>(kAutoMaxSlots, d.H * (n_c_max + d.N));
         }
         nC = chains + slots;
-        nA = 2 * slots;
+        nA = slots;
         nScan = std::min<int64_t>(chains, slots);
     }
     // workspace layout
@@ -321,6 +328,13 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         g_last_G = -1;
         g_last_s = -1;
     }
+    // one CTA per (chain, 8 state columns); 16 columns when that needs more than one wave
+    auto launch_scan = [&]() {
+        if (nScan * (DV / 8) <= sms)
+            kS8<<<dim3((unsigned)nScan, DV / 8), scan_threads<DK, 8>(), smemS8, stream>>>(p);
+        else
+            kS16<<<dim3((unsigned)nScan, DV / 16), scan_threads<DK, 16>(), smemS16, stream>>>(p);
+    };
     int launches = d.varlen ? 1 : 0;
     if (kTc) {
         const int64_t units = chunk_ub * d.H;
@@ -329,14 +343,14 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
             ++launches;
         }
-        if (nA > 0) { kAt<<<(unsigned)nA, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, tq, p); ++launches; }
-        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / kScanCols), kThreads, smemS, stream>>>(p); ++launches; }
+        if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
+        if (nScan > 0) { launch_scan(); ++launches; }
         if (g_ev_start) cudaEventRecord(g_ev_start, stream);
         if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
         if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
     } else {
         if (nA > 0) { kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p); ++launches; }
-        if (nScan > 0) { kS<<<dim3((unsigned)nScan, DV / kScanCols), kThreads, smemS, stream>>>(p); ++launches; }
+        if (nScan > 0) { launch_scan(); ++launches; }
         if (g_ev_start) cudaEventRecord(g_ev_start, stream);
         if (nC > 0) { kC<<<(unsigned)nC, kThreads, smemC, stream>>>(p); ++launches; }
         if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);

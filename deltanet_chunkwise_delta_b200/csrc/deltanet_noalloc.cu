@@ -93,7 +93,9 @@ dn_status na_setup(int dev, unsigned char** scratch) {
     if (cudaFuncSetAttribute(dn::tc::k_tc_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::tc::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             dn::PrepSmem::TOTAL) != cudaSuccess)
+                             dn::PrepSmem::TOTAL) != cudaSuccess ||
+        cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return DN_ERR_CUDA;
     g_na_scratch[dev] = static_cast<unsigned char*>(ptr);
     *scratch = static_cast<unsigned char*>(ptr);

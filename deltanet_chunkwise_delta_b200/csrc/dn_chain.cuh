@@ -20,6 +20,7 @@
 #pragma once
 
 #include "dn_common.cuh"
+#include "dn_sm100.cuh"
 #include "dn_warp_gemm.cuh"
 
 namespace dn {
@@ -385,95 +386,129 @@ __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
         int mode;
         const Item it = item_A(p.sched, i, mode);
-        if (mode == kModeP)
+        if (mode == kModeHP) {
+            // both maps of the segment, one after the other
+            run_segment<E, DK, DV, true, false, STAGES>(p, it, kModeH, smem);
+            __syncthreads();
+            run_segment<E, DK, DK, false, false, STAGES>(p, it, kModeP, smem);
+        } else if (mode == kModeP) {
             run_segment<E, DK, DK, false, false, STAGES>(p, it, mode, smem);
-        else
+        } else {
             run_segment<E, DK, DV, true, false, STAGES>(p, it, mode, smem);
+        }
         __syncthreads();
     }
 }
 
 // Segment scan: start(g+1) = P_g start(g) + H_g, start(1) = end state of
-// segment 0.  fp32; one CTA per (chain, kScanCols columns of the state).  P_{g+1}
-// and the CTA's columns of H_{g+1} are prefetched (cp.async, second buffer) while
-// step g is computed; rows of P are padded by 4 floats so that a warp reading 32
-// rows as float4 hits 8 distinct 16-byte bank groups per access.
-constexpr int kScanCols = 8;
-template <int DK>
+// segment 0.  fp32; one CTA per (chain, COLS columns of the state), 4 columns
+// per thread.  P_{g+1} is prefetched by one bulk copy into the second buffer,
+// and each thread's H_{g+1} values into registers, while step g is computed.
+// P is stored unpadded and the CTA's columns of the state transposed (one
+// row of DK per column); lane a starts its sweep over k at 4 (a mod 8), so that
+// both the float4 reads of P's rows and those of the state's columns fall into
+// 8 distinct 16-byte bank groups per quarter-warp.  COLS is 16 when 8-column
+// CTAs would need more than one wave.
+template <int DK, int COLS>
+__host__ __device__ constexpr int scan_threads() { return DK * COLS / 4; }
+template <int DK, int COLS>
 __host__ __device__ constexpr int scan_smem_bytes() {
-    return (2 * DK * (DK + 4) + 3 * DK * kScanCols) * 4;
+    return (2 * DK * DK + DK * COLS) * 4 + 32;
 }
-template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads) k_scan(Params p) {
-    extern __shared__ __align__(16) float fsm[];
-    constexpr int LD = DK + 4;
-    constexpr int GROUPS = kThreads / DK;       // column groups (threads per row)
-    constexpr int CPT = kScanCols / GROUPS;     // columns per thread
-    static_assert(CPT == 2 || CPT == 4, "columns per thread");
-    float* Pm[2] = {fsm, fsm + DK * LD};        // DK x LD, two buffers
-    float* Sm = fsm + 2 * DK * LD;              // DK x kScanCols
-    float* Hm[2] = {Sm + DK * kScanCols, Sm + 2 * DK * kScanCols};  // DK x kScanCols, two buffers
+template <int DK, int DV, int COLS>
+__global__ void __launch_bounds__(DK * COLS / 4) k_scan(Params p) {
+    extern __shared__ __align__(128) float fsm[];
+    constexpr int NT = DK * COLS / 4;
+    constexpr uint32_t kPBytes = (uint32_t)DK * DK * 4u;
+    constexpr uint32_t kPiece = kPBytes < 16384u ? kPBytes : 16384u;
+    static_assert((DK & (DK - 1)) == 0 && DK >= 32, "rows");
+    float* St = fsm + 2 * DK * DK;                          // COLS x DK (state columns)
+    auto Pm = [&](int b) { return fsm + b * DK * DK; };     // DK x DK, two buffers
+    uint64_t* bars = reinterpret_cast<uint64_t*>(St + DK * COLS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2);
     const int tid = threadIdx.x;
-    const int a = tid % DK, cg = tid / DK;
-    const int c0 = blockIdx.y * kScanCols;
+    const int a = tid % DK, c = 4 * (tid / DK);            // state row, first of 4 columns
+    const int c0 = blockIdx.y * COLS;
+    const int rot = 4 * (a & 7);
     const int n = count_scan(p.sched);
-    // P_g and H_g's columns into buffers g % 2 (one cp.async group; an empty group
-    // past the last step)
+    if (tid == 0) {
+        sm100::mbar_init(&bars[0], 1);
+        sm100::mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        sm100::mbar_fence_init();
+    }
+    __syncthreads();
+    // per buffer (bit b): parity of its next completion, and a copy in flight into
+    // it (at most one: a buffer is refilled only after its last step was computed)
+    uint32_t phase = 0, pending = 0;
+    float4 hn = make_float4(0.f, 0.f, 0.f, 0.f);
+    // P_g into buffer g % 2, this thread's 4 values of H_g into hn
     auto prefetch = [&](const Item& it, int g) {
-        if (g + 1 < it.G) {
-            const float* Pg = p.wsP + (int64_t)(it.slot + g) * DK * DK;
-            float* dst = Pm[g & 1];
-            for (int e = tid; e < DK * DK / 4; e += kThreads) {
-                const int r = (4 * e) / DK, c = (4 * e) % DK;
-                cp_async16(smem_addr(dst + r * LD + c), Pg + 4 * e, 16);
-            }
-            const float* Hg = p.wsH + (int64_t)(it.slot + g) * DK * DV + c0;
-            for (int e = tid; e < DK * kScanCols / 4; e += kThreads) {
-                const int r = (4 * e) / kScanCols, c = (4 * e) % kScanCols;
-                cp_async16(smem_addr(Hm[g & 1] + 4 * e), Hg + r * DV + c, 16);
-            }
+        if (g + 1 >= it.G) return;
+        const int b = g & 1;
+        pending |= 1u << b;
+        if (tid == 0) {
+            const uint8_t* Pg = reinterpret_cast<const uint8_t*>(p.wsP + (int64_t)(it.slot + g) * DK * DK);
+            uint8_t* dst = reinterpret_cast<uint8_t*>(Pm(b));
+            sm100::mbar_expect_tx(&bars[b], kPBytes);
+            for (uint32_t o = 0; o < kPBytes; o += kPiece) sm100::bulk_load(dst + o, Pg + o, kPiece, &bars[b]);
         }
-        cp_async_commit();
+        hn = *reinterpret_cast<const float4*>(p.wsH + (int64_t)(it.slot + g) * DK * DV + (int64_t)a * DV + c0 + c);
     };
-    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < n; i += gridDim.x) {
         const Item it = item_scan(p.sched, i);
         const float* E0 = p.wsH + (int64_t)it.slot * DK * DV;
         float* out0 = p.wsS + (int64_t)it.slot * DK * DV;
         prefetch(it, 1);
-        for (int e = tid; e < DK * kScanCols; e += kThreads) {
-            const int r = e / kScanCols, c = e % kScanCols;
-            const float x = E0[r * DV + c0 + c];
-            Sm[e] = x;
-            out0[r * DV + c0 + c] = x;
+        for (int e = tid; e < DK * COLS; e += NT) {
+            const int r = e % DK, cc = e / DK;
+            const float x = E0[r * DV + c0 + cc];
+            St[cc * DK + r] = x;
+            out0[r * DV + c0 + cc] = x;
         }
         for (int g = 1; g + 1 < it.G; ++g) {
+            float acc[4] = {hn.x, hn.y, hn.z, hn.w};
             prefetch(it, g + 1);
-            cp_async_wait<1>();  // P_g has landed
-            __syncthreads();
-            float acc[CPT];
-#pragma unroll
-            for (int j = 0; j < CPT; ++j) acc[j] = Hm[g & 1][a * kScanCols + cg * CPT + j];
-            const float* prow = Pm[g & 1] + a * LD;
-            const float* scol = Sm + cg * CPT;
+            const int b = g & 1;
+            const bool landed = sm100::mbar_wait(&bars[b], (phase >> b) & 1u, abort_flag);
+            if (landed) {
+                phase ^= 1u << b;
+                pending &= ~(1u << b);
+            }
+            if (__syncthreads_or(!landed)) {  // also: S(g) is written
+                ok = false;
+                break;
+            }
+            const float* prow = Pm(b) + a * DK;
+            const float* scol = St + c * DK;
 #pragma unroll 4
-            for (int b = 0; b < DK; b += 4) {
-                const float4 pv = *reinterpret_cast<const float4*>(prow + b);
-                const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
+            for (int k0 = 0; k0 < DK; k0 += 4) {
+                const int k = (k0 + rot) & (DK - 1);
+                const float4 pv = *reinterpret_cast<const float4*>(prow + k);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-#pragma unroll
-                    for (int j = 0; j < CPT; ++j) acc[j] = fmaf(pe[e], scol[(b + e) * kScanCols + j], acc[j]);
+                for (int j = 0; j < 4; ++j) {
+                    const float4 sv = *reinterpret_cast<const float4*>(scol + j * DK + k);
+                    acc[j] = fmaf(pv.x, sv.x, acc[j]);
+                    acc[j] = fmaf(pv.y, sv.y, acc[j]);
+                    acc[j] = fmaf(pv.z, sv.z, acc[j]);
+                    acc[j] = fmaf(pv.w, sv.w, acc[j]);
+                }
             }
             __syncthreads();  // every thread has read S(g) and P_g
-            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV + a * DV + c0 + cg * CPT;
+            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV + (int64_t)a * DV + c0 + c;
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) {
-                Sm[a * kScanCols + cg * CPT + j] = acc[j];
-                outg[j] = acc[j];
-            }
+            for (int j = 0; j < 4; ++j) St[(c + j) * DK + a] = acc[j];
+            *reinterpret_cast<float4*>(outg) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
-        cp_async_wait<0>();
         __syncthreads();
+    }
+    // copies still in flight must land before the CTA exits (also after a time-out)
+    if (tid == 0) {
+        volatile int drain = 0;
+        for (int b = 0; b < 2; ++b)
+            if ((pending >> b) & 1u) sm100::mbar_wait(&bars[b], (phase >> b) & 1u, &drain, 200000000ull);
+        if (*abort_flag) atomicExch(p.err, kErrTimeout);
     }
 }
 

@@ -40,6 +40,7 @@ enum SegMode : int {
     kModeEnd = 1,    // first segment: end state from the true initial state (no output)
     kModeH = 2,      // zero-start local writes H_g of a segment
     kModeP = 3,      // transition product P_g of a segment (state is d_k x d_k, starts at I)
+    kModeHP = 4,     // both maps of a segment, H_g and P_g, in one item
 };
 
 // How work items are enumerated.
@@ -101,7 +102,7 @@ __device__ __forceinline__ int count_C(const Sched& s) {
     return s.list ? s.counts[0] : s.B * s.H * s.G;
 }
 __device__ __forceinline__ int count_A(const Sched& s) {
-    return s.list ? s.counts[1] : (s.G >= 2 ? s.B * s.H * (2 * s.G - 3) : 0);
+    return s.list ? s.counts[1] : (s.G >= 2 ? s.B * s.H * (s.G - 1) : 0);
 }
 __device__ __forceinline__ int count_scan(const Sched& s) {
     return s.list ? s.counts[2] : (s.G >= 2 ? s.B * s.H : 0);
@@ -114,7 +115,7 @@ __device__ __forceinline__ Item item_C(const Sched& s, int i) {
     return it;
 }
 
-// Summary items: per chain, [End(g=0), H(1), P(1), H(2), P(2), ..., H(G-2), P(G-2)].
+// Summary items: per chain, [End(g=0), HP(1), HP(2), ..., HP(G-2)].
 __device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
     Item it;
     if (s.list) {
@@ -123,15 +124,10 @@ __device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
         it.g &= 0xffff;
         return it;
     }
-    const int per = 2 * s.G - 3;
+    const int per = s.G - 1;
     const int chain = i / per, r = i % per;
-    if (r == 0) {
-        mode = kModeEnd;
-        dense_chain_item(s, chain, 0, it);
-    } else {
-        mode = ((r - 1) & 1) ? kModeP : kModeH;
-        dense_chain_item(s, chain, 1 + (r - 1) / 2, it);
-    }
+    mode = r == 0 ? kModeEnd : kModeHP;
+    dense_chain_item(s, chain, r, it);
     return it;
 }
 

@@ -19,10 +19,12 @@
 // A = B L; each diagonal block by forward substitution (one warp per block,
 // one column per lane, fp32), then N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj in
 // order of i - j with tf32 mma.sync, and T = N B.
-// One CTA of 4 warps per (chunk, head) at a time, three CTAs per SM, so the
-// latency of the solve is hidden by parallelism across chunks.  The q/k tile
-// of the next unit is loaded by TMA as soon as this unit's product has read
-// the current one.
+// One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM, so the
+// latency of the solve is hidden by parallelism across chunks.  A CTA's shared
+// memory is one 32 KB region that holds the unit's q/k tile until the product
+// has read it, and then the solve's blocks, the P tile (staged where N is
+// written later) and the T tile (staged where A was); the next unit's tile is
+// loaded once the T copy has read its staging.
 #pragma once
 
 #include "dn_chain.cuh"
@@ -49,23 +51,27 @@ static __device__ unsigned long long g_dn_trace_prep[16 * 8];
 #endif
 
 constexpr int kPrepThreads = 128;
-constexpr int kPrepCtasPerSm = 3;
+constexpr int kPrepCtasPerSm = 6;
 constexpr int kBlkLd = 20;  // fp32 16 x 16 blocks, 16-byte aligned rows
 constexpr int kBlkFloats = 16 * kBlkLd;
 
-// Shared memory of the pre-pass (byte offsets from a 1024-aligned base).
+// Shared memory of the pre-pass (byte offsets from a 1024-aligned base).  The
+// region [0, 32 KB) holds [Q d0-63 | K d0-63 | Q d64-127 | K d64-127] while the
+// q/k tile is loaded and read by the product, then the blocks of the solve:
 struct PrepSmem {
-    static constexpr int OFF_QK = 0;                              // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127]
-    static constexpr int OFF_A = 32768;                           // 10 blocks of A = B L
-    static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N
-    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 6 staging blocks; P tile staging
-    static constexpr int OFF_BETA = OFF_X + 8192;                 // 2 x 64 step sizes
+    static constexpr int OFF_QK = 0;
+    static constexpr int OFF_A = 0;                               // 10 blocks of A = B L; later the T tile
+    static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N; before them the P tile
+    static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 5 staging blocks of the off-diagonal solve
+    static constexpr int OFF_BETA = 32768;                        // 2 x 64 step sizes
     static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE
     static constexpr int OFF_MISC = OFF_BAR + 16;                 // TMEM address, abort flag
     static constexpr int USED = OFF_MISC + 16;
     static constexpr int TOTAL = USED + 1024;                     // slack for 1024-byte alignment
 };
-static_assert(PrepSmem::TOTAL * kPrepCtasPerSm <= 227 * 1024, "pre-pass shared memory");
+static_assert(PrepSmem::OFF_X + 5 * kBlkFloats * 4 <= PrepSmem::OFF_BETA, "solve blocks fit the q/k region");
+static_assert(PrepSmem::OFF_N + 8192 <= PrepSmem::OFF_X, "P staging fits the N blocks");
+static_assert((PrepSmem::TOTAL + 1024) * kPrepCtasPerSm <= 228 * 1024, "pre-pass shared memory");
 
 __device__ __forceinline__ int blk_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
 
@@ -183,7 +189,6 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         DN_TRP(it_, 0);
         const bool got = sm100::mbar_wait(&bars[0], it_ & 1, abort_flag);
         cp_async_wait<0>();
-        if (tid == 0) sm100::bulk_wait_read0();  // the previous T copy has read the A blocks
         if (__syncthreads_or(!got)) break;
         in_flight = false;
         DN_TRP(it_, 1);
@@ -198,59 +203,65 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             sm100::umma_commit(&bars[1]);
         }
         const bool gdone = sm100::mbar_wait(&bars[1], it_ & 1, abort_flag);
+        // the product has read the q/k tile: the region now takes the solve's blocks
         if (__syncthreads_or(!gdone)) break;
         sm100::tc_fence_after();
-        // the product has read the q/k tile: load the next unit's
-        const int un = u + gridDim.x;
-        if (un < units) {
-            issue(un, bb ^ 1);
-            in_flight = true;
-        }
         const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + bb * kChunk;
         {
             const int i = 32 * (warp & 1) + lane;  // row of Q K^T (warps 0, 1) or K K^T (warps 2, 3)
-            uint32_t v[64];
-            sm100::tmem_ld64(tmem + ((uint32_t)(32 * warp) << 16), v);
+            const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
             if (warp >= 2) {
                 // A = B L, blocked: row i of block row bi; blocks left of the diagonal
                 // row-major, the diagonal block transposed (for the column sweeps)
                 const int bi = i >> 4, ri = i & 15;
                 const float bta = betas[i];
 #pragma unroll
-                for (int bj = 0; bj < 4; ++bj) {
-                    if (bj > bi) continue;
-                    float* blk = Ablk + blk_index(bi, bj) * kBlkFloats;
-                    if (bj < bi) {
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t v[32];
+                    sm100::tmem_ld32(taddr + 32 * hc, v);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            float4 f;
-                            f.x = bta * __uint_as_float(v[16 * bj + 4 * q4 + 0]);
-                            f.y = bta * __uint_as_float(v[16 * bj + 4 * q4 + 1]);
-                            f.z = bta * __uint_as_float(v[16 * bj + 4 * q4 + 2]);
-                            f.w = bta * __uint_as_float(v[16 * bj + 4 * q4 + 3]);
-                            *reinterpret_cast<float4*>(blk + ri * kBlkLd + 4 * q4) = f;
+                    for (int bh = 0; bh < 2; ++bh) {
+                        const int bj = 2 * hc + bh;
+                        if (bj > bi) continue;
+                        float* blk = Ablk + blk_index(bi, bj) * kBlkFloats;
+                        if (bj < bi) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                float4 f;
+                                f.x = bta * __uint_as_float(v[16 * bh + 4 * q4 + 0]);
+                                f.y = bta * __uint_as_float(v[16 * bh + 4 * q4 + 1]);
+                                f.z = bta * __uint_as_float(v[16 * bh + 4 * q4 + 2]);
+                                f.w = bta * __uint_as_float(v[16 * bh + 4 * q4 + 3]);
+                                *reinterpret_cast<float4*>(blk + ri * kBlkLd + 4 * q4) = f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c)
+                                blk[c * kBlkLd + ri] = c < ri ? bta * __uint_as_float(v[16 * bh + c]) : 0.f;
                         }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            blk[c * kBlkLd + ri] = c < ri ? bta * __uint_as_float(v[16 * bj + c]) : 0.f;
                     }
                 }
             } else {
-                // P = (Q K^T) o M_c, inclusive: bf16 row i of the unit's P tile, staged in
-                // the X blocks (free until the off-diagonal solve)
-                uint8_t* ps = smem + L::OFF_X;
+                // P = (Q K^T) o M_c, inclusive: bf16 row i of the unit's P tile, staged
+                // where the N blocks are written after the diagonal solve
+                uint8_t* ps = smem + L::OFF_N;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    float x[8];
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t v[32];
+                    sm100::tmem_ld32(taddr + 32 * hc, v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = (8 * c8 + e <= i) ? __uint_as_float(v[8 * c8 + e]) : 0.f;
-                    uint4 w;
-                    w.x = sm100::pack_bf16(x[0], x[1]);
-                    w.y = sm100::pack_bf16(x[2], x[3]);
-                    w.z = sm100::pack_bf16(x[4], x[5]);
-                    w.w = sm100::pack_bf16(x[6], x[7]);
-                    *reinterpret_cast<uint4*>(ps + sm100::swz128(i, 8 * c8)) = w;
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        const int col = 32 * hc + 8 * c8;
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] = (col + e <= i) ? __uint_as_float(v[8 * c8 + e]) : 0.f;
+                        uint4 w;
+                        w.x = sm100::pack_bf16(x[0], x[1]);
+                        w.y = sm100::pack_bf16(x[2], x[3]);
+                        w.z = sm100::pack_bf16(x[4], x[5]);
+                        w.w = sm100::pack_bf16(x[6], x[7]);
+                        *reinterpret_cast<uint4*>(ps + sm100::swz128(i, col)) = w;
+                    }
                 }
                 sm100::fence_async_smem();
             }
@@ -258,7 +269,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         sm100::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes + 8192, smem + L::OFF_X, 8192);
+            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes + 8192, smem + L::OFF_N, 8192);
             sm100::bulk_commit();
         }
         DN_TRP(it_, 2);
@@ -291,13 +302,15 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 #pragma unroll
                 for (int i = j + 2; i < 16; ++i) cur[i] = nxt[i];
             }
+            // the P copy has read its staging, which the N blocks overwrite
+            if (tid == 0) sm100::bulk_wait_read0();
+            __syncthreads();
             if (lane < 16) {
                 float* Nb = Nblk + blk_index(warp, warp) * kBlkFloats;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) Nb[i * kBlkLd + c] = x[i];
             }
         }
-        if (tid == 0) sm100::bulk_wait_read0();  // the P copy has read the X blocks
         __syncthreads();
         DN_TRP(it_, 3);
         // off-diagonal blocks N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj; the products that
@@ -305,9 +318,9 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         {
             auto A_ = [&](int i, int j) { return Ablk + blk_index(i, j) * kBlkFloats; };
             auto N_ = [&](int i, int j) { return Nblk + blk_index(i, j) * kBlkFloats; };
-            float* X = Xs + warp * kBlkFloats;          // per-warp staging
-            float* Y20 = Xs + 4 * kBlkFloats;           // shared partial sums
-            float* Y31 = Xs + 5 * kBlkFloats;
+            float* X = Xs + warp * kBlkFloats;          // per-warp staging (warps 0-2)
+            float* Y20 = Xs + 3 * kBlkFloats;           // shared partial sums
+            float* Y31 = Xs + 4 * kBlkFloats;
             float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             float y30[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             // phase 1: N_{i+1,i} for i = 0, 1, 2 (warps 0-2); warp 3: A20 N00 and A31 N11
@@ -344,20 +357,19 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             __syncthreads();
         }
         DN_TRP(it_, 4);
-        // T = N diag(beta) -> bf16 tile (128-byte rows, 128-byte swizzle), built in the
-        // A blocks (no longer read) and copied out in one piece
+        // T = N diag(beta) -> bf16 tile (128-byte rows, 128-byte swizzle), built where
+        // the A blocks were and copied out in one piece.  Thread: row i (consecutive
+        // over a warp's lanes, so that a quarter-warp's 16-byte accesses fall into 8
+        // distinct bank groups), half hh of the columns.
         {
-            const int i = tid >> 1, hh = tid & 1, bi = i >> 4;
+            const int i = 32 * (warp & 1) + lane, hh = warp >> 1, bi = i >> 4;
             uint8_t* tg = smem + L::OFF_A;
-            float bj32[32];
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-                const float4 f = *reinterpret_cast<const float4*>(betas + 32 * hh + 4 * q4);
-                bj32[4 * q4] = f.x; bj32[4 * q4 + 1] = f.y; bj32[4 * q4 + 2] = f.z; bj32[4 * q4 + 3] = f.w;
-            }
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int j0 = 32 * hh + 8 * cc, bj = j0 >> 4;
+                const float4 b0 = *reinterpret_cast<const float4*>(betas + j0);
+                const float4 b1 = *reinterpret_cast<const float4*>(betas + j0 + 4);
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                 float vals[8];
                 if (bj <= bi) {
                     const float* nr = Nblk + blk_index(bi, bj) * kBlkFloats + (i & 15) * kBlkLd + (j0 & 15);
@@ -365,7 +377,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                     const float4 f1 = *reinterpret_cast<const float4*>(nr + 4);
                     const float nv[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) vals[e] = (j0 + e <= i) ? nv[e] * bj32[8 * cc + e] : 0.f;
+                    for (int e = 0; e < 8; ++e) vals[e] = (j0 + e <= i) ? nv[e] * bv[e] : 0.f;
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) vals[e] = 0.f;
@@ -380,10 +392,19 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             sm100::fence_async_smem();
         }
         __syncthreads();
+        // copy T out; once the copy has read its staging the region takes the next
+        // unit's q/k tile
+        const int un = u + gridDim.x;
         if (tid == 0) {
             sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes, smem + L::OFF_A, 8192);
             sm100::bulk_commit();
+            sm100::bulk_wait_read0();
         }
+        if (un < units) {
+            issue(un, bb ^ 1);
+            in_flight = true;
+        }
+        DN_TRP(it_, 5);
     }
     // a load issued for a unit this CTA then gave up on must land before exit
     if (in_flight) {

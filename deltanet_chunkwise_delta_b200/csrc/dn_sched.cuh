@@ -5,7 +5,7 @@
 // the maps (P_g, H_g) of every run before them ("Context Parallelism for
 // DeltaNet", section 3: the chunk update is affine in the incoming state, so
 // runs compose).  Work per call:
-//   summary pass   run 0: end state; runs 1..G-2: H_g and P_g (two items)
+//   summary pass   run 0: end state; runs 1..G-2: H_g and P_g (one item each)
 //   segment scan   start states of runs 1..G-1
 //   boundary pass  every run from its start state: outputs, final state
 // The run length s minimises a simple model of the call's duration, with
@@ -22,7 +22,7 @@ namespace dn {
 
 struct CostModel {
     float c = 1.0f;      // boundary pass, per chunk
-    float a = 0.65f;     // summary pass, per chunk (no output, no Q)
+    float a = 0.9f;      // summary pass, per chunk (two chains, no output, no Q)
     float scan = 2.0f;   // one step of the segment scan
 };
 
@@ -36,7 +36,7 @@ __host__ __device__ inline float dense_cost(const CostModel& m, int chains, int 
                                             int slots) {
     const int G = n_c > 0 ? (n_c + s - 1) / s : 1;
     const long long runs = (long long)chains * G;
-    const long long summ = G >= 2 ? (long long)chains * (2 * G - 3) : 0;
+    const long long summ = G >= 2 ? (long long)chains * (G - 1) : 0;
     const float wC = (float)((runs + slots - 1) / slots);
     const float wA = (float)((summ + slots - 1) / slots);
     return m.c * min(s, n_c) * wC + m.a * s * wA + m.scan * (G - 1);
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
                 const int c = nc[n];
                 const int G = c > 0 ? (c + s - 1) / s : 1;
                 extra += G - 1;
-                if (G >= 2) wA += 2 * G - 3;
+                if (G >= 2) wA += G - 1;
                 gmax = max(gmax, G);
             }
             for (int o = 16; o > 0; o >>= 1) {
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
         if (pos < N) {
             const int c = nc[order[pos]];
             const int G = c > 0 ? (c + s - 1) / s : 1;
-            v = make_int4(H * G, G >= 2 ? H * (2 * G - 3) : 0, G >= 2 ? H : 0, H * (G - 1));
+            v = make_int4(H * G, G >= 2 ? H * (G - 1) : 0, G >= 2 ? H : 0, H * (G - 1));
         }
         int4 inc = v;
         for (int o = 1; o < 32; o <<= 1) {
@@ -264,18 +264,9 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
                 it.cbase = cumchunks[n] + g * s;
                 itemsC[o.x + h * G + g] = it;
                 if (G >= 2 && g + 1 < G) {
-                    const int abase = o.y + h * (2 * G - 3);
-                    if (g == 0) {
-                        Item x = it;
-                        x.g = 0 | (kModeEnd << 16);
-                        itemsA[abase] = x;
-                    } else {
-                        Item x = it;
-                        x.g = g | (kModeH << 16);
-                        itemsA[abase + 1 + 2 * (g - 1)] = x;
-                        x.g = g | (kModeP << 16);
-                        itemsA[abase + 2 + 2 * (g - 1)] = x;
-                    }
+                    Item x = it;
+                    x.g = g | ((g == 0 ? kModeEnd : kModeHP) << 16);
+                    itemsA[o.y + h * (G - 1) + g] = x;
                 }
                 if (G >= 2 && g == 0) itemsScan[o.z + h] = it;
             }
