@@ -193,6 +193,23 @@ dn_status make_token_map(CUtensorMap* m, const void* base, int64_t B, int64_t T,
     return r == CUDA_SUCCESS ? DN_OK : DN_ERR_UNSUPPORTED;
 }
 
+// 2-D map over the segment transition products P_g (rows of DK fp32), boxes of
+// 32 columns x DK rows with the 128-byte swizzle (the segment scan's operand layout).
+dn_status make_p_map(CUtensorMap* m, const void* base, int64_t rows, int dk) {
+    std::memset(m, 0, sizeof *m);
+    if (rows == 0) return DN_OK;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return DN_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)dk, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)dk * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)dk};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DN_OK : DN_ERR_UNSUPPORTED;
+}
+
 struct Dims {
     int64_t B, T, H, dk, dv, N;
     bool varlen;
@@ -328,12 +345,14 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         g_last_G = -1;
         g_last_s = -1;
     }
+    CUtensorMap tp;
+    if ((st = make_p_map(&tp, p.wsP, slots * DK, DK)) != DN_OK) return st;
     // one CTA per (chain, 8 state columns); 16 columns when that needs more than one wave
     auto launch_scan = [&]() {
         if (nScan * (DV / 8) <= sms)
-            kS8<<<dim3((unsigned)nScan, DV / 8), scan_threads<DK, 8>(), smemS8, stream>>>(p);
+            kS8<<<dim3((unsigned)nScan, DV / 8), scan_threads<DK, 8>(), smemS8, stream>>>(tp, p);
         else
-            kS16<<<dim3((unsigned)nScan, DV / 16), scan_threads<DK, 16>(), smemS16, stream>>>(p);
+            kS16<<<dim3((unsigned)nScan, DV / 16), scan_threads<DK, 16>(), smemS16, stream>>>(tp, p);
     };
     int launches = d.varlen ? 1 : 0;
     if (kTc) {
@@ -519,6 +538,12 @@ int dn_trace_copy(unsigned long long* host) {
 }
 int dn_trace_copy_prep(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_dn_trace_prep, sizeof(g_dn_trace_prep)) == cudaSuccess ? 0 : 1;
+}
+int dn_trace_copy_scan(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_dn_trace_scan, sizeof(g_dn_trace_scan)) == cudaSuccess ? 0 : 1;
+}
+int dn_trace_copy_sum(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, tcs::g_dn_trace_sum, sizeof(tcs::g_dn_trace_sum)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

@@ -401,35 +401,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
 }
 
 // Segment scan: start(g+1) = P_g start(g) + H_g, start(1) = end state of
-// segment 0.  fp32; one CTA per (chain, COLS columns of the state), 4 columns
-// per thread.  P_{g+1} is prefetched by one bulk copy into the second buffer,
-// and each thread's H_{g+1} values into registers, while step g is computed.
-// P is stored unpadded and the CTA's columns of the state transposed (one
-// row of DK per column); lane a starts its sweep over k at 4 (a mod 8), so that
-// both the float4 reads of P's rows and those of the state's columns fall into
-// 8 distinct 16-byte bank groups per quarter-warp.  COLS is 16 when 8-column
-// CTAs would need more than one wave.
+// segment 0.  One CTA per (chain, COLS columns of the state); warp w computes
+// state rows 16 w .. + 15 of the CTA's columns with tensor-core tf32 products
+// in three passes (hi hi + hi lo + lo hi, the operands split into a tf32 head
+// and a tf32 tail), which keeps the sums at fp32 accuracy.  P_{g+1} is
+// prefetched by TMA (boxes of 32 columns, 128-byte swizzle, so that the
+// fragment reads of 8 rows hit distinct banks) and each thread's H_{g+1}
+// values into registers while step g is computed; the CTA's state columns are
+// kept transposed with rows padded by 4 floats.  COLS is 16 when 8-column CTAs
+// would need more than one wave.
 template <int DK, int COLS>
-__host__ __device__ constexpr int scan_threads() { return DK * COLS / 4; }
+__host__ __device__ constexpr int scan_threads() { return 2 * DK; }
 template <int DK, int COLS>
 __host__ __device__ constexpr int scan_smem_bytes() {
-    return (2 * DK * DK + DK * COLS) * 4 + 32;
+    return 2 * DK * DK * 4 + COLS * (DK + 4) * 4 + 32 + 1024;
+}
+#ifdef DN_TRACE
+static __device__ unsigned long long g_dn_trace_scan[64 * 4];
+#define DN_TSC(g, slot)                                                                   \
+    do {                                                                                  \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && (g) < 64)            \
+            g_dn_trace_scan[(g) * 4 + (slot)] = sm100::globaltimer();                     \
+    } while (0)
+#else
+#define DN_TSC(g, slot) \
+    do {                \
+    } while (0)
+#endif
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = sm100::to_tf32(x);
+    lo = sm100::to_tf32(x - __uint_as_float(hi));
 }
 template <int DK, int DV, int COLS>
-__global__ void __launch_bounds__(DK * COLS / 4) k_scan(Params p) {
-    extern __shared__ __align__(128) float fsm[];
-    constexpr int NT = DK * COLS / 4;
+__global__ void __launch_bounds__(2 * DK) k_scan(const __grid_constant__ CUtensorMap tp, Params p) {
+    extern __shared__ uint8_t scan_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(scan_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    constexpr int SLD = DK + 4;                 // padded row of a transposed state column
+    constexpr int NTILE = COLS / 8;             // n8 tiles
     constexpr uint32_t kPBytes = (uint32_t)DK * DK * 4u;
-    constexpr uint32_t kPiece = kPBytes < 16384u ? kPBytes : 16384u;
-    static_assert((DK & (DK - 1)) == 0 && DK >= 32, "rows");
-    float* St = fsm + 2 * DK * DK;                          // COLS x DK (state columns)
-    auto Pm = [&](int b) { return fsm + b * DK * DK; };     // DK x DK, two buffers
-    uint64_t* bars = reinterpret_cast<uint64_t*>(St + DK * COLS);
+    static_assert(DK % 32 == 0 && COLS % 8 == 0, "tiles");
+    auto Pm = [&](int b) { return smem + b * kPBytes; };    // DK/32 swizzled boxes of DK rows x 32 columns
+    float* St = reinterpret_cast<float*>(smem + 2 * kPBytes);  // COLS x SLD
+    uint64_t* bars = reinterpret_cast<uint64_t*>(St + COLS * SLD);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2);
-    const int tid = threadIdx.x;
-    const int a = tid % DK, c = 4 * (tid / DK);            // state row, first of 4 columns
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
+    const int ra = 16 * warp + gq;              // fragment rows ra, ra + 8
     const int c0 = blockIdx.y * COLS;
-    const int rot = 4 * (a & 7);
     const int n = count_scan(p.sched);
     if (tid == 0) {
         sm100::mbar_init(&bars[0], 1);
@@ -441,19 +459,29 @@ __global__ void __launch_bounds__(DK * COLS / 4) k_scan(Params p) {
     // per buffer (bit b): parity of its next completion, and a copy in flight into
     // it (at most one: a buffer is refilled only after its last step was computed)
     uint32_t phase = 0, pending = 0;
-    float4 hn = make_float4(0.f, 0.f, 0.f, 0.f);
-    // P_g into buffer g % 2, this thread's 4 values of H_g into hn
+    float2 hn[NTILE][2];
+    // P_g into buffer g % 2, this thread's fragment of H_g into hn
     auto prefetch = [&](const Item& it, int g) {
         if (g + 1 >= it.G) return;
         const int b = g & 1;
         pending |= 1u << b;
         if (tid == 0) {
-            const uint8_t* Pg = reinterpret_cast<const uint8_t*>(p.wsP + (int64_t)(it.slot + g) * DK * DK);
-            uint8_t* dst = reinterpret_cast<uint8_t*>(Pm(b));
             sm100::mbar_expect_tx(&bars[b], kPBytes);
-            for (uint32_t o = 0; o < kPBytes; o += kPiece) sm100::bulk_load(dst + o, Pg + o, kPiece, &bars[b]);
+#pragma unroll
+            for (int bx = 0; bx < DK / 32; ++bx)
+                sm100::tma_load_2d(Pm(b) + bx * DK * 128, &tp, &bars[b], 32 * bx, (it.slot + g) * DK);
         }
-        hn = *reinterpret_cast<const float4*>(p.wsH + (int64_t)(it.slot + g) * DK * DV + (int64_t)a * DV + c0 + c);
+        const float* Hg = p.wsH + (int64_t)(it.slot + g) * DK * DV + c0 + 2 * tq;
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                hn[nt][h] = *reinterpret_cast<const float2*>(Hg + (int64_t)(ra + 8 * h) * DV + 8 * nt);
+    };
+    // element (r, k) of a P buffer
+    auto pel = [&](const uint8_t* pb, int r, int k) {
+        return *reinterpret_cast<const float*>(pb + (k >> 5) * (DK * 128) + r * 128 +
+                                               ((((k & 31) >> 2) ^ (r & 7)) << 4) + ((k & 3) << 2));
     };
     bool ok = true;
     for (int i = blockIdx.x; ok && i < n; i += gridDim.x) {
@@ -461,14 +489,25 @@ __global__ void __launch_bounds__(DK * COLS / 4) k_scan(Params p) {
         const float* E0 = p.wsH + (int64_t)it.slot * DK * DV;
         float* out0 = p.wsS + (int64_t)it.slot * DK * DV;
         prefetch(it, 1);
-        for (int e = tid; e < DK * COLS; e += NT) {
+        for (int e = tid; e < DK * COLS; e += 2 * DK) {
             const int r = e % DK, cc = e / DK;
             const float x = E0[r * DV + c0 + cc];
-            St[cc * DK + r] = x;
+            St[cc * SLD + r] = x;
             out0[r * DV + c0 + cc] = x;
         }
+        DN_TSC(0, 0);
         for (int g = 1; g + 1 < it.G; ++g) {
-            float acc[4] = {hn.x, hn.y, hn.z, hn.w};
+            DN_TSC(g, 0);
+            // four independent accumulations (even / odd k steps, head x head / the
+            // two head x tail terms) keep several products in flight per warp
+            float acc[NTILE][4], accH[NTILE][4], accL[2][NTILE][4];
+#pragma unroll
+            for (int nt = 0; nt < NTILE; ++nt) {
+                acc[nt][0] = hn[nt][0].x; acc[nt][1] = hn[nt][0].y;
+                acc[nt][2] = hn[nt][1].x; acc[nt][3] = hn[nt][1].y;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) accH[nt][e] = accL[0][nt][e] = accL[1][nt][e] = 0.f;
+            }
             prefetch(it, g + 1);
             const int b = g & 1;
             const bool landed = sm100::mbar_wait(&bars[b], (phase >> b) & 1u, abort_flag);
@@ -480,26 +519,45 @@ __global__ void __launch_bounds__(DK * COLS / 4) k_scan(Params p) {
                 ok = false;
                 break;
             }
-            const float* prow = Pm(b) + a * DK;
-            const float* scol = St + c * DK;
-#pragma unroll 4
-            for (int k0 = 0; k0 < DK; k0 += 4) {
-                const int k = (k0 + rot) & (DK - 1);
-                const float4 pv = *reinterpret_cast<const float4*>(prow + k);
+            DN_TSC(g, 1);
+            const uint8_t* pb = Pm(b);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 sv = *reinterpret_cast<const float4*>(scol + j * DK + k);
-                    acc[j] = fmaf(pv.x, sv.x, acc[j]);
-                    acc[j] = fmaf(pv.y, sv.y, acc[j]);
-                    acc[j] = fmaf(pv.z, sv.z, acc[j]);
-                    acc[j] = fmaf(pv.w, sv.w, acc[j]);
+            for (int ks = 0; ks < DK / 8; ++ks) {
+                const int k = 8 * ks + tq;
+                uint32_t ah[4], al[4];
+                split_tf32(pel(pb, ra, k), ah[0], al[0]);
+                split_tf32(pel(pb, ra + 8, k), ah[1], al[1]);
+                split_tf32(pel(pb, ra, k + 4), ah[2], al[2]);
+                split_tf32(pel(pb, ra + 8, k + 4), ah[3], al[3]);
+#pragma unroll
+                for (int nt = 0; nt < NTILE; ++nt) {
+                    const float* sc = St + (8 * nt + gq) * SLD + k;
+                    uint32_t bh0, bl0, bh1, bl1;
+                    split_tf32(sc[0], bh0, bl0);
+                    split_tf32(sc[4], bh1, bl1);
+                    float (&hacc)[4] = (ks & 1) ? accH[nt] : acc[nt];
+                    sm100::mma_tf32(accL[ks & 1][nt], al[0], al[1], al[2], al[3], bh0, bh1);
+                    sm100::mma_tf32(accL[ks & 1][nt], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+                    sm100::mma_tf32(hacc, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
                 }
             }
-            __syncthreads();  // every thread has read S(g) and P_g
-            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV + (int64_t)a * DV + c0 + c;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) St[(c + j) * DK + a] = acc[j];
-            *reinterpret_cast<float4*>(outg) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][e] += accH[nt][e] + (accL[0][nt][e] + accL[1][nt][e]);
+            __syncthreads();  // every thread has read S(g) and P_g
+            DN_TSC(g, 2);
+            float* outg = p.wsS + (int64_t)(it.slot + g) * DK * DV + c0 + 2 * tq;
+#pragma unroll
+            for (int nt = 0; nt < NTILE; ++nt) {
+                const int cc = 8 * nt + 2 * tq;
+                St[cc * SLD + ra] = acc[nt][0];
+                St[(cc + 1) * SLD + ra] = acc[nt][1];
+                St[cc * SLD + ra + 8] = acc[nt][2];
+                St[(cc + 1) * SLD + ra + 8] = acc[nt][3];
+                *reinterpret_cast<float2*>(outg + (int64_t)ra * DV + 8 * nt) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2*>(outg + (int64_t)(ra + 8) * DV + 8 * nt) = make_float2(acc[nt][2], acc[nt][3]);
+            }
         }
         __syncthreads();
     }

@@ -22,7 +22,7 @@ namespace dn {
 
 struct CostModel {
     float c = 1.0f;      // boundary pass, per chunk
-    float a = 0.9f;      // summary pass, per chunk (two chains, no output, no Q)
+    float a = 1.25f;     // summary pass, per chunk (two chains, no output, no Q)
     float scan = 2.0f;   // one step of the segment scan
 };
 

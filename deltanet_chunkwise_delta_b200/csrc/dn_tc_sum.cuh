@@ -98,6 +98,21 @@ enum : int {
 };
 static_assert(B_GAP2 + 2 <= NBAR, "barrier count");
 
+// Optional timeline of CTA 1 (the first two-chain item of a split chain; build
+// with -DDN_TRACE): globaltimer stamps per chunk and pipeline event.
+#ifdef DN_TRACE
+static __device__ unsigned long long g_dn_trace_sum[64 * 32];
+#define DN_TS(cond, r, slot)                                                                      \
+    do {                                                                                          \
+        if ((cond) && blockIdx.x == 1 && (r) >= 0 && (r) < 64 && (threadIdx.x & 31) == 0)          \
+            g_dn_trace_sum[(r) * 32 + (slot)] = globaltimer();                                    \
+    } while (0)
+#else
+#define DN_TS(cond, r, slot) \
+    do {                     \
+    } while (0)
+#endif
+
 __global__ void __launch_bounds__(kThreadsSum, 1)
     k_tc_summary(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -208,8 +223,10 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
             for (int r = 0; r < nch; ++r) {
                 const int sa = r % NA;
                 const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
+                DN_TS(true, r, 0);
                 if (!mbar_wait3(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1, abort_flag))
                     break;
+                DN_TS(true, r, 1);
                 bool ok = true;
                 for (int x = 0; x < nx; ++x) {
                     if (x == 1 && !mbar_wait(&bars[B_SBF + 1], r & 1, abort_flag)) {
@@ -232,6 +249,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                         }
                     }
                     umma_commit(&bars[B_C1 + x]);
+                    DN_TS(true, r, 2 + x);
                 }
                 if (!ok) break;
                 mbar_arrive(&bars[B_GAP1 + (r & 1)]);
@@ -240,6 +258,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                         ok = false;
                         break;
                     }
+                    DN_TS(true, r, 4 + 2 * x);
                     tc_fence_after();
                     const uint64_t zo = (uint64_t)((x * Z_BYTES) >> 4);
 #pragma unroll
@@ -247,6 +266,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                         umma_bf16(tmem + tm_s(x), dZ + zo + (uint64_t)((j * 32) >> 4),
                                   dK + sta + (uint64_t)((j * 2048) >> 4), i_c3, 1u);
                     umma_commit(&bars[B_SFULL + x]);
+                    DN_TS(true, r, 5 + 2 * x);
                     if (x == 0) mbar_arrive(&bars[B_GAP2 + (r & 1)]);
                 }
                 if (!ok) break;
@@ -301,12 +321,14 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
             for (int r = 0; ok && r + 1 < nch; ++r) {
                 // gap 1: chunk r + 1's data; W^T(r) was read out before chunk r's products
                 if (!wait_data(r + 1) || !mbar_wait(&bars[B_GAP1 + (r & 1)], (r >> 1) & 1, abort_flag)) break;
+                DN_TS(true, r, 8);
                 tc_fence_after();
                 issue_w(r + 1);
                 // gap 2: Z_H^T(r) read out of the U^T columns, chain H's update queued
                 if (!mbar_wait(&bars[B_ZFULL], r & 1, abort_flag) ||
                     !mbar_wait(&bars[B_GAP2 + (r & 1)], (r >> 1) & 1, abort_flag))
                     break;
+                DN_TS(true, r, 9);
                 tc_fence_after();
                 issue_u(r + 1);
             }
@@ -322,6 +344,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
             if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
                                                     abort_flag)))
                 break;
+            DN_TS(q == 0, r, 10);
             tc_fence_after();
             {
                 RowFrags f;
@@ -332,6 +355,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_WFULL]);
+            DN_TS(q == 0, r, 11);
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ chain epilogues
@@ -394,6 +418,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                 // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
                 // the state update)
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
+                DN_TS(wq == 0, r, 12 + 4 * x);
                 tc_fence_after();
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -409,9 +434,11 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_ZFULL + x]);
+                DN_TS(wq == 0, r, 13 + 4 * x);
                 // S_x^T -> bf16 (and fp32 out after the last chunk); the chunk's first
                 // product (the only reader of the bf16 copy) is complete
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + x], r & 1, abort_flag))) break;
+                DN_TS(wq == 0, r, 14 + 4 * x);
                 tc_fence_after();
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
@@ -428,6 +455,7 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
+                DN_TS(wq == 0, r, 15 + 4 * x);
             }
         }
     }
