@@ -306,7 +306,7 @@ def run_b200(args, w: wl.Workload):
                 "frac": achieved / hbm_peak,
                 "traffic": stored_traffic(w.name) if tc_kernel else None,
                 "peak_kind": peak_kind,
-                "kernel": "k_tc_chain<true> (boundary pass)" if tc_kernel else "k_boundary",
+                "kernel": "k_tc_chain (boundary pass)" if tc_kernel else "k_boundary",
                 "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": kernel_bytes}
     # the whole path against its roofline: slower of FLOPs at the bf16 peak and bytes at HBM
     t_roof = max(th * flops_per_token_head(w.dk, w.dv) / (tc_peak * 1e12),

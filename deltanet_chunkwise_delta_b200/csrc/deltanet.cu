@@ -230,7 +230,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kA = k_summary<E, DK, DV, STAGES>;
     auto* kS8 = k_scan<DK, DV, 8>;
     auto* kS16 = k_scan<DK, DV, 16>;
-    auto* kCt = tc::k_tc_chain<true>;
+    auto* kCt = tc::k_tc_chain;
     auto* kAt = tcs::k_tc_summary;
     auto* kPrep = k_ut_prep;
     constexpr int smemPrep = PrepSmem::TOTAL;

@@ -90,7 +90,7 @@ dn_status na_setup(int dev, unsigned char** scratch) {
     }
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DN_ERR_CUDA;
-    if (cudaFuncSetAttribute(dn::tc::k_tc_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(dn::tc::k_tc_chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::tc::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::PrepSmem::TOTAL) != cudaSuccess ||
@@ -190,7 +190,7 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     const int64_t cap = (int64_t)sms * dn::kPrepCtasPerSm;
     const int grid = (int)(units < cap ? units : cap);
     dn::k_ut_prep<<<grid, dn::kPrepThreads, dn::PrepSmem::TOTAL, stream>>>(tq, tk, p);
-    dn::tc::k_tc_chain<true><<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
+    dn::tc::k_tc_chain<<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }

@@ -1,4 +1,5 @@
-// Tensor-core (tcgen05 / TMEM / TMA) chain kernel for bf16, d_k = d_v = 128.
+// Tensor-core (tcgen05 / TMEM / TMA) boundary pass for bf16, d_k = d_v = 128:
+// every run of chunks from its true start state, with the outputs.
 //
 // Same per-chunk algorithm as dn_chain.cuh ("Linear Attention, Visualized",
 // DeltaNet, "Complete per-chunk algorithm"), evaluated in the transposed
@@ -164,19 +165,16 @@ __device__ __forceinline__ void store_token_rows(const RowFrags& f, int q, uint8
                           pack_bf16(scale * __uint_as_float(f.hi[g][2]), scale * __uint_as_float(f.hi[g][3])));
 }
 
-template <bool HAS_Q>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+static __global__ void __launch_bounds__(kThreadsTc, 1)
     k_tc_chain(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    const int n_items = HAS_Q ? count_C(p.sched) : count_A(p.sched);
+    const int n_items = count_C(p.sched);
     if ((int)blockIdx.x >= n_items) return;
-    int mode = kModeOut;
-    const Item it = HAS_Q ? item_C(p.sched, blockIdx.x) : item_A(p.sched, blockIdx.x, mode);
-    const bool has_v = mode != kModeP;
+    const Item it = item_C(p.sched, blockIdx.x);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -226,27 +224,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int nch = (ntok + kChunk - 1) / kChunk;
 
     // start state and destination of the run
-    const float* x_in = nullptr;
-    float* x_out = nullptr;
-    bool identity = false;
     const float* s0 = p.s0 ? p.s0 + it.seq * p.s0_sn + it.head * p.s0_sh : nullptr;
-    if (mode == kModeOut) {
-        x_in = it.g == 0 ? s0 : p.wsS + (int64_t)(it.slot + it.g - 1) * D * D;
-        if (it.g == it.G - 1 && p.sT) x_out = p.sT + it.seq * p.sT_sn + it.head * p.sT_sh;
-    } else if (mode == kModeEnd) {
-        x_in = s0;
-        x_out = p.wsH + (int64_t)it.slot * D * D;
-    } else if (mode == kModeH) {
-        x_out = p.wsH + (int64_t)(it.slot + it.g) * D * D;
-    } else {
-        identity = true;
-        x_out = p.wsP + (int64_t)(it.slot + it.g) * D * D;
-    }
+    const float* x_in = it.g == 0 ? s0 : p.wsS + (int64_t)(it.slot + it.g - 1) * D * D;
+    float* x_out = (it.g == it.G - 1 && p.sT) ? p.sT + it.seq * p.sT_sn + it.head * p.sT_sh : nullptr;
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ ring A: q, k
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = (HAS_Q ? 16384u : 0u) + 16384u;
+            const uint32_t bytes = 32768u;
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
                 const int s = r % NA;
@@ -256,7 +241,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int t0 = it.tok0 + r * kChunk;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
-                    if (HAS_Q) tma_load_4d(st + a_q(r) + a * 16384, &tq, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
+                    tma_load_4d(st + a_q(r) + a * 16384, &tq, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
                     tma_load_4d(st + A_K + a * 8192, &tk, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
                 }
                 issued = r + 1;
@@ -270,7 +255,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     } else if (warp == kTmaBWarp) {
         // ------------------------------------------------------------ ring B: v, T
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = (has_v ? 16384u : 0u) + 8192u;
+            const uint32_t bytes = 16384u + 8192u;
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
                 const int s = r & 1;
@@ -278,11 +263,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 mbar_expect_tx(&bars[B_FULLB + s], bytes);
                 uint8_t* st = smem + OFF_B + s * B_STAGE;
                 const int t0 = it.tok0 + r * kChunk;
-                if (has_v) {
 #pragma unroll
-                    for (int a = 0; a < 2; ++a)
-                        tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
-                }
+                for (int a = 0; a < 2; ++a)
+                    tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
                 bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnitBytes, 8192,
                           &bars[B_FULLB + s]);
                 issued = r + 1;
@@ -293,12 +276,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ state-chain products
-        // Per chunk: [Z^T | O^T] = [U^T | 0] + S^T [-W^T | Q^T] (one product; N = 64
-        // without queries), S^T += Z^T K, O^T += Z^T P^T.  After the first it opens
-        // a gap for the chunk-parallel issuer.
+        // Per chunk: [Z^T | O^T] = [U^T | 0] + S^T [-W^T | Q^T] (one product of N = 128),
+        // S^T += Z^T K, O^T += Z^T P^T.  After the first it opens a gap for the
+        // chunk-parallel issuer.
         if (lane == 0 && nch > 0) {
             const uint32_t sb = saddr(smem);
-            const uint32_t i_c1 = idesc_bf16(128, HAS_Q ? 128 : 64, false, false);
+            const uint32_t i_c1 = idesc_bf16(128, 128, false, false);
             const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
             const uint32_t i_o = idesc_bf16(128, 64, false, false);
             const uint64_t dWQ = sdesc(sb, 16, 1024);           // [-W; Q] / [Q; -W] token rows, K-major
@@ -308,19 +291,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int sa = r % NA, s = r & 1;
                 const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
                 DN_TR(true, r, 0);
-                const bool ready =
-                    HAS_Q ? mbar_wait4(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1,
-                                       &bars[B_OFREE + s], (r >> 1) & 1, abort_flag)
-                          : mbar_wait3(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1, abort_flag);
+                const bool ready = mbar_wait4(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1,
+                                              &bars[B_OFREE + s], (r >> 1) & 1, abort_flag);
                 if (!ready) break;
                 DN_TR(true, r, 3);
                 tc_fence_after();
                 // [Z^T | O^T] = [U^T | 0] + S^T [-W^T | Q^T]  (odd chunks: [O^T | Z^T])
-                const uint32_t d1 = HAS_Q ? tm_c1(r) : TM_ZU;
+                const uint32_t d1 = tm_c1(r);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint64_t o = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
-                    umma_bf16_ts(tmem + d1, tmem + TM_SBF + 8 * j, dWQ + sta + o, i_c1, has_v ? 1u : (j > 0 ? 1u : 0u));
+                    umma_bf16_ts(tmem + d1, tmem + TM_SBF + 8 * j, dWQ + sta + o, i_c1, 1u);
                 }
                 umma_commit(&bars[B_C1]);
                 mbar_arrive(&bars[B_GAP1 + s]);
@@ -335,7 +316,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                                  1u);
                 umma_commit(&bars[B_SFULL]);
                 mbar_arrive(&bars[B_GAP2 + s]);
-                if (HAS_Q) {
+                {
                     // O^T += Z^T P^T
                     if (!mbar_wait(&bars[B_PFULL + s], (r >> 1) & 1, abort_flag)) break;
                     tc_fence_after();
@@ -378,12 +359,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             auto issue_u = [&](int c) {
                 const int s = c & 1;
                 const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
-                if (has_v) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        umma_bf16(tmem + TM_ZU, dVT + stb + (uint64_t)((j * 2048) >> 4),
-                                  dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
-                }
+                for (int j = 0; j < 4; ++j)
+                    umma_bf16(tmem + TM_ZU, dVT + stb + (uint64_t)((j * 2048) >> 4),
+                              dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 umma_commit(&bars[B_UFULL]);
                 umma_commit(&bars[B_EMPTYB + s]);
             };
@@ -476,7 +455,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             DN_TR(q == 0, c, 26);
             return true;
         };
-        if (HAS_Q) {
+        {
             // both O^T buffers start at zero: the first product accumulates into them
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
@@ -505,24 +484,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_WTFREE]);
-                store_token_rows(f, q, stage + (HAS_Q ? a_w(r) : 0), 16384, -1.f);
+                store_token_rows(f, q, stage + a_w(r), 16384, -1.f);
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_WFULL]);
             DN_TR(q == 0, r, 14);
-            if (HAS_Q && r >= 1) {
+            if (r >= 1) {
                 // chunk r - 1 complete: copy in chunk r + 1's P tile (into chunk r - 1's
                 // buffer), write out O of chunk r - 1
                 if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL], (r - 1) & 1, abort_flag))) break;
                 if (q == 0 && lane == 0 && r + 1 < nch) issue_p(r + 1);
                 if (!store_o(r - 1)) break;
-            } else if (HAS_Q && q == 0 && lane == 0) {
+            } else if (q == 0 && lane == 0) {
                 issue_p(0);
                 if (nch > 1) issue_p(1);
             }
         }
-        if (HAS_Q && nch > 0 && !*abort_flag &&
+        if (nch > 0 && !*abort_flag &&
             __all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL], (nch - 1) & 1, abort_flag)))
             store_o(nch - 1);
         // the last P copies must have landed, and the TMA stores of O completed,
@@ -533,7 +512,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             for (int c = p_issued - 2 < 0 ? 0 : p_issued - 2; c < p_issued; ++c)
                 mbar_wait(&bars[B_PFULL + (c & 1)], (c >> 1) & 1, &drain, 200000000ull);
         }
-        if (HAS_Q && q == 0 && lane == 0) bulk_wait0();
+        if (q == 0 && lane == 0) bulk_wait0();
     } else if (warp < 8) {
         // ------------------------------------------------------------ chain epilogue
         // Warp w handles d_v rows 32 (w % 4) .. + 31 (its tensor-memory lane quarter)
@@ -548,7 +527,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int a = 64 * h + c;
                 float x = 0.f;
                 if (x_in) x = x_in[(int64_t)a * D + d];
-                else if (identity) x = (a == d) ? 1.f : 0.f;
                 v[c] = __float_as_uint(x);
             }
             if (nch == 0) {
@@ -569,7 +547,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             // Z^T -> bf16 (A operand of the S^T update and of O^T += Z^T P^T), once the
             // previous chunk's O^T += Z^T P^T has read the previous one
             DN_TR(warp == 0, r, 27);
-            if (HAS_Q && r >= 1 &&
+            if (r >= 1 &&
                 !__all_sync(0xffffffffu, mbar_wait(&bars[B_OFULL], (r - 1) & 1, abort_flag)))
                 break;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1], r & 1, abort_flag))) break;

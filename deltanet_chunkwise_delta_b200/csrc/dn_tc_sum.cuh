@@ -33,6 +33,8 @@
 // tensor memory and reports DN_ERR_TIMEOUT through the error flag.
 #pragma once
 
+#include <type_traits>
+
 #include "dn_common.cuh"
 #include "dn_sm100.cuh"
 #include "dn_tc.cuh"
@@ -113,7 +115,7 @@ static __device__ unsigned long long g_dn_trace_sum[64 * 32];
     } while (0)
 #endif
 
-__global__ void __launch_bounds__(kThreadsSum, 1)
+static __global__ void __launch_bounds__(kThreadsSum, 1)
     k_tc_summary(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -123,7 +125,6 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
     if ((int)blockIdx.x >= n_items) return;
     int mode = kModeEnd;
     const Item it = item_A(p.sched, blockIdx.x, mode);
-    const bool two = mode == kModeHP;  // chain P runs too
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -164,301 +165,311 @@ __global__ void __launch_bounds__(kThreadsSum, 1)
     const int ntok = it.tok1 - it.tok0;
     const int nch = (ntok + kChunk - 1) / kChunk;
 
-    if (warp == kTmaWarp) {
-        // ------------------------------------------------------------ ring A: k
-        if (lane == 0 && nch > 0) {
-            int issued = 0;
-            for (int r = 0; r < nch; ++r) {
-                const int s = r % NA;
-                if (r >= NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / NA) - 1) & 1, abort_flag)) break;
-                mbar_expect_tx(&bars[B_FULLA + s], 16384u);
-                uint8_t* st = smem + s * A_STAGE;
-                const int t0 = it.tok0 + r * kChunk;
-#pragma unroll
-                for (int a = 0; a < 2; ++a)
-                    tma_load_4d(st + A_K + a * 8192, &tk, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
-                issued = r + 1;
+    // the item's chain count is a compile-time constant of the role code below, so
+    // that each issuing thread runs straight-line product sequences
+    auto roles = [&](auto two_c) {
+        constexpr bool TWO = decltype(two_c)::value;
+        if (warp == kTmaWarp) {
+            // ------------------------------------------------------------ ring A: k
+            if (lane == 0 && nch > 0) {
+                int issued = 0;
+                for (int r = 0; r < nch; ++r) {
+                    const int s = r % NA;
+                    if (r >= NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / NA) - 1) & 1, abort_flag)) break;
+                    mbar_expect_tx(&bars[B_FULLA + s], 16384u);
+                    uint8_t* st = smem + s * A_STAGE;
+                    const int t0 = it.tok0 + r * kChunk;
+    #pragma unroll
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_4d(st + A_K + a * 8192, &tk, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
+                    issued = r + 1;
+                }
+                // the last loads issued must have landed before the CTA may exit (even after an abort)
+                volatile int drain = 0;
+                for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
+                    mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, 200000000ull);
             }
-            // the last loads issued must have landed before the CTA may exit (even after an abort)
-            volatile int drain = 0;
-            for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
-                mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, 200000000ull);
-        }
-    } else if (warp == kTmaBWarp) {
-        // ------------------------------------------------------------ ring B: v, T
-        if (lane == 0 && nch > 0) {
-            int issued = 0;
-            for (int r = 0; r < nch; ++r) {
-                const int s = r & 1;
-                if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
-                mbar_expect_tx(&bars[B_FULLB + s], 16384u + 8192u);
-                uint8_t* st = smem + OFF_B + s * B_STAGE;
-                const int t0 = it.tok0 + r * kChunk;
-#pragma unroll
-                for (int a = 0; a < 2; ++a) tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
-                bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnitBytes, 8192,
-                          &bars[B_FULLB + s]);
-                issued = r + 1;
+        } else if (warp == kTmaBWarp) {
+            // ------------------------------------------------------------ ring B: v, T
+            if (lane == 0 && nch > 0) {
+                int issued = 0;
+                for (int r = 0; r < nch; ++r) {
+                    const int s = r & 1;
+                    if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
+                    mbar_expect_tx(&bars[B_FULLB + s], 16384u + 8192u);
+                    uint8_t* st = smem + OFF_B + s * B_STAGE;
+                    const int t0 = it.tok0 + r * kChunk;
+    #pragma unroll
+                    for (int a = 0; a < 2; ++a) tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
+                    bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnitBytes, 8192,
+                              &bars[B_FULLB + s]);
+                    issued = r + 1;
+                }
+                volatile int drain = 0;
+                for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
+                    mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, 200000000ull);
             }
-            volatile int drain = 0;
-            for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
-                mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, 200000000ull);
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ chain products
-        // Per chunk and chain: Z_x^T = [U^T] + S_x^T (-W^T), then S_x^T += Z_x^T K.
-        // Chain P's first product is queued behind chain H's, and each state
-        // update as soon as its chain's Z^T is in shared memory.  Gap 1 (after the
-        // first products) lets the parallel issuer queue W^T of the next chunk, gap
-        // 2 (after chain H's update) its U^T.
-        if (lane == 0 && nch > 0) {
-            const uint32_t sb = saddr(smem);
-            const uint32_t i_c1 = idesc_bf16(128, 64, false, false);
-            const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
-            const uint64_t dW = sdesc(sb, 16, 1024);             // -W token rows, K-major
-            const uint64_t dK = sdesc(sb + A_K, 8192, 1024);     // K, MN-major
-            const uint64_t dZ = sdesc(sb + OFF_Z, 16, 1024);     // Z^T rows, K-major (+ Z_BYTES for P)
-            const uint64_t dSP = sdesc(sb + OFF_SP, 16, 1024);   // S_P^T bf16 rows, K-major
-            const int nx = two ? 2 : 1;
-            for (int r = 0; r < nch; ++r) {
-                const int sa = r % NA;
-                const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
-                DN_TS(true, r, 0);
-                if (!mbar_wait3(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1, abort_flag))
-                    break;
-                DN_TS(true, r, 1);
-                bool ok = true;
-                for (int x = 0; x < nx; ++x) {
-                    if (x == 1 && !mbar_wait(&bars[B_SBF + 1], r & 1, abort_flag)) {
-                        ok = false;
+        } else if (warp == kMmaWarp) {
+            // ------------------------------------------------------------ chain products
+            // Per chunk and chain: Z_x^T = [U^T] + S_x^T (-W^T), then S_x^T += Z_x^T K.
+            // Chain P's first product is queued behind chain H's, and each state
+            // update as soon as its chain's Z^T is in shared memory.  Gap 1 (after the
+            // first products) lets the parallel issuer queue W^T of the next chunk, gap
+            // 2 (after chain H's update) its U^T.
+            if (lane == 0 && nch > 0) {
+                const uint32_t sb = saddr(smem);
+                const uint32_t i_c1 = idesc_bf16(128, 64, false, false);
+                const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
+                const uint64_t dW = sdesc(sb, 16, 1024);             // -W token rows, K-major
+                const uint64_t dK = sdesc(sb + A_K, 8192, 1024);     // K, MN-major
+                const uint64_t dZ = sdesc(sb + OFF_Z, 16, 1024);     // Z^T rows, K-major (+ Z_BYTES for P)
+                const uint64_t dSP = sdesc(sb + OFF_SP, 16, 1024);   // S_P^T bf16 rows, K-major
+                for (int r = 0; r < nch; ++r) {
+                    const int sa = r % NA;
+                    const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
+                    DN_TS(true, r, 0);
+                    if (!mbar_wait3(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1, abort_flag))
                         break;
-                    }
+                    DN_TS(true, r, 1);
+                    // chain H: Z_H^T = U^T + S_H^T (-W^T), A operand (bf16 S_H^T) in tensor memory
                     tc_fence_after();
-                    if (x == 0) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint64_t o = (uint64_t)(((j >> 2) * 8192 + (j & 3) * 32) >> 4);
-                            umma_bf16_ts(tmem + tm_zu(0), tmem + TM_SBF + 8 * j, dW + sta + o, i_c1, 1u);
-                        }
-                    } else {
-#pragma unroll
+    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint64_t o = (uint64_t)(((j >> 2) * 8192 + (j & 3) * 32) >> 4);
+                        umma_bf16_ts(tmem + tm_zu(0), tmem + TM_SBF + 8 * j, dW + sta + o, i_c1, 1u);
+                    }
+                    umma_commit(&bars[B_C1]);
+                    DN_TS(true, r, 2);
+                    if constexpr (TWO) {
+                        // chain P: Z_P^T = S_P^T (-W^T), A operand in shared memory
+                        if (!mbar_wait(&bars[B_SBF + 1], r & 1, abort_flag)) break;
+                        tc_fence_after();
+    #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const uint64_t o = (uint64_t)(((j >> 2) * 8192 + (j & 3) * 32) >> 4);
                             const uint64_t oa = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
                             umma_bf16(tmem + tm_zu(1), dSP + oa, dW + sta + o, i_c1, j > 0 ? 1u : 0u);
                         }
+                        umma_commit(&bars[B_C1 + 1]);
+                        DN_TS(true, r, 3);
                     }
-                    umma_commit(&bars[B_C1 + x]);
-                    DN_TS(true, r, 2 + x);
-                }
-                if (!ok) break;
-                mbar_arrive(&bars[B_GAP1 + (r & 1)]);
-                for (int x = 0; x < nx; ++x) {
-                    if (!mbar_wait(&bars[B_ZFULL + x], r & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    DN_TS(true, r, 4 + 2 * x);
+                    mbar_arrive(&bars[B_GAP1 + (r & 1)]);
+                    // S_H^T += Z_H^T K
+                    if (!mbar_wait(&bars[B_ZFULL], r & 1, abort_flag)) break;
+                    DN_TS(true, r, 4);
                     tc_fence_after();
-                    const uint64_t zo = (uint64_t)((x * Z_BYTES) >> 4);
-#pragma unroll
+    #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        umma_bf16(tmem + tm_s(x), dZ + zo + (uint64_t)((j * 32) >> 4),
-                                  dK + sta + (uint64_t)((j * 2048) >> 4), i_c3, 1u);
-                    umma_commit(&bars[B_SFULL + x]);
-                    DN_TS(true, r, 5 + 2 * x);
-                    if (x == 0) mbar_arrive(&bars[B_GAP2 + (r & 1)]);
-                }
-                if (!ok) break;
-                // the stage's -W rows and k are read by the products above (and k by W^T of
-                // the chunk, complete before its -W rows were written)
-                umma_commit(&bars[B_EMPTYA + sa]);
-            }
-        }
-    } else if (warp == kParMmaWarp) {
-        // ------------------------------------------------------------ chunk-parallel products
-        // W^T and U^T (into chain H's Z columns) of chunk r + 1, each issued in one of
-        // the chain's gaps so that it never queues in front of a chain product: W^T
-        // once chunk r's first products are queued (its own -W rows were read out
-        // before them), U^T once Z_H^T(r) has been read out and chain H's update is
-        // queued.
-        if (lane == 0 && nch > 0) {
-            const uint32_t sb = saddr(smem);
-            const uint32_t i_tt = idesc_bf16(128, 64, true, false);
-            const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
-            const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
-            const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
-            auto issue_w = [&](int c) {
-                const uint64_t sta = (uint64_t)(((c % NA) * A_STAGE) >> 4);
-                const uint64_t stb = (uint64_t)(((c & 1) * B_STAGE) >> 4);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    umma_bf16(tmem + TM_WT, dKT + sta + (uint64_t)((j * 2048) >> 4),
-                              dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
-                umma_commit(&bars[B_WUFULL]);
-            };
-            // U^T of chunk c; its ring-B stage is consumed after it (W^T came first)
-            auto issue_u = [&](int c) {
-                const int s = c & 1;
-                const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    umma_bf16(tmem + tm_zu(0), dVT + stb + (uint64_t)((j * 2048) >> 4),
-                              dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
-                umma_commit(&bars[B_UFULL]);
-                umma_commit(&bars[B_EMPTYB + s]);
-            };
-            auto wait_data = [&](int c) -> bool {
-                return mbar_wait2(&bars[B_FULLA + c % NA], (c / NA) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
-                                  abort_flag);
-            };
-            bool ok = wait_data(0);
-            if (ok) {
-                tc_fence_after();
-                issue_w(0);
-                issue_u(0);
-            }
-            for (int r = 0; ok && r + 1 < nch; ++r) {
-                // gap 1: chunk r + 1's data; W^T(r) was read out before chunk r's products
-                if (!wait_data(r + 1) || !mbar_wait(&bars[B_GAP1 + (r & 1)], (r >> 1) & 1, abort_flag)) break;
-                DN_TS(true, r, 8);
-                tc_fence_after();
-                issue_w(r + 1);
-                // gap 2: Z_H^T(r) read out of the U^T columns, chain H's update queued
-                if (!mbar_wait(&bars[B_ZFULL], r & 1, abort_flag) ||
-                    !mbar_wait(&bars[B_GAP2 + (r & 1)], (r >> 1) & 1, abort_flag))
-                    break;
-                DN_TS(true, r, 9);
-                tc_fence_after();
-                issue_u(r + 1);
-            }
-        }
-    } else if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------ -W rows
-        const int q = warp - 8;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        for (int r = 0; r < nch; ++r) {
-            uint8_t* stage = smem + (r % NA) * A_STAGE;
-            // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's k stage,
-            // once the stage holds the chunk (its previous chunk's products are done)
-            if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
-                                                    abort_flag)))
-                break;
-            DN_TS(q == 0, r, 10);
-            tc_fence_after();
-            {
-                RowFrags f;
-                tmem_load_rows(tmem + lane_base + TM_WT, f);
-                tc_fence_before();
-                store_token_rows(f, q, stage, 8192, -1.f);
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_WFULL]);
-            DN_TS(q == 0, r, 11);
-        }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ chain epilogues
-        // Warp w serves chain x = w / 4 and d_v rows 32 (w % 4) .. + 31 (its lane quarter).
-        const int x = warp >> 2, wq = warp & 3;
-        const int d = 32 * wq + lane;  // d_v row of S_x^T, Z_x^T
-        const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        if (x == 0 || two) {
-            // start state and destination of this chain
-            const float* x_in = nullptr;
-            float* x_out;
-            if (x == 1) {
-                x_out = p.wsP + (int64_t)(it.slot + it.g) * D * D;
-            } else if (mode == kModeEnd) {
-                x_in = p.s0 ? p.s0 + it.seq * p.s0_sn + it.head * p.s0_sh : nullptr;
-                x_out = p.wsH + (int64_t)it.slot * D * D;
-            } else {
-                x_out = p.wsH + (int64_t)(it.slot + it.g) * D * D;
-            }
-            uint8_t* zs = smem + OFF_Z + x * Z_BYTES;
-            // bf16 copy of S_x^T columns 64 hh .. + 63 of row d: chain H into tensor
-            // memory, chain P into K block hh of its shared-memory operand
-            auto store_sbf = [&](int xx, int hh, const uint32_t(&pk)[32]) {
-                if (xx == 0) {
-                    tmem_st32(tmem + lane_base + TM_SBF + 32 * hh, pk);
-                } else {
-                    uint8_t* sp = smem + OFF_SP + hh * 16384;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(sp + swz128(d, 8 * c)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                }
-            };
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t v[64];
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int a = 64 * hh + c;
-                    float y = 0.f;
-                    if (x_in) y = x_in[(int64_t)a * D + d];
-                    else if (x == 1) y = (a == d) ? 1.f : 0.f;
-                    v[c] = __float_as_uint(y);
-                }
-                if (nch == 0) {
-                    for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
-                } else {
-                    tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                    uint32_t pk[32];
-                    pack_pairs<64>(v, pk);
-                    store_sbf(x, hh, pk);
+                        umma_bf16(tmem + tm_s(0), dZ + (uint64_t)((j * 32) >> 4), dK + sta + (uint64_t)((j * 2048) >> 4),
+                                  i_c3, 1u);
+                    umma_commit(&bars[B_SFULL]);
+                    DN_TS(true, r, 5);
+                    mbar_arrive(&bars[B_GAP2 + (r & 1)]);
+                    if constexpr (TWO) {
+                        // S_P^T += Z_P^T K
+                        if (!mbar_wait(&bars[B_ZFULL + 1], r & 1, abort_flag)) break;
+                        DN_TS(true, r, 6);
+                        tc_fence_after();
+                        const uint64_t zo = (uint64_t)(Z_BYTES >> 4);
+    #pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            umma_bf16(tmem + tm_s(1), dZ + zo + (uint64_t)((j * 32) >> 4),
+                                      dK + sta + (uint64_t)((j * 2048) >> 4), i_c3, 1u);
+                        umma_commit(&bars[B_SFULL + 1]);
+                        DN_TS(true, r, 7);
+                    }
+                    // the stage's -W rows and k are read by the products above (and k by W^T of
+                    // the chunk, complete before its -W rows were written)
+                    umma_commit(&bars[B_EMPTYA + sa]);
                 }
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
+        } else if (warp == kParMmaWarp) {
+            // ------------------------------------------------------------ chunk-parallel products
+            // W^T and U^T (into chain H's Z columns) of chunk r + 1, each issued in one of
+            // the chain's gaps so that it never queues in front of a chain product: W^T
+            // once chunk r's first products are queued (its own -W rows were read out
+            // before them), U^T once Z_H^T(r) has been read out and chain H's update is
+            // queued.
+            if (lane == 0 && nch > 0) {
+                const uint32_t sb = saddr(smem);
+                const uint32_t i_tt = idesc_bf16(128, 64, true, false);
+                const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
+                const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
+                const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
+                auto issue_w = [&](int c) {
+                    const uint64_t sta = (uint64_t)(((c % NA) * A_STAGE) >> 4);
+                    const uint64_t stb = (uint64_t)(((c & 1) * B_STAGE) >> 4);
+    #pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        umma_bf16(tmem + TM_WT, dKT + sta + (uint64_t)((j * 2048) >> 4),
+                                  dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                    umma_commit(&bars[B_WUFULL]);
+                };
+                // U^T of chunk c; its ring-B stage is consumed after it (W^T came first)
+                auto issue_u = [&](int c) {
+                    const int s = c & 1;
+                    const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
+    #pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        umma_bf16(tmem + tm_zu(0), dVT + stb + (uint64_t)((j * 2048) >> 4),
+                                  dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                    umma_commit(&bars[B_UFULL]);
+                    umma_commit(&bars[B_EMPTYB + s]);
+                };
+                auto wait_data = [&](int c) -> bool {
+                    return mbar_wait2(&bars[B_FULLA + c % NA], (c / NA) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
+                                      abort_flag);
+                };
+                bool ok = wait_data(0);
+                if (ok) {
+                    tc_fence_after();
+                    issue_w(0);
+                    issue_u(0);
+                }
+                for (int r = 0; ok && r + 1 < nch; ++r) {
+                    // gap 1: chunk r + 1's data; W^T(r) was read out before chunk r's products
+                    if (!wait_data(r + 1) || !mbar_wait(&bars[B_GAP1 + (r & 1)], (r >> 1) & 1, abort_flag)) break;
+                    DN_TS(true, r, 8);
+                    tc_fence_after();
+                    issue_w(r + 1);
+                    // gap 2: Z_H^T(r) read out of the U^T columns, chain H's update queued
+                    if (!mbar_wait(&bars[B_ZFULL], r & 1, abort_flag) ||
+                        !mbar_wait(&bars[B_GAP2 + (r & 1)], (r >> 1) & 1, abort_flag))
+                        break;
+                    DN_TS(true, r, 9);
+                    tc_fence_after();
+                    issue_u(r + 1);
+                }
+            }
+        } else if (warp >= 8 && warp < 12) {
+            // ------------------------------------------------------------ -W rows
+            const int q = warp - 8;
+            const uint32_t lane_base = (uint32_t)(32 * q) << 16;
             for (int r = 0; r < nch; ++r) {
-                // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
-                // the state update)
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
-                DN_TS(wq == 0, r, 12 + 4 * x);
+                uint8_t* stage = smem + (r % NA) * A_STAGE;
+                // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's k stage,
+                // once the stage holds the chunk (its previous chunk's products are done)
+                if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
+                                                        abort_flag)))
+                    break;
+                DN_TS(q == 0, r, 10);
                 tc_fence_after();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[32], pk[16];
-                    tmem_ld32(tmem + lane_base + tm_zu(x) + 32 * hh, v);
-                    pack_pairs<32>(v, pk);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(zs + swz128(d, 32 * hh + 8 * c)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                {
+                    RowFrags f;
+                    tmem_load_rows(tmem + lane_base + TM_WT, f);
+                    tc_fence_before();
+                    store_token_rows(f, q, stage, 8192, -1.f);
                 }
                 fence_async_smem();
-                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_ZFULL + x]);
-                DN_TS(wq == 0, r, 13 + 4 * x);
-                // S_x^T -> bf16 (and fp32 out after the last chunk); the chunk's first
-                // product (the only reader of the bf16 copy) is complete
-                if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + x], r & 1, abort_flag))) break;
-                DN_TS(wq == 0, r, 14 + 4 * x);
-                tc_fence_after();
-#pragma unroll 1
+                if (lane == 0) mbar_arrive(&bars[B_WFULL]);
+                DN_TS(q == 0, r, 11);
+            }
+        } else if (warp < 8) {
+            // ------------------------------------------------------------ chain epilogues
+            // Warp w serves chain x = w / 4 and d_v rows 32 (w % 4) .. + 31 (its lane quarter).
+            const int x = warp >> 2, wq = warp & 3;
+            const int d = 32 * wq + lane;  // d_v row of S_x^T, Z_x^T
+            const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+            if (x == 0 || TWO) {
+                // start state and destination of this chain
+                const float* x_in = nullptr;
+                float* x_out;
+                if (x == 1) {
+                    x_out = p.wsP + (int64_t)(it.slot + it.g) * D * D;
+                } else if (mode == kModeEnd) {
+                    x_in = p.s0 ? p.s0 + it.seq * p.s0_sn + it.head * p.s0_sh : nullptr;
+                    x_out = p.wsH + (int64_t)it.slot * D * D;
+                } else {
+                    x_out = p.wsH + (int64_t)(it.slot + it.g) * D * D;
+                }
+                uint8_t* zs = smem + OFF_Z + x * Z_BYTES;
+                // bf16 copy of S_x^T columns 64 hh .. + 63 of row d: chain H into tensor
+                // memory, chain P into K block hh of its shared-memory operand
+                auto store_sbf = [&](int xx, int hh, const uint32_t(&pk)[32]) {
+                    if (xx == 0) {
+                        tmem_st32(tmem + lane_base + TM_SBF + 32 * hh, pk);
+                    } else {
+                        uint8_t* sp = smem + OFF_SP + hh * 16384;
+    #pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(sp + swz128(d, 8 * c)) =
+                                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    }
+                };
+    #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t v[64], pk[32];
-                    tmem_ld64(tmem + lane_base + tm_s(x) + 64 * hh, v);
-                    pack_pairs<64>(v, pk);
-                    store_sbf(x, hh, pk);
-                    if (r == nch - 1) {
-#pragma unroll
+                    uint32_t v[64];
+    #pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const int a = 64 * hh + c;
+                        float y = 0.f;
+                        if (x_in) y = x_in[(int64_t)a * D + d];
+                        else if (x == 1) y = (a == d) ? 1.f : 0.f;
+                        v[c] = __float_as_uint(y);
+                    }
+                    if (nch == 0) {
                         for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
+                    } else {
+                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                        uint32_t pk[32];
+                        pack_pairs<64>(v, pk);
+                        store_sbf(x, hh, pk);
                     }
                 }
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
-                DN_TS(wq == 0, r, 15 + 4 * x);
+                for (int r = 0; r < nch; ++r) {
+                    // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
+                    // the state update)
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
+                    DN_TS(wq == 0, r, 12 + 4 * x);
+                    tc_fence_after();
+    #pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t v[32], pk[16];
+                        tmem_ld32(tmem + lane_base + tm_zu(x) + 32 * hh, v);
+                        pack_pairs<32>(v, pk);
+    #pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(zs + swz128(d, 32 * hh + 8 * c)) =
+                                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[B_ZFULL + x]);
+                    DN_TS(wq == 0, r, 13 + 4 * x);
+                    // S_x^T -> bf16 (and fp32 out after the last chunk); the chunk's first
+                    // product (the only reader of the bf16 copy) is complete
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + x], r & 1, abort_flag))) break;
+                    DN_TS(wq == 0, r, 14 + 4 * x);
+                    tc_fence_after();
+    #pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t v[64], pk[32];
+                        tmem_ld64(tmem + lane_base + tm_s(x) + 64 * hh, v);
+                        pack_pairs<64>(v, pk);
+                        store_sbf(x, hh, pk);
+                        if (r == nch - 1) {
+    #pragma unroll
+                            for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
+                        }
+                    }
+                    fence_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
+                    DN_TS(wq == 0, r, 15 + 4 * x);
+                }
             }
         }
-    }
+    };
+    if (mode == kModeHP) roles(std::true_type{});
+    else roles(std::false_type{});
 
     tc_fence_before();
     __syncthreads();
