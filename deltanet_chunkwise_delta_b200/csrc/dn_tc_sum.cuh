@@ -76,6 +76,21 @@ constexpr int SMEM_USED = OFF_MISC + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
+// 32 consecutive 32-bit tensor-memory columns of this thread's lane, without
+// waiting: follow with tmem_wait_st() before the columns are signalled as written.
+__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // tensor-memory columns (512 allocated), chain x = 0 (H) or 1 (P): S_x^T fp32,
 // U^T / Z_H^T and Z_P^T fp32 (64 tokens), S_H^T bf16 (128 d_k in 64 columns), W^T
 __device__ __forceinline__ uint32_t tm_s(int x) { return 128u * (uint32_t)x; }
@@ -388,7 +403,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 // memory, chain P into K block hh of its shared-memory operand
                 auto store_sbf = [&](int xx, int hh, const uint32_t(&pk)[32]) {
                     if (xx == 0) {
-                        tmem_st32(tmem + lane_base + TM_SBF + 32 * hh, pk);
+                        tmem_st32_nowait(tmem + lane_base + TM_SBF + 32 * hh, pk);
                     } else {
                         uint8_t* sp = smem + OFF_SP + hh * 16384;
     #pragma unroll
@@ -418,6 +433,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                         store_sbf(x, hh, pk);
                     }
                 }
+                tmem_wait_st();  // the bf16 copy's tensor-memory stores
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
@@ -459,6 +475,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                             for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
                         }
                     }
+                    tmem_wait_st();  // the bf16 copy's tensor-memory stores
                     fence_async_smem();
                     tc_fence_before();
                     __syncwarp();
