@@ -22,12 +22,10 @@
 //   warps 8-11  chunk-parallel epilogue: W^T -> -W token rows in shared
 //               memory; O -> global (TMA store); lane 0 of warp 8 copies each
 //               chunk's P tile in
-//   warp 12     issues the state-chain products, one thread; owns the tensor
-//               memory
+//   warp 12     issues the state-chain products and the output product that
+//               reads the chain's operand, one thread; owns the tensor memory
 //   warp 13     TMA loads of q, k (3-stage ring), one thread
-//   warp 14     issues the chunk-parallel products (W^T, U^T) and each chunk's
-//               output product O^T += Z^T P^T (behind the next chunk's U^T), one
-//               thread
+//   warp 14     issues the chunk-parallel products (U^T, W^T), one thread
 //   warp 15     TMA loads of v and bulk copies of T (2-stage ring), one thread
 // The tensor pipe runs products in issue order, and a waiting issuer thread
 // pays about 150 cycles per barrier even when the phase is already complete.
@@ -285,8 +283,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t sb = saddr(smem);
             const uint32_t i_c1 = idesc_bf16(128, 128, false, false);
             const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
+            const uint32_t i_o = idesc_bf16(128, 64, false, false);
             const uint64_t dWQ = sdesc(sb, 16, 1024);           // [-W; Q] / [Q; -W] token rows, K-major
             const uint64_t dK = sdesc(sb + A_K, 8192, 1024);    // K, MN-major
+            const uint64_t dP = sdesc(sb + OFF_PB, 16, 1024);   // P^T, K-major (+ 8 KB for odd chunks)
             for (int r = 0; r < nch; ++r) {
                 const int sa = r % NA, s = r & 1;
                 const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
@@ -316,10 +316,19 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                                  1u);
                 umma_commit(&bars[B_SFULL]);
                 mbar_arrive(&bars[B_GAP2 + s]);
+                {
+                    // O^T += Z^T P^T
+                    if (!mbar_wait(&bars[B_PFULL + s], (r >> 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const uint64_t pofs = (uint64_t)((s * 8192) >> 4);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        umma_bf16_ts(tmem + tm_o(r), tmem + TM_ZBF + 8 * j, dP + pofs + (uint64_t)((j * 32) >> 4),
+                                     i_o, 1u);
+                    umma_commit(&bars[B_OFULL]);
+                }
                 // the stage's -W, q and k are read by the products above (and k by W^T of
-                // the chunk, complete before its -W rows were written); the output product
-                // O^T += Z^T P^T is the parallel issuer's, so that this thread goes straight on
-                // to the next chunk's first product
+                // the chunk, complete before its -W rows were written)
                 umma_commit(&bars[B_EMPTYA + sa]);
                 DN_TR(true, r, 11);
             }
@@ -337,22 +346,6 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
             const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
             const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
-            const uint32_t i_o = idesc_bf16(128, 64, false, false);
-            const uint64_t dP = sdesc(sb + OFF_PB, 16, 1024);          // P^T, K-major (+ 8 KB for odd chunks)
-            // O^T(c) += Z^T(c) P^T(c), once Z^T(c) is in tensor memory (the caller waited for
-            // it) and P(c) in its buffer; commits the output barrier
-            auto issue_o = [&](int c) -> bool {
-                const int s = c & 1;
-                if (!mbar_wait(&bars[B_PFULL + s], (c >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint64_t pofs = (uint64_t)((s * 8192) >> 4);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    umma_bf16_ts(tmem + tm_o(c), tmem + TM_ZBF + 8 * j, dP + pofs + (uint64_t)((j * 32) >> 4), i_o,
-                                 1u);
-                umma_commit(&bars[B_OFULL]);
-                return true;
-            };
             auto issue_w = [&](int c) {
                 const uint64_t sta = (uint64_t)(((c % NA) * A_STAGE) >> 4);
                 const uint64_t stb = (uint64_t)(((c & 1) * B_STAGE) >> 4);
@@ -386,33 +379,20 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             for (int r = 0; ok && r + 1 < nch; ++r) {
                 // gap 1: chunk r + 1's data, chunk r's W^T read out
                 if (!wait_data(r + 1) || !mbar_wait(&bars[B_WTFREE], r & 1, abort_flag) ||
-                    !mbar_wait(&bars[B_GAP1 + (r & 1)], (r >> 1) & 1, abort_flag)) {
-                    ok = false;
+                    !mbar_wait(&bars[B_GAP1 + (r & 1)], (r >> 1) & 1, abort_flag))
                     break;
-                }
                 DN_TR(true, r, 6);
                 tc_fence_after();
                 issue_w(r + 1);
                 DN_TR(true, r, 7);
                 // gap 2: Z^T(r) read out of the U^T / Z^T columns (before its S^T update)
                 if (!mbar_wait(&bars[B_ZFREE], r & 1, abort_flag) ||
-                    !mbar_wait(&bars[B_GAP2 + (r & 1)], (r >> 1) & 1, abort_flag)) {
-                    ok = false;
+                    !mbar_wait(&bars[B_GAP2 + (r & 1)], (r >> 1) & 1, abort_flag))
                     break;
-                }
                 tc_fence_after();
                 issue_u(r + 1);
                 DN_TR(true, r, 4);
-                // chunk r's output product, behind U^T(r + 1)
-                if (!issue_o(r)) {
-                    ok = false;
-                    break;
-                }
             }
-            // the last chunk's output product
-            if (ok && nch > 0 && mbar_wait(&bars[B_ZFREE], (nch - 1) & 1, abort_flag) &&
-                mbar_wait(&bars[B_GAP2 + ((nch - 1) & 1)], ((nch - 1) >> 1) & 1, abort_flag))
-                issue_o(nch - 1);
         }
     } else if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ chunk-parallel epilogue
