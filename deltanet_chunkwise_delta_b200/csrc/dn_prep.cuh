@@ -24,7 +24,8 @@
 // memory is one 32 KB region that holds the unit's q/k tile until the product
 // has read it, and then the solve's blocks, the P tile (staged where N is
 // written later) and the T tile (staged where A was); the next unit's tile is
-// loaded once the T copy has read its staging.
+// loaded as soon as the T tile is built, its first box once the T copy has read
+// the staging.
 #pragma once
 
 #include "dn_chain.cuh"
@@ -159,17 +160,20 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
     // q/k tile of unit u (TMA, thread 0) and its step sizes into beta buffer `bb`
     // (cp.async, zero past the chunk's last token, which zeroes T's rows and
     // columns there; one group)
-    auto issue = [&](int u, int bb) {
+    // With t_staged, the T tile of the previous unit is being copied out of the first
+    // 8 KB of the region: the three other boxes go first, the Q box that overwrites the
+    // staging once the copy has read it.
+    auto issue = [&](int u, int bb, bool t_staged) {
         const int id = u / H, head = u % H;
         int b, t0, t1;
         chunk_range(p.sched, id, b, t0, t1);
         if (tid == 0) {
             sm100::mbar_expect_tx(&bars[0], 32768u);
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                sm100::tma_load_4d(smem + L::OFF_QK + a * 16384, &tq, &bars[0], a * 64, head, t0, b);
-                sm100::tma_load_4d(smem + L::OFF_QK + a * 16384 + 8192, &tk, &bars[0], a * 64, head, t0, b);
-            }
+            sm100::tma_load_4d(smem + L::OFF_QK + 8192, &tk, &bars[0], 0, head, t0, b);
+            sm100::tma_load_4d(smem + L::OFF_QK + 16384, &tq, &bars[0], 64, head, t0, b);
+            sm100::tma_load_4d(smem + L::OFF_QK + 16384 + 8192, &tk, &bars[0], 64, head, t0, b);
+            if (t_staged) sm100::bulk_wait_read0();
+            sm100::tma_load_4d(smem + L::OFF_QK, &tq, &bars[0], 0, head, t0, b);
         }
         if (tid < kChunk) {
             const bool ok = tid < t1 - t0;
@@ -182,7 +186,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
     const uint32_t i_g = sm100::idesc_bf16(128, 64, false, false);
     const uint64_t dQK = sm100::sdesc(sm100::saddr(smem + L::OFF_QK), 16, 1024);
     bool in_flight = true;
-    issue(blockIdx.x, 0);
+    issue(blockIdx.x, 0, false);
     int it_ = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++it_) {
         const int bb = it_ & 1;
@@ -392,16 +396,15 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             sm100::fence_async_smem();
         }
         __syncthreads();
-        // copy T out; once the copy has read its staging the region takes the next
-        // unit's q/k tile
+        // copy T out; the region takes the next unit's q/k tile (the box over the T
+        // staging once the copy has read it)
         const int un = u + gridDim.x;
         if (tid == 0) {
             sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes, smem + L::OFF_A, 8192);
             sm100::bulk_commit();
-            sm100::bulk_wait_read0();
         }
         if (un < units) {
-            issue(un, bb ^ 1);
+            issue(un, bb ^ 1, true);
             in_flight = true;
         }
         DN_TRP(it_, 5);
