@@ -154,6 +154,29 @@ dn_status get_ws(int dev, cudaStream_t stream, size_t bytes, StreamWs& out) {
     return DN_OK;
 }
 
+// A second stream (and a fork / join event pair) per (device, caller's stream), for
+// work that runs next to the caller's stream within one call.
+struct AuxStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::map<std::pair<int, cudaStream_t>, AuxStream> g_aux;
+
+dn_status get_aux(int dev, cudaStream_t stream, AuxStream& out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    AuxStream& a = g_aux[std::make_pair(dev, stream)];
+    if (!a.stream) {
+        if (cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess) {
+            a = AuxStream();
+            return DN_ERR_CUDA;
+        }
+    }
+    out = a;
+    return DN_OK;
+}
+
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -264,18 +287,22 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     size_t bytes = 0;
     int64_t slots = 0, nC = 0, nA = 0, nScan = 0;
     int G = 1, s = 1;
+    bool e_in_c = false;
     if (!d.varlen) {
         if (forced_s > 0) {
             s = forced_s;
         } else {
-            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots);
+            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, kTc);
             s = ch.s;
         }
         G = n_c_max > 0 ? (int)((n_c_max + s - 1) / s) : 1;
         slots = chains * (G - 1);
         if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
         nC = chains * G;
-        nA = G >= 2 ? chains * (G - 1) : 0;
+        // tensor-core path: run 0 of a split chain is computed once, by its boundary item,
+        // next to the summary pass (which then has no end-state items)
+        e_in_c = kTc && G >= 2;
+        nA = G >= 2 ? chains * (G - 1 - (e_in_c ? 1 : 0)) : 0;
         nScan = G >= 2 ? chains : 0;
     } else {
         if (forced_s > 0) {
@@ -320,6 +347,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         sc.H = (int)d.H;
         sc.n_chunks = (int)n_c_max;
         sc.G = G;
+        sc.e_in_c = e_in_c ? 1 : 0;
         sc.s = s;
         g_last_G = G;
         g_last_s = s;
@@ -362,11 +390,35 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
             ++launches;
         }
-        if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
-        if (nScan > 0) { launch_scan(); ++launches; }
-        if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-        if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
-        if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
+        if (e_in_c) {
+            // run 0 of every chain (with outputs and its end state) on a second stream, next
+            // to the summary pass, which leaves SMs free; the scan waits for both
+            AuxStream aux;
+            if ((st = get_aux(dev, stream, aux)) != DN_OK) return st;
+            Params p0 = p;
+            p0.sched.c_part = 1;
+            if (cudaEventRecord(aux.fork, stream) != cudaSuccess ||
+                cudaStreamWaitEvent(aux.stream, aux.fork, 0) != cudaSuccess)
+                return DN_ERR_CUDA;
+            kCt<<<(unsigned)chains, tc::kThreadsTc, tc::SMEM_BYTES, aux.stream>>>(tq, tk, tv, to, p0);
+            ++launches;
+            if (cudaEventRecord(aux.join, aux.stream) != cudaSuccess) return DN_ERR_CUDA;
+            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
+            if (cudaStreamWaitEvent(stream, aux.join, 0) != cudaSuccess) return DN_ERR_CUDA;
+            if (nScan > 0) { launch_scan(); ++launches; }
+            Params p1 = p;
+            p1.sched.c_part = 2;
+            if (g_ev_start) cudaEventRecord(g_ev_start, stream);
+            kCt<<<(unsigned)(chains * (G - 1)), tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p1);
+            ++launches;
+            if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
+        } else {
+            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
+            if (nScan > 0) { launch_scan(); ++launches; }
+            if (g_ev_start) cudaEventRecord(g_ev_start, stream);
+            if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
+            if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
+        }
     } else {
         if (nA > 0) { kA<<<(unsigned)nA, kThreads, smemA, stream>>>(p); ++launches; }
         if (nScan > 0) { launch_scan(); ++launches; }

@@ -50,6 +50,8 @@ struct Sched {
     int list;           // 0 = dense, 1 = list
     int B, T, H;        // dense shape
     int n_chunks, G, s; // dense segmentation
+    int e_in_c;         // dense: run 0's end state comes from the boundary pass (no E items)
+    int c_part;         // dense boundary items: 0 all runs, 1 run 0 only, 2 runs 1..G-1
     const Item* itemsC;     // list: boundary-pass items
     const Item* itemsA;     // list: summary items; Item.g carries mode in bits 16+
     const Item* itemsScan;  // list: one per chain with G >= 2
@@ -99,10 +101,12 @@ __device__ __forceinline__ void dense_chain_item(const Sched& s, int chain, int 
 }
 
 __device__ __forceinline__ int count_C(const Sched& s) {
-    return s.list ? s.counts[0] : s.B * s.H * s.G;
+    if (s.list) return s.counts[0];
+    const int runs = s.c_part == 0 ? s.G : (s.c_part == 1 ? 1 : s.G - 1);
+    return s.B * s.H * runs;
 }
 __device__ __forceinline__ int count_A(const Sched& s) {
-    return s.list ? s.counts[1] : (s.G >= 2 ? s.B * s.H * (s.G - 1) : 0);
+    return s.list ? s.counts[1] : (s.G >= 2 ? s.B * s.H * (s.G - 1 - s.e_in_c) : 0);
 }
 __device__ __forceinline__ int count_scan(const Sched& s) {
     return s.list ? s.counts[2] : (s.G >= 2 ? s.B * s.H : 0);
@@ -111,11 +115,14 @@ __device__ __forceinline__ int count_scan(const Sched& s) {
 __device__ __forceinline__ Item item_C(const Sched& s, int i) {
     Item it;
     if (s.list) return s.itemsC[i];
-    dense_chain_item(s, i / s.G, i % s.G, it);
+    if (s.c_part == 0) dense_chain_item(s, i / s.G, i % s.G, it);
+    else if (s.c_part == 1) dense_chain_item(s, i, 0, it);
+    else dense_chain_item(s, i / (s.G - 1), 1 + i % (s.G - 1), it);
     return it;
 }
 
-// Summary items: per chain, [End(g=0), HP(1), HP(2), ..., HP(G-2)].
+// Summary items: per chain, [End(g=0), HP(1), HP(2), ..., HP(G-2)], or without the End
+// item when the boundary pass's run-0 item writes run 0's end state (e_in_c).
 __device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
     Item it;
     if (s.list) {
@@ -124,8 +131,8 @@ __device__ __forceinline__ Item item_A(const Sched& s, int i, int& mode) {
         it.g &= 0xffff;
         return it;
     }
-    const int per = s.G - 1;
-    const int chain = i / per, r = i % per;
+    const int per = s.G - 1 - s.e_in_c;
+    const int chain = i / per, r = i % per + s.e_in_c;
     mode = r == 0 ? kModeEnd : kModeHP;
     dense_chain_item(s, chain, r, it);
     return it;

@@ -31,11 +31,14 @@ struct SegChoice {
     float cost;
 };
 
-// Cost of run length s for `chains` chains of equal length n_c (dense input).
+// Cost of run length s for `chains` chains of equal length n_c (dense input).  With
+// e_in_c, run 0 of a split chain is computed once, by its boundary item, which runs
+// next to the summary items (so the summary phase has G - 1 items per chain, the
+// boundary phase after the scan G - 1 more).
 __host__ __device__ inline float dense_cost(const CostModel& m, int chains, int n_c, int s,
-                                            int slots) {
+                                            int slots, bool e_in_c = false) {
     const int G = n_c > 0 ? (n_c + s - 1) / s : 1;
-    const long long runs = (long long)chains * G;
+    const long long runs = (long long)chains * ((e_in_c && G >= 2) ? G - 1 : G);
     const long long summ = G >= 2 ? (long long)chains * (G - 1) : 0;
     const float wC = (float)((runs + slots - 1) / slots);
     const float wA = (float)((summ + slots - 1) / slots);
@@ -43,14 +46,14 @@ __host__ __device__ inline float dense_cost(const CostModel& m, int chains, int 
 }
 
 inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots,
-                              int max_slots) {
+                              int max_slots, bool e_in_c = false) {
     SegChoice best{n_c > 0 ? n_c : 1, 3.0e38f};
     if (n_c <= 0) return {1, 0.f};
     for (int G = 1; G <= 256 && G <= n_c; ++G) {
         const int s = (n_c + G - 1) / G;
         const int Gs = (n_c + s - 1) / s;
         if ((long long)chains * (Gs - 1) > max_slots) break;
-        const float cst = dense_cost(m, chains, n_c, s, slots);
+        const float cst = dense_cost(m, chains, n_c, s, slots, e_in_c);
         if (cst < best.cost) best = {s, cst};
     }
     return best;

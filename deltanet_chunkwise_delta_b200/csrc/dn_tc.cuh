@@ -226,7 +226,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
     // start state and destination of the run
     const float* s0 = p.s0 ? p.s0 + it.seq * p.s0_sn + it.head * p.s0_sh : nullptr;
     const float* x_in = it.g == 0 ? s0 : p.wsS + (int64_t)(it.slot + it.g - 1) * D * D;
+    // the last run writes the final state; with e_in_c, run 0 of a split chain writes its
+    // end state where the segment scan reads it
     float* x_out = (it.g == it.G - 1 && p.sT) ? p.sT + it.seq * p.sT_sn + it.head * p.sT_sh : nullptr;
+    if (it.g == 0 && it.G >= 2 && !p.sched.list && p.sched.e_in_c) x_out = p.wsH + (int64_t)it.slot * D * D;
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ ring A: q, k
