@@ -9,10 +9,13 @@ Two independent float64 statements of the method:
 
 * ``token_recurrence`` -- the plain definition, a C float64 token-serial loop
   ("Linear Attention, Visualized", DeltaNet, "Recurrent form"), threaded over
-  (sequence, head).  Built from ``deltanet_oracle.c`` with gcc.
+  (sequence, head); with a gate ``g`` = ln a_t it runs the Gated DeltaNet
+  recurrence of the same page (section "Gated DeltaNet (GDN)").  Built from
+  ``deltanet_oracle.c`` with gcc.
 * ``chunkwise`` (module) -- numpy float64 statements of the chunk form, the
   WY transition product, the segment composition and the full-sequence closed
-  form, for tiny inputs.
+  form, for tiny inputs, and of the gated chunk form ("Complete per-chunk
+  algorithm" of the GDN section).
 """
 from __future__ import annotations
 
@@ -39,7 +42,7 @@ def build(force: bool = False) -> str:
             os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
-                               "-o", tmp, _SRC])
+                               "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -49,10 +52,11 @@ def _load():
     with _lock:
         if _lib is None:
             lib = ctypes.CDLL(build())
-            f = lib.dn_oracle_fwd
+            f = lib.gdn_oracle_fwd
             f.restype = ctypes.c_int
             f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
-                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                          ctypes.c_int64,
                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
@@ -66,11 +70,12 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
                      heads=None, out_dtype=torch.float64, want_out=True,
-                     n_threads: Optional[int] = None):
+                     n_threads: Optional[int] = None, g=None):
     """Run the float64 token recurrence on CPU tensors.
 
     q, k: [B, T, H, dk]; v: [B, T, H, dv] (fp32, bf16 or fp64); beta: [B, T, H]
-    fp32; initial_state: [N, H, dk, dv] or None; cu_seqlens: int32 [N+1] or None.
+    fp32; initial_state: [N, H, dk, dv] or None; cu_seqlens: int32 [N+1] or None;
+    g: [B, T, H] fp32 log decay (Gated DeltaNet) or None (plain DeltaNet).
     ``heads``: (h_begin, h_end) to compute a subset of heads (others are NaN).
     Returns (out [B, T, H, dv] in ``out_dtype`` or None, final_state [N, H, dk, dv]
     float64).
@@ -78,6 +83,7 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
     lib = _load()
     q = q.contiguous(); k = k.contiguous(); v = v.contiguous()
     beta = beta.to(torch.float32).contiguous()
+    gate = None if g is None else g.to(torch.float32).contiguous()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     codes = {torch.float32: 0, torch.bfloat16: 1, torch.float64: 2}
@@ -98,10 +104,12 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
     fs = torch.full((n_seq, H, dk, dv), float("nan"), dtype=torch.float64)
     if n_threads is None:
         n_threads = os.cpu_count() or 1
-    rc = lib.dn_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta), _ptr(s0),
-                           _ptr(cu), n_seq, B, T, H, dk, dv, h0, h1,
-                           _ptr(out), 0 if out_dtype == torch.float32 else 2,
-                           _ptr(fs), int(n_threads))
+    if gate is not None and tuple(gate.shape) != tuple(beta.shape):
+        raise ValueError("g must have the shape of beta")
+    rc = lib.gdn_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta), _ptr(gate),
+                            _ptr(s0), _ptr(cu), n_seq, B, T, H, dk, dv, h0, h1,
+                            _ptr(out), 0 if out_dtype == torch.float32 else 2,
+                            _ptr(fs), int(n_threads))
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return out, fs

@@ -164,3 +164,114 @@ def linear_attention(Q, K, V):
     """Causal linear attention, parallel form (Q K^T o M) V."""
     M, _ = causal_masks(K.shape[0])
     return ((Q @ K.T) * M) @ V
+
+
+# --- Gated DeltaNet ("Linear Attention, Visualized", section "Gated DeltaNet (GDN)") ---
+#
+# Every function below takes the per-token decays a (shape [n], 0 < a <= 1)
+# next to beta; the recurrence is S_t = a_t (I - beta_t k_t^T k_t) S_{t-1}
+# + beta_t k_t^T v_t.
+
+def decay_products(a):
+    """lambda[i:j] = prod_{s=i}^{j} a_s with 1-based inclusive bounds, and 1 when
+    i > j ("Complete per-chunk algorithm" of the GDN section)."""
+    def lam(i, j):
+        return float(np.prod(a[i - 1:j])) if i <= j else 1.0
+    return lam
+
+
+def gated_chunk_factors(Kc, Vc, bc, ac):
+    """Per-chunk quantities of the GDN chunk algorithm, taken as the page
+    defines them:
+      Gamma[l, i] = lambda[i+1:l] for i <= l, else 0 (1-based l, i);
+      left-decayed rows  q<-_l = lambda[1:l] q_l,  k<-_l = lambda[1:l] k_l;
+      right-decayed rows k->_l = lambda[l+1:C] k_l;
+      L = (K K^T o Gamma) o M_c^-, (I + B L) T = B, U = T V, W<- = T K<-.
+    Returns a dict with Gamma, L, T, U, W (= W<-), Kl (= K<-), Kr (= K->),
+    left (the lambda[1:l] column) and lamC (= lambda[1:C])."""
+    c = Kc.shape[0]
+    lam = decay_products(ac)
+    Gam = np.zeros((c, c))
+    for l in range(c):
+        for i in range(l + 1):
+            Gam[l, i] = lam(i + 2, l + 1)
+    left = np.array([lam(1, l + 1) for l in range(c)])
+    right = np.array([lam(l + 2, c) for l in range(c)])
+    _, Mm = causal_masks(c)
+    Bm = np.diag(bc)
+    L = ((Kc @ Kc.T) * Gam) * Mm
+    T = solve_triangular(np.eye(c) + Bm @ L, Bm, lower=True, unit_diagonal=True)
+    Kl = left[:, None] * Kc
+    Kr = right[:, None] * Kc
+    return {"Gamma": Gam, "L": L, "T": T, "U": (T @ Vc if Vc is not None else None),
+            "W": T @ Kl, "Kl": Kl, "Kr": Kr, "left": left, "lamC": lam(1, c)}
+
+
+def gated_chunk_step(Qc, Kc, Vc, bc, ac, S):
+    """One chunk of the GDN boundary pass: Z = U - W<- S,
+    O = Q<- S + (Q K^T o Gamma) Z, S' = lambda[1:C] S + K->^T Z.
+    Returns (O_chunk, S')."""
+    f = gated_chunk_factors(Kc, Vc, bc, ac)
+    Z = f["U"] - f["W"] @ S
+    O = (f["left"][:, None] * Qc) @ S + ((Qc @ Kc.T) * f["Gamma"]) @ Z
+    return O, f["lamC"] * S + f["Kr"].T @ Z
+
+
+def gated_chunkwise(Q, K, V, beta, a, S0=None, C: int = 64):
+    """The GDN per-chunk algorithm threaded over all chunks from S0.
+    Returns (O, S_final)."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    O = np.zeros((n, dv))
+    for s, e in chunk_bounds(n, C):
+        O[s:e], S = gated_chunk_step(Q[s:e], K[s:e], V[s:e], beta[s:e], a[s:e], S)
+    return O, S
+
+
+def gated_segment_map(K, V, beta, a, C: int = 64):
+    """Affine map S_end = P S_start + H of a run of chunks under GDN: one chunk
+    is S' = (lambda[1:C] I - K->^T W<-) S + K->^T U, and chunks compose in order
+    as in ``segment_map``.  Returns (P, H)."""
+    dk = K.shape[1]
+    P = np.eye(dk)
+    H = np.zeros((dk, V.shape[1]))
+    for s, e in chunk_bounds(K.shape[0], C):
+        f = gated_chunk_factors(K[s:e], V[s:e], beta[s:e], a[s:e])
+        Lam = f["lamC"] * np.eye(dk) - f["Kr"].T @ f["W"]
+        Hr = f["Kr"].T @ f["U"]
+        P, H = Lam @ P, Lam @ H + Hr
+    return P, H
+
+
+def gated_context_parallel(Q, K, V, beta, a, S0=None, C: int = 64, n_segments: int = 2):
+    """``context_parallel`` with the GDN chunk maps.  Returns (O, S_final)."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    chunks = chunk_bounds(n, C)
+    nc = len(chunks)
+    n_segments = max(1, min(n_segments, nc))
+    edges = [round(g * nc / n_segments) for g in range(n_segments + 1)]
+    segs = [(chunks[edges[g]][0], chunks[edges[g + 1] - 1][1]) for g in range(n_segments)]
+    maps = [gated_segment_map(K[s:e], V[s:e], beta[s:e], a[s:e], C) for s, e in segs]
+    starts = [np.zeros((dk, dv)) if S0 is None else S0.copy()]
+    for P, H in maps[:-1]:
+        starts.append(P @ starts[-1] + H)
+    O = np.zeros((n, dv))
+    S = None
+    for (s, e), Sg in zip(segs, starts):
+        O[s:e], S = gated_chunkwise(Q[s:e], K[s:e], V[s:e], beta[s:e], a[s:e], Sg, C)
+    return O, S
+
+
+def decayed_linear_attention(Q, K, V, a):
+    """Linear attention with scalar decay (the Mamba-2 row of the page's table,
+    one chunk spanning the sequence, zero start): O = (Q K^T o D) V with
+    D[t, s] = lambda[s+1:t] for s <= t."""
+    n = K.shape[0]
+    lam = decay_products(a)
+    D = np.zeros((n, n))
+    for t in range(n):
+        for s in range(t + 1):
+            D[t, s] = lam(s + 2, t + 1)
+    return ((Q @ K.T) * D) @ V

@@ -16,18 +16,25 @@
  *
  * This is the column-convention recurrence S_t = S_{t-1}(I - b k k^T) + b v k^T,
  * o_t = S_t q_t of "Context Parallelism for DeltaNet" (section 2) transposed.
+ * Gated DeltaNet (same page, section "Gated DeltaNet (GDN)") multiplies the
+ * whole transition by a per-token scalar decay a_t,
+ *     S_t = a_t (I - beta_t k_t^T k_t) S_{t-1} + beta_t k_t^T v_t,
+ * so with a gate the loop first decays the state, S <- a_t S_{t-1}, and then
+ * makes the same prediction, correction and write from the decayed state.
+ * The gate arrives as g_t = ln a_t (fp32 [B, T, H]); a_t = exp(g_t) in float64.
  * S starts from the caller's initial state (or zero) at the first token of each
  * sequence.  No query scaling is applied.  Inputs stored as bf16 are widened
  * exactly to float64; every sum is accumulated in float64.
  *
  * Layouts (contiguous, row-major):
- *   q, k   [B, T, H, dk]     v, out [B, T, H, dv]     beta [B, T, H] (fp32)
+ *   q, k   [B, T, H, dk]     v, out [B, T, H, dv]     beta, gate [B, T, H] (fp32)
  *   init_state, final_state [N, H, dk, dv]
  * With cu_seqlens (host int32 [N+1]) B must be 1 and sequence n covers tokens
  * cu[n] .. cu[n+1]-1; without it N = B and sequence n is batch row n.
  * Only heads h_begin .. h_end-1 are computed; other heads' outputs are left
  * untouched.  out may be NULL (state only).
  */
+#include <math.h>
 #include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -50,6 +57,7 @@ typedef struct {
     const void *q, *k, *v;
     int in_dtype;
     const float* beta;
+    const float* gate;          /* g = ln a, or NULL (no decay) */
     const double* init_state;   /* float64 copy or NULL */
     const int32_t* cu;
     int64_t n_seq, B, T, H, dk, dv, h_begin, h_end;
@@ -83,6 +91,11 @@ static void run_job(oracle_ctx* c, int64_t job, double* S, double* kt, double* q
         const int64_t qk_off = (tok * H + h) * dk;
         const int64_t v_off = (tok * H + h) * dv;
         const double b = (double)c->beta[tok * H + h];
+        if (c->gate) {
+            /* decay first: the prediction below reads a_t S_{t-1} */
+            const double a = exp((double)c->gate[tok * H + h]);
+            for (int64_t e = 0; e < dk * dv; ++e) S[e] *= a;
+        }
         for (int64_t a = 0; a < dk; ++a) {
             kt[a] = load_elt(c->k, c->in_dtype, qk_off + a);
             qt[a] = load_elt(c->q, c->in_dtype, qk_off + a);
@@ -126,13 +139,14 @@ static void* worker(void* arg) {
     return NULL;
 }
 
-/* Returns 0 on success, -1 on a bad argument, -2 on allocation failure. */
-int dn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
-                  const float* beta, const double* init_state,
-                  const int32_t* cu_seqlens, int64_t n_seq,
-                  int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
-                  int64_t h_begin, int64_t h_end,
-                  void* out, int out_dtype, double* final_state, int n_threads) {
+/* Returns 0 on success, -1 on a bad argument, -2 on allocation failure.
+ * gate may be NULL (plain DeltaNet). */
+int gdn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+                   const float* beta, const float* gate, const double* init_state,
+                   const int32_t* cu_seqlens, int64_t n_seq,
+                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                   int64_t h_begin, int64_t h_end,
+                   void* out, int out_dtype, double* final_state, int n_threads) {
     if ((B * T > 0) && (!q || !k || !v || !beta)) return -1;
     if (in_dtype != OR_F32 && in_dtype != OR_BF16 && in_dtype != OR_F64) return -1;
     if (out_dtype != OR_F32 && out_dtype != OR_F64) return -1;
@@ -147,7 +161,7 @@ int dn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     }
     oracle_ctx c;
     memset(&c, 0, sizeof c);
-    c.q = q; c.k = k; c.v = v; c.in_dtype = in_dtype; c.beta = beta;
+    c.q = q; c.k = k; c.v = v; c.in_dtype = in_dtype; c.beta = beta; c.gate = gate;
     c.init_state = init_state; c.cu = cu_seqlens; c.n_seq = n_seq;
     c.B = B; c.T = T; c.H = H; c.dk = dk; c.dv = dv;
     c.h_begin = h_begin; c.h_end = h_end;
@@ -169,4 +183,15 @@ int dn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     free(th);
     pthread_mutex_destroy(&c.lock);
     return 0;
+}
+
+/* Plain DeltaNet: the gated loop with every a_t = 1 (no decay step at all). */
+int dn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+                  const float* beta, const double* init_state,
+                  const int32_t* cu_seqlens, int64_t n_seq,
+                  int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                  int64_t h_begin, int64_t h_end,
+                  void* out, int out_dtype, double* final_state, int n_threads) {
+    return gdn_oracle_fwd(q, k, v, in_dtype, beta, NULL, init_state, cu_seqlens, n_seq, B, T, H,
+                          dk, dv, h_begin, h_end, out, out_dtype, final_state, n_threads);
 }

@@ -33,3 +33,18 @@ def test_config_shapes():
     assert (W["long_65k"].T, W["long_65k"].H, W["long_65k"].init_state) == (65536, 16, True)
     assert (W["ctx_1m"].T, W["ctx_1m"].H) == (1 << 20, 8)
     assert W["tiny_fp32"].dtype == torch.float32 and W["tiny_fp32"].dk == 64
+
+
+def test_gate_recipe():
+    """Gated workloads add g = logsigmoid(N(0,1) + 4) after the other draws, so
+    their q, k, v, beta and initial state equal the plain workload's."""
+    w = wl.custom(1, 4096, 2, 64, 64, torch.bfloat16, init_state=True, gated=True)
+    a = wl.generate(w, seed=5)
+    b = wl.generate(wl.custom(1, 4096, 2, 64, 64, torch.bfloat16, init_state=True), seed=5)
+    for key in ("q", "k", "v", "beta", "initial_state"):
+        assert torch.equal(a[key], b[key])
+    assert b["g"] is None and a["g"].shape == (1, 4096, 2) and a["g"].dtype == torch.float32
+    assert (a["g"] < 0).all()
+    med = float(a["g"].exp().median())
+    assert 0.97 < med < 0.99
+    assert wl.WORKLOADS["gdn_65k"].gated and not wl.WORKLOADS["long_65k"].gated
