@@ -3,7 +3,7 @@
 
 One step = one deltanet_fwd call over the whole workload (every step of the
 path: WY/UT factors, segment summaries, segment scan, boundary pass with
-output).  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
+output); for the Gated DeltaNet workloads (gdn_*) one gated_deltanet_fwd call.  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
 d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 beta, zero initial state, fp32
 final state), synthetic seeded inputs.  Inputs (q, k, v: 201 MB) exceed the
 126 MB L2, so no flush is needed between steps.
@@ -50,11 +50,11 @@ def flops_per_token_head(dk: int, dv: int, C: int = CHUNK) -> float:
 
 
 def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
-    """q, k, v, o once each, beta once, initial state read if given, final
-    state written."""
+    """q, k, v, o once each, beta once (and the log decay g once for Gated
+    DeltaNet), initial state read if given, final state written."""
     es = 2 if w.dtype == torch.bfloat16 else 4
     th = w.tokens * w.H
-    b = th * (es * (2 * w.dk + 2 * w.dv) + 4)
+    b = th * (es * (2 * w.dk + 2 * w.dv) + 4 + (4 if w.gated else 0))
     st = w.n_seq * w.H * w.dk * w.dv * 4
     if w.init_state:
         b += st
@@ -200,9 +200,10 @@ def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0):
     n_threads = os.cpu_count() or 1
     sl = lambda t: t[b:b + 1, :tokens].contiguous()
     s0 = None if x["initial_state"] is None else x["initial_state"][b:b + 1].contiguous()
+    gate = None if x.get("g") is None else sl(x["g"])
     t0 = time.perf_counter()
     oracle.token_recurrence(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]), s0,
-                            n_threads=n_threads)
+                            n_threads=n_threads, g=gate)
     return time.perf_counter() - t0, min(n_threads, w.H)
 
 
@@ -255,9 +256,16 @@ def run_b200(args, w: wl.Workload):
     fs = torch.empty((w.n_seq, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
+    def call(d, o, f):
+        if w.gated:
+            dn.gated_deltanet_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["initial_state"],
+                                  d["cu_seqlens"], out=o, final_state=f, stream=stream)
+        else:
+            dn.deltanet_fwd(d["q"], d["k"], d["v"], d["beta"], d["initial_state"],
+                            d["cu_seqlens"], out=o, final_state=f, stream=stream)
+
     def step():
-        dn.deltanet_fwd(g["q"], g["k"], g["v"], g["beta"], g["initial_state"], g["cu_seqlens"],
-                        out=out, final_state=fs, stream=stream)
+        call(g, out, fs)
 
     step()
     if dn.get_error(stream) != 0:
@@ -297,10 +305,10 @@ def run_b200(args, w: wl.Workload):
     tflops = ws * th * flops_per_token_head(w.dk, w.dv) / (ms / 1e3) / 1e12
     hbm_peak, tc_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(w)
-    # the boundary (output) kernel moves q, k, v, o and the states; beta is read by the
-    # UT pre-pass
-    kernel_bytes = alg_bytes - 4.0 * w.tokens * w.H
-    tc_path = w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+    tc_path = not w.gated and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+    # the tensor-core boundary kernel moves q, k, v, o and the states (beta is read by the
+    # UT pre-pass); the mma.sync boundary kernel reads beta (and g) itself
+    kernel_bytes = alg_bytes - (4.0 * w.tokens * w.H if tc_path else 0.0)
     if tc_path and w.seqlens is None and G >= 2:
         # split dense chains: run 0 of every chain is computed by its own launch next to
         # the summary pass; the timed launch covers runs 1..G-1 (q, k, v, o of their
@@ -309,7 +317,7 @@ def run_b200(args, w: wl.Workload):
         th_b = w.B * (w.T - s * CHUNK) * w.H
         kernel_bytes = float(th_b * es * (2 * w.dk + 2 * w.dv) + w.n_seq * w.H * w.dk * w.dv * 4)
     achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9
-    tc_kernel = w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+    tc_kernel = tc_path
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
                 "traffic": stored_traffic(w.name) if tc_kernel else None,
@@ -366,8 +374,7 @@ def run_b200(args, w: wl.Workload):
                 ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_read[b])          # this set's previous outputs are downloaded
-            dn.deltanet_fwd(di["q"], di["k"], di["v"], di["beta"], di["initial_state"],
-                            di["cu_seqlens"], out=o_b, final_state=fs_b, stream=stream)
+            call(di, o_b, fs_b)
             ev_done[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[b])
@@ -413,7 +420,8 @@ def run_b200(args, w: wl.Workload):
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
                    "chunk": CHUNK, "segments_per_chain": G, "chunks_per_segment": s,
-                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}"},
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}",
+                   "variant": "gated DeltaNet" if w.gated else "DeltaNet"},
         "tflops": tflops,
         "tflops_unit": "algorithmic TFLOP/s (6Cd^2 + 5C^2d + C^3/3 per chunk-head)",
         "roofline": roofline,

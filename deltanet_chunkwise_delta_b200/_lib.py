@@ -21,7 +21,8 @@ DN_OK, DN_ERR_INVALID_ARG, DN_ERR_UNSUPPORTED, DN_ERR_ALIAS, DN_ERR_CUDA, \
     DN_ERR_WORKSPACE, DN_ERR_SEQLENS, DN_ERR_TIMEOUT = range(8)
 DN_F32, DN_BF16, DN_I32 = 0, 1, 2
 
-EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "deltanet_status_string",
+EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "gated_deltanet_fwd", "gated_deltanet_fwd_ex",
+            "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
             "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events")
 
@@ -63,6 +64,12 @@ def load(path: Optional[str] = None):
         lib.deltanet_fwd_ex.restype = ctypes.c_int
         lib.deltanet_fwd_ex.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p,
                                         ctypes.c_int]
+        lib.gated_deltanet_fwd.restype = ctypes.c_int
+        lib.gated_deltanet_fwd.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P,
+                                           ctypes.c_void_p]
+        lib.gated_deltanet_fwd_ex.restype = ctypes.c_int
+        lib.gated_deltanet_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P,
+                                              ctypes.c_void_p, ctypes.c_int]
         lib.deltanet_fwd_noalloc.restype = ctypes.c_int
         lib.deltanet_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
         lib.deltanet_status_string.restype = ctypes.c_char_p
@@ -122,6 +129,17 @@ def call(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
     return lib.deltanet_fwd(*args, stream)
 
 
+def call_gated(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+               stream, seg_chunks: int = 0) -> int:
+    """Raw Gated DeltaNet call: returns the dn_status code (no exception)."""
+    lib = load()
+    ds = [describe(t) for t in (q, k, v, beta, g, initial_state, cu_seqlens, out, final_state)]
+    args = [_ref(x) for x in ds[:7]] + [int(chunk_size)] + [_ref(x) for x in ds[7:]]
+    if seg_chunks:
+        return lib.gated_deltanet_fwd_ex(*args, stream, int(seg_chunks))
+    return lib.gated_deltanet_fwd(*args, stream)
+
+
 def _stream_handle(device, stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -153,6 +171,33 @@ def deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.
         final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     st = call(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
               _stream_handle(q.device, stream), seg_chunks)
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state
+
+
+def gated_deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.Tensor,
+                       g: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+                       cu_seqlens: Optional[torch.Tensor] = None, chunk_size: int = 64,
+                       out: Optional[torch.Tensor] = None,
+                       final_state: Optional[torch.Tensor] = None,
+                       output_final_state: bool = True, stream=None, seg_chunks: int = 0):
+    """Gated DeltaNet forward on CUDA tensors through the C ABI.
+
+    As ``deltanet_fwd``, plus ``g`` [B, T, H] fp32: the per-token decay as its
+    natural log, g = ln a (the state update is S <- a (I - beta k^T k) S + beta k^T v).
+    """
+    if not q.is_cuda:
+        raise ValueError("gated_deltanet_fwd runs on CUDA tensors only")
+    B, T, H, _ = q.shape
+    dk, dv = q.shape[3], v.shape[3]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = call_gated(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    _stream_handle(q.device, stream), seg_chunks)
     if st != DN_OK:
         raise DeltaNetError(st, status_string(st))
     return out, final_state

@@ -238,19 +238,21 @@ struct Dims {
     bool varlen;
 };
 
-template <typename E, int DK, int DV, int STAGES>
+template <typename E, int DK, int DV, int STAGES, bool GATED>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
-    // bf16 with d_k = d_v = 128 runs on the tensor-core (tcgen05) chain kernel
-    constexpr bool kTc = std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
-    using LC = ChainSmem<E, DK, DV, true, true, STAGES>;
-    using LH = ChainSmem<E, DK, DV, true, false, STAGES>;
-    using LP = ChainSmem<E, DK, DK, false, false, STAGES>;
+    // bf16 DeltaNet with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels; Gated
+    // DeltaNet and the other shapes on the mma.sync chain kernels
+    constexpr bool kTc =
+        !GATED && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
+    using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED>;
+    using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED>;
+    using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED>;
     const int smemC = LC::TOTAL;
     const int smemA = LH::TOTAL > LP::TOTAL ? LH::TOTAL : LP::TOTAL;
     const int smemS8 = scan_smem_bytes<DK, 8>(), smemS16 = scan_smem_bytes<DK, 16>();
-    auto* kC = k_boundary<E, DK, DV, STAGES>;
-    auto* kA = k_summary<E, DK, DV, STAGES>;
+    auto* kC = k_boundary<E, DK, DV, STAGES, GATED>;
+    auto* kA = k_summary<E, DK, DV, STAGES, GATED>;
     auto* kS8 = k_scan<DK, DV, 8>;
     auto* kS16 = k_scan<DK, DV, 16>;
     auto* kCt = tc::k_tc_chain;
@@ -431,9 +433,25 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     return DN_OK;
 }
 
+template <bool GATED>
+dn_status dispatch(Params& p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
+                   const int* cup, int32_t dt) {
+    const int64_t dk = d.dk, dv = d.dv;
+    if (dt == DN_F32) return launch<float, 64, 64, 1, GATED>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 128 && dv == 128)
+        return launch<__nv_bfloat16, 128, 128, 2, GATED>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 128 && dv == 64)
+        return launch<__nv_bfloat16, 128, 64, 2, GATED>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 64 && dv == 128)
+        return launch<__nv_bfloat16, 64, 128, 2, GATED>(p, d, dev, sms, stream, forced_s, cup);
+    return launch<__nv_bfloat16, 64, 64, 2, GATED>(p, d, dev, sms, stream, forced_s, cup);
+}
+
+// gate: Gated DeltaNet's log decay [B, T, H] fp32, or null for DeltaNet.
 dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
-                   const dn_tensor* beta, const dn_tensor* s0, const dn_tensor* cu, int chunk,
-                   dn_tensor* out, dn_tensor* sT, void* stream_ptr, int forced_s) {
+                   const dn_tensor* beta, const dn_tensor* gate, const dn_tensor* s0,
+                   const dn_tensor* cu, int chunk, dn_tensor* out, dn_tensor* sT,
+                   void* stream_ptr, int forced_s) {
     if (!q || !k || !v || !beta || !out) return DN_ERR_INVALID_ARG;
     if (q->ndim != 4 || k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return DN_ERR_INVALID_ARG;
     if (forced_s < 0) return DN_ERR_INVALID_ARG;
@@ -454,6 +472,13 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
         if (beta->stride[i] < 0) return DN_ERR_INVALID_ARG;
     if (numel(beta) > 0 && (!beta->data || (reinterpret_cast<uintptr_t>(beta->data) & 3)))
         return DN_ERR_INVALID_ARG;
+    if (gate) {
+        if (!shape_eq(gate, 3, bd) || gate->dtype != DN_F32) return DN_ERR_INVALID_ARG;
+        for (int i = 0; i < 3; ++i)
+            if (gate->stride[i] < 0) return DN_ERR_INVALID_ARG;
+        if (numel(gate) > 0 && (!gate->data || (reinterpret_cast<uintptr_t>(gate->data) & 3)))
+            return DN_ERR_INVALID_ARG;
+    }
     if (B * T >= (int64_t(1) << 31) || H >= 65536) return DN_ERR_INVALID_ARG;
 
     int64_t N = B;
@@ -476,7 +501,7 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     if (dt == DN_BF16 ? !bf16_ok : !f32_ok) return DN_ERR_UNSUPPORTED;
 
     // aliasing: outputs against inputs and each other
-    const dn_tensor* ins[6] = {q, k, v, beta, s0, cu};
+    const dn_tensor* ins[7] = {q, k, v, beta, gate, s0, cu};
     for (const dn_tensor* o : {static_cast<const dn_tensor*>(out), static_cast<const dn_tensor*>(sT)}) {
         if (!o) continue;
         for (const dn_tensor* in : ins)
@@ -500,20 +525,18 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     p.v_sb = v->stride[0]; p.v_st = v->stride[1]; p.v_sh = v->stride[2];
     p.o_sb = out->stride[0]; p.o_st = out->stride[1]; p.o_sh = out->stride[2];
     p.b_sb = beta->stride[0]; p.b_st = beta->stride[1]; p.b_sh = beta->stride[2];
+    if (gate) {
+        p.g = static_cast<const float*>(gate->data);
+        p.g_sb = gate->stride[0]; p.g_st = gate->stride[1]; p.g_sh = gate->stride[2];
+    }
     if (s0) { p.s0_sn = s0->stride[0]; p.s0_sh = s0->stride[1]; }
     if (sT) { p.sT_sn = sT->stride[0]; p.sT_sh = sT->stride[1]; }
 
     Dims d{B, T, H, dk, dv, N, varlen};
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     const int* cup = varlen ? static_cast<const int*>(cu->data) : nullptr;
-    if (dt == DN_F32) return launch<float, 64, 64, 1>(p, d, dev, sms, stream, forced_s, cup);
-    if (dk == 128 && dv == 128)
-        return launch<__nv_bfloat16, 128, 128, 2>(p, d, dev, sms, stream, forced_s, cup);
-    if (dk == 128 && dv == 64)
-        return launch<__nv_bfloat16, 128, 64, 2>(p, d, dev, sms, stream, forced_s, cup);
-    if (dk == 64 && dv == 128)
-        return launch<__nv_bfloat16, 64, 128, 2>(p, d, dev, sms, stream, forced_s, cup);
-    return launch<__nv_bfloat16, 64, 64, 2>(p, d, dev, sms, stream, forced_s, cup);
+    if (gate) return dispatch<true>(p, d, dev, sms, stream, forced_s, cup, dt);
+    return dispatch<false>(p, d, dev, sms, stream, forced_s, cup, dt);
 }
 
 }  // namespace
@@ -524,15 +547,35 @@ dn_status deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* 
                        const dn_tensor* beta, const dn_tensor* initial_state,
                        const dn_tensor* cu_seqlens, int chunk_size, dn_tensor* out,
                        dn_tensor* final_state, void* stream) {
-    return fwd_impl(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
-                    stream, 0);
+    return fwd_impl(q, k, v, beta, nullptr, initial_state, cu_seqlens, chunk_size, out,
+                    final_state, stream, 0);
 }
 
 dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                           const dn_tensor* beta, const dn_tensor* initial_state,
                           const dn_tensor* cu_seqlens, int chunk_size, dn_tensor* out,
                           dn_tensor* final_state, void* stream, int seg_chunks) {
-    return fwd_impl(q, k, v, beta, initial_state, cu_seqlens, chunk_size, out, final_state,
+    return fwd_impl(q, k, v, beta, nullptr, initial_state, cu_seqlens, chunk_size, out,
+                    final_state, stream, seg_chunks);
+}
+
+dn_status gated_deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                             const dn_tensor* beta, const dn_tensor* g,
+                             const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                             int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                             void* stream) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, 0);
+}
+
+dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                const dn_tensor* beta, const dn_tensor* g,
+                                const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                                void* stream, int seg_chunks) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     stream, seg_chunks);
 }
 

@@ -14,6 +14,20 @@
 // S_0 = I, so each chunk applies I - K_r^T W_r, subsection "Compact the
 // transition product with WY").
 //
+// Gated DeltaNet (same page, section "Gated DeltaNet (GDN)", its "Complete
+// per-chunk algorithm") adds a per-token decay a_t = exp(g_t).  With
+// lambda[i:j] = a_i ... a_j inside the chunk and Gamma[l][i] = lambda[i+1:l]:
+//   L_r = (K_r K_r^T o Gamma) o M_c^-,  (I + B_r L_r) T_r = B_r,  U_r = T_r V_r
+//   W<-_r = T_r diag(lambda[1:l]) K_r,  Z_r = U_r - W<-_r S_r
+//   O_r = diag(lambda[1:l]) Q_r S_r + (Q_r K_r^T o Gamma) Z_r
+//   S_{r+1} = lambda[1:C] S_r + (diag(lambda[l+1:C]) K_r)^T Z_r
+// Decay products are exponentials of differences of the chunk's running sum of
+// g (fp32), so none of them is formed as a ratio of small numbers.  The left
+// factor of W is folded into a second copy of T (columns scaled), the right
+// factor of the state update into K (rows scaled in place once its other uses
+// are done), the readout factor into the rows of Q S, and lambda[1:C] into the
+// state registers.
+//
 // The state stays in registers (fp32) for the whole run; W, U, Z, T and the
 // masked scores never leave shared memory.  Only q, k, v, beta are read and o
 // written per chunk.  Loads of chunk r+1 are issued before chunk r is computed.
@@ -27,7 +41,7 @@ namespace dn {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES>
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false>
 struct ChainSmem {
     static constexpr int ES = sizeof(E);
     static constexpr int Q_BYTES = kChunk * DK * ES;
@@ -42,13 +56,16 @@ struct ChainSmem {
     static constexpr int OFF_K = OFF_Q + (HAS_Q ? STAGES * Q_BYTES : 0);
     static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
     static constexpr int OFF_BETA = OFF_V + (HAS_V ? STAGES * V_BYTES : 0);
-    static constexpr int OFF_SOLVE = OFF_BETA + STAGES * kChunk * 4;
+    static constexpr int OFF_GATE = OFF_BETA + STAGES * kChunk * 4;  // g per stage
+    static constexpr int OFF_DECAY = OFF_GATE + (GATED ? STAGES * kChunk * 4 : 0);
+    static constexpr int OFF_SOLVE = OFF_DECAY + (GATED ? 4 * kChunk * 4 : 0);
     static constexpr int OFF_T = align_up(OFF_SOLVE + UNION_BYTES, 128);
     static constexpr int OFF_W = OFF_T + kChunk * kChunk * ES;
     static constexpr int OFF_X = OFF_W + kChunk * DK * ES;
     static constexpr int OFF_Z = OFF_X + DK * NX * ES;
     static constexpr int OFF_P = OFF_Z + kChunk * NX * ES;
-    static constexpr int TOTAL = OFF_P + (HAS_Q ? kChunk * kChunk * ES : 0);
+    static constexpr int OFF_T2 = OFF_P + (HAS_Q ? kChunk * kChunk * ES : 0);
+    static constexpr int TOTAL = OFF_T2 + (GATED ? kChunk * kChunk * ES : 0);
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -91,12 +108,14 @@ __device__ __forceinline__ float to_e<float>(float x) {
 }
 
 // Blocked solve of (I + A) N = I for the strictly lower A (= B L, 64 x 64, fp32,
-// row stride 65), followed by T = N diag(beta) written to a swizzled tile.
+// row stride 65), followed by T = N diag(beta) written to a swizzled tile, and,
+// when colscale is given, T diag(colscale) to a second tile T2.
 // Diagonal 16 x 16 blocks by forward substitution, one column per thread;
 // off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order of i - j.
 template <typename E, int NT = kThreads>
 __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
-                                         const float* beta, E* Ts) {
+                                         const float* beta, E* Ts,
+                                         const float* colscale = nullptr, E* T2 = nullptr) {
     constexpr int LD = 65;
     const int tid = threadIdx.x;
     if (tid < 64) {
@@ -152,14 +171,15 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
         const int i = e >> 6, j = e & 63;
         const float val = j <= i ? Nf[i * LD + j] * beta[j] : 0.f;
         Ts[Swz<E>::template off<kChunk>(i, j)] = to_e<E>(val);
+        if (colscale) T2[Swz<E>::template off<kChunk>(i, j)] = to_e<E>(val * colscale[j]);
     }
 }
 
 // Runs one work item.  mode selects start state, output and destination.
-template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES>
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false>
 __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int mode,
                                             char* smem) {
-    using L = ChainSmem<E, DK, NX, HAS_V, HAS_Q, STAGES>;
+    using L = ChainSmem<E, DK, NX, HAS_V, HAS_Q, STAGES, GATED>;
     using SW = Swz<E>;
     constexpr int MT_S = DK / 64;  // 16-row tiles of the state per warp
     constexpr int NT_X = NX / 16;  // 8-column tiles per warp (NX / 2 columns)
@@ -169,6 +189,13 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     E* Ks = reinterpret_cast<E*>(smem + L::OFF_K);
     E* Vs = reinterpret_cast<E*>(smem + L::OFF_V);
     float* betas = reinterpret_cast<float*>(smem + L::OFF_BETA);
+    float* gates = reinterpret_cast<float*>(smem + L::OFF_GATE);
+    // per chunk (gated): running sum of g, lambda[1:l], lambda[l+1:C], lambda[1:C]
+    float* gsum = reinterpret_cast<float*>(smem + L::OFF_DECAY);
+    float* lam_l = gsum + kChunk;
+    float* lam_r = lam_l + kChunk;
+    float* lam_c = lam_r + kChunk;
+    E* Ts2 = reinterpret_cast<E*>(smem + L::OFF_T2);
     float* Af = reinterpret_cast<float*>(smem + L::OFF_SOLVE);
     float* Nf = Af + kChunk * L::SOLVE_LD;
     float* Xt = Nf + kChunk * L::SOLVE_LD;
@@ -228,6 +255,7 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     const E* vg = static_cast<const E*>(p.v) + it.b * p.v_sb + it.head * p.v_sh;
     E* og = static_cast<E*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
     const float* bg = p.beta + it.b * p.b_sb + it.head * p.b_sh;
+    const float* gg = GATED ? p.g + it.b * p.g_sb + it.head * p.g_sh : nullptr;
 
     const int ntok = it.tok1 - it.tok0;
     const int nchunks = (ntok + kChunk - 1) / kChunk;
@@ -242,6 +270,17 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
             const bool ok = tid < rows;
             cp_async4(smem_addr(betas + stg * kChunk + tid), ok ? bg + (t0 + tid) * p.b_st : bg,
                       ok ? 4 : 0);
+        }
+        if (GATED && warp == 0) {
+            // warp 0 loads all 64 gates (two per lane: it scans them itself after its own
+            // wait, with no barrier); rows past the run read g = 0, an identity step
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = 2 * lane + h;
+                const bool ok = i < rows;
+                cp_async4(smem_addr(gates + stg * kChunk + i), ok ? gg + (t0 + i) * p.g_st : gg,
+                          ok ? 4 : 0);
+            }
         }
         cp_async_commit();
     };
@@ -267,6 +306,32 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         const E* Vc = Vs + stg * (L::V_BYTES / L::ES);
         const float* bc = betas + stg * kChunk;
 
+        if constexpr (GATED) {
+            // running sum of g over the chunk (warp scan of lane pairs) and the decay
+            // products as exponentials of its differences; published by barrier (a)
+            if (warp == 0) {
+                const float x0 = gates[stg * kChunk + 2 * lane];
+                const float x1 = gates[stg * kChunk + 2 * lane + 1];
+                const float pair = x0 + x1;
+                float incl = pair;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const float c0 = (incl - pair) + x0;
+                const float c1 = c0 + x1;
+                const float total = __shfl_sync(0xffffffffu, c1, 31);
+                gsum[2 * lane] = c0;
+                gsum[2 * lane + 1] = c1;
+                lam_l[2 * lane] = expf(c0);
+                lam_l[2 * lane + 1] = expf(c1);
+                lam_r[2 * lane] = expf(total - c0);
+                lam_r[2 * lane + 1] = expf(total - c1);
+                if (lane == 0) lam_c[0] = expf(total);
+            }
+        }
+
         // (a) state -> operand copy
 #pragma unroll
         for (int m = 0; m < MT_S; ++m) store_frag<NT_X, NX>(Xb, s_r0 + 16 * m, x_c0, s[m], 1.f);
@@ -275,6 +340,19 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         // (b) A = B L (strict lower, fp32) and, with output, P = (Q K^T) o M_c
         {
             float acc[4][4];
+            // Gamma[row][col] = lambda[col+1:row] on and below the diagonal (gated)
+            float gam[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    gam[nt][e] = 1.f;
+                    if constexpr (GATED) {
+                        const int row = 16 * mt + g8 + 8 * (e >> 1);
+                        const int col = 32 * nh + 8 * nt + 2 * t4 + (e & 1);
+                        gam[nt][e] = col <= row ? expf(gsum[row] - gsum[col]) : 0.f;
+                    }
+                }
             zero_frag(acc);
             warp_gemm<DK, 4, DK, false, DK, false>(acc, Kc, 16 * mt, Kc, 32 * nh);
 #pragma unroll
@@ -283,7 +361,8 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
                 for (int e = 0; e < 4; ++e) {
                     const int row = 16 * mt + g8 + 8 * (e >> 1);
                     const int col = 32 * nh + 8 * nt + 2 * t4 + (e & 1);
-                    Af[row * L::SOLVE_LD + col] = col < row ? bc[row] * acc[nt][e] : 0.f;
+                    Af[row * L::SOLVE_LD + col] =
+                        col < row ? bc[row] * (acc[nt][e] * gam[nt][e]) : 0.f;
                 }
             if (HAS_Q) {
                 zero_frag(acc);
@@ -294,7 +373,7 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
                     for (int e = 0; e < 4; ++e) {
                         const int row = 16 * mt + g8 + 8 * (e >> 1);
                         const int col = 32 * nh + 8 * nt + 2 * t4 + (e & 1);
-                        if (col > row) acc[nt][e] = 0.f;
+                        acc[nt][e] = col > row ? 0.f : acc[nt][e] * gam[nt][e];
                     }
                 store_frag<4, kChunk>(Ps, 16 * mt, 32 * nh, acc, 1.f);
             }
@@ -302,7 +381,8 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         __syncthreads();
 
         // (c) T = (I + B L)^{-1} B
-        ut_solve<E>(Af, Nf, Xt, bc, Ts);
+        if constexpr (GATED) ut_solve<E>(Af, Nf, Xt, bc, Ts, lam_l, Ts2);
+        else ut_solve<E>(Af, Nf, Xt, bc, Ts);
         __syncthreads();
 
         // (d) -W = -T K (stored negated), U = T V (kept in registers as Z's start)
@@ -311,7 +391,8 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         {
             float w[NT_W][4];
             zero_frag(w);
-            warp_gemm<kChunk, NT_W, kChunk, false, DK, true>(w, Ts, 16 * mt, Kc, nh * (DK / 2));
+            warp_gemm<kChunk, NT_W, kChunk, false, DK, true>(w, GATED ? Ts2 : Ts, 16 * mt, Kc,
+                                                             nh * (DK / 2));
             store_frag<NT_W, DK>(Ws, 16 * mt, nh * (DK / 2), w, -1.f);
             if (HAS_V) warp_gemm<kChunk, NT_X, kChunk, false, NX, true>(z, Ts, 16 * mt, Vc, x_c0);
         }
@@ -323,8 +404,34 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         if constexpr (HAS_Q) {
             zero_frag(o);
             warp_gemm<DK, NT_X, DK, false, NX, true>(o, Qc, 16 * mt, Xb, x_c0);
+            if constexpr (GATED) {
+                // readout of the decayed state: row l of Q S times lambda[1:l]
+#pragma unroll
+                for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[nt][e] *= lam_l[16 * mt + g8 + 8 * (e >> 1)];
+            }
         }
         store_frag<NT_X, NX>(Zs, 16 * mt, x_c0, z, 1.f);
+        if constexpr (GATED) {
+            // K's other uses are done: scale its rows by lambda[l+1:C] for the state
+            // update, and decay the state by lambda[1:C]
+            constexpr int V = 16 / sizeof(E);
+            E* Kw = const_cast<E*>(Kc);
+            for (int idx = tid; idx < kChunk * (DK / V); idx += kThreads) {
+                const float f = lam_r[idx / (DK / V)];
+                E* c = Kw + idx * V;  // swizzling permutes chunks within a row only
+#pragma unroll
+                for (int j = 0; j < V; ++j) c[j] = to_e<E>(float(c[j]) * f);
+            }
+            const float fc = lam_c[0];
+#pragma unroll
+            for (int m = 0; m < MT_S; ++m)
+#pragma unroll
+                for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[m][nt][e] *= fc;
+        }
         __syncthreads();
 
         // (f) O += (Q K^T o M_c) Z
@@ -368,18 +475,18 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     }
 }
 
-template <typename E, int DK, int DV, int STAGES>
+template <typename E, int DK, int DV, int STAGES, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1) k_boundary(Params p) {
     extern __shared__ __align__(128) char smem[];
     const int n = count_C(p.sched);
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
         const Item it = item_C(p.sched, i);
-        run_segment<E, DK, DV, true, true, STAGES>(p, it, kModeOut, smem);
+        run_segment<E, DK, DV, true, true, STAGES, GATED>(p, it, kModeOut, smem);
         __syncthreads();
     }
 }
 
-template <typename E, int DK, int DV, int STAGES>
+template <typename E, int DK, int DV, int STAGES, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
     extern __shared__ __align__(128) char smem[];
     const int n = count_A(p.sched);
@@ -388,13 +495,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
         const Item it = item_A(p.sched, i, mode);
         if (mode == kModeHP) {
             // both maps of the segment, one after the other
-            run_segment<E, DK, DV, true, false, STAGES>(p, it, kModeH, smem);
+            run_segment<E, DK, DV, true, false, STAGES, GATED>(p, it, kModeH, smem);
             __syncthreads();
-            run_segment<E, DK, DK, false, false, STAGES>(p, it, kModeP, smem);
+            run_segment<E, DK, DK, false, false, STAGES, GATED>(p, it, kModeP, smem);
         } else if (mode == kModeP) {
-            run_segment<E, DK, DK, false, false, STAGES>(p, it, mode, smem);
+            run_segment<E, DK, DK, false, false, STAGES, GATED>(p, it, mode, smem);
         } else {
-            run_segment<E, DK, DV, true, false, STAGES>(p, it, mode, smem);
+            run_segment<E, DK, DV, true, false, STAGES, GATED>(p, it, mode, smem);
         }
         __syncthreads();
     }

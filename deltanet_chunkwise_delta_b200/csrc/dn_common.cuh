@@ -67,6 +67,7 @@ struct Params {
     const void* v;
     void* o;
     const float* beta;
+    const float* g;      // Gated DeltaNet: log decay ln a_t [B, T, H]; null for DeltaNet
     const float* s0;     // may be null
     float* sT;           // may be null
     int64_t q_sb, q_st, q_sh;
@@ -74,6 +75,7 @@ struct Params {
     int64_t v_sb, v_st, v_sh;
     int64_t o_sb, o_st, o_sh;
     int64_t b_sb, b_st, b_sh;
+    int64_t g_sb, g_st, g_sh;
     int64_t s0_sn, s0_sh;
     int64_t sT_sn, sT_sh;
     float* wsP;          // [slots][d_k][d_k]

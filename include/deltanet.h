@@ -104,6 +104,44 @@ dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tenso
                           int seg_chunks);
 
 /*
+ * gated_deltanet_fwd -- Gated DeltaNet forward pass ("Linear Attention,
+ * Visualized", section "Gated DeltaNet (GDN)"): the same recurrence with a
+ * per-token scalar decay a_t on the whole transition,
+ *
+ *     S_t = a_t (I - beta_t k_t^T k_t) S_{t-1} + beta_t k_t^T v_t,   o_t = q_t S_t,
+ *
+ * i.e. S <- a_t S first, then the DeltaNet prediction, correction and write
+ * from the decayed state.  It is evaluated with that section's "Complete
+ * per-chunk algorithm" (decay products lambda[i:j] inside a chunk, the mask
+ * Gamma[l][i] = lambda[i+1:l], left-decayed q, k and right-decayed k) and the
+ * same split of each chain across SMs (a chunk is still an affine map of the
+ * state, S' = (lambda[1:C] I - K->^T W<-) S + K->^T U).
+ *
+ *   g             [B, T, H] fp32, the decay as its natural log: g_t = ln a_t
+ *                 (finite; the pages use 0 < a_t <= 1, i.e. g_t <= 0).  Decay
+ *                 products are formed as exp of differences of the chunk's
+ *                 running fp32 sum of g, so their relative error grows with
+ *                 |sum of g over a chunk| times 2^-24.
+ *   other arguments, layouts, ownership, aliasing (g is an input) and errors
+ *   as deltanet_fwd; g == NULL returns DN_ERR_INVALID_ARG.
+ *
+ * All supported shapes run on the mma.sync chain kernels (the tcgen05 kernels
+ * serve deltanet_fwd only).
+ */
+dn_status gated_deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                             const dn_tensor* beta, const dn_tensor* g,
+                             const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                             int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                             void* stream);
+
+/* gated_deltanet_fwd with the seg_chunks override of deltanet_fwd_ex. */
+dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                const dn_tensor* beta, const dn_tensor* g,
+                                const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                                void* stream, int seg_chunks);
+
+/*
  * deltanet_fwd_noalloc -- the forward pass without any device allocation.
  * (No counterpart on the pages: this is a deployment variant of deltanet_fwd.)
  *
@@ -158,7 +196,7 @@ int deltanet_last_launches(void);
 
 /*
  * deltanet_set_kernel_events -- profiling hook.  While set (non-NULL), every
- * deltanet_fwd / deltanet_fwd_ex call on this thread records start_event on
+ * deltanet_fwd / gated_deltanet_fwd (and _ex) call on this thread records start_event on
  * its stream right before launching the boundary-pass kernel (the output
  * kernel, which dominates the call) and stop_event right after it, so that
  * cudaEventElapsedTime gives that kernel's device time.  The caller owns the

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "deltanet.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(deltanet_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:gated_)?deltanet_\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -131,3 +131,31 @@ def test_rejects_bad_varlen_descriptors(lib):
     assert call(lib, q1, k1, v1, b1, cu=cu_f, out=o1) == L.DN_ERR_INVALID_ARG
     s_wrong_n = desc([1, 3, 128, 64], L.DN_F32, 0x500000000)   # N = 2 from cu
     assert call(lib, q1, k1, v1, b1, s0=s_wrong_n, cu=cu, out=o1) == L.DN_ERR_INVALID_ARG
+
+
+def call_gated(lib, q, k, v, beta, g, s0=None, cu=None, chunk=64, out=None, sT=None):
+    r = lambda x: None if x is None else ctypes.byref(x)
+    return lib.gated_deltanet_fwd(r(q), r(k), r(v), r(beta), r(g), r(s0), r(cu), chunk, r(out),
+                                  r(sT), None)
+
+
+def test_gated_rejects_bad_gate(lib):
+    """The log-decay tensor follows beta's rules: [B, T, H] fp32, 4-byte aligned,
+    non-negative strides, required, and no output may overlap it."""
+    q, k, v, beta, s0, out, sT = good()
+    g = desc([2, 100, 3], L.DN_F32, 0x100000000 + 7 * 2**28)
+    assert call_gated(lib, q, k, v, beta, None, out=out) == L.DN_ERR_INVALID_ARG
+    g_shape = desc([2, 100, 4], L.DN_F32, g.data)
+    assert call_gated(lib, q, k, v, beta, g_shape, out=out) == L.DN_ERR_INVALID_ARG
+    g_type = desc([2, 100, 3], L.DN_BF16, g.data)
+    assert call_gated(lib, q, k, v, beta, g_type, out=out) == L.DN_ERR_INVALID_ARG
+    g_align = desc([2, 100, 3], L.DN_F32, g.data + 2)
+    assert call_gated(lib, q, k, v, beta, g_align, out=out) == L.DN_ERR_INVALID_ARG
+    g_neg = desc([2, 100, 3], L.DN_F32, g.data, strides=[300, -3, 1])
+    assert call_gated(lib, q, k, v, beta, g_neg, out=out) == L.DN_ERR_INVALID_ARG
+    o_on_g = desc([2, 100, 3, 64], L.DN_BF16, g.data)
+    assert call_gated(lib, q, k, v, beta, g, out=o_on_g) == L.DN_ERR_ALIAS
+    assert call_gated(lib, q, k, v, beta, g, out=out, chunk=32) == L.DN_ERR_UNSUPPORTED
+    r = lambda x: ctypes.byref(x)
+    assert lib.gated_deltanet_fwd_ex(r(q), r(k), r(v), r(beta), None, None, None, 64, r(out),
+                                     None, None, 2) == L.DN_ERR_INVALID_ARG
