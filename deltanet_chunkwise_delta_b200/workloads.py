@@ -23,6 +23,10 @@ Recipe (all on the CPU, so every consumer sees bit-identical inputs):
     "Gated DeltaNet (GDN)") then draw the log decay g = ln a = logsigmoid(z + 4),
     z ~ N(0,1) in fp32, shape [B, T, H]: a has median 0.982 and 5 % below 0.91,
     so a state keeps about a third of itself across one 64-token chunk;
+  * Gated Delta Product workloads (same page, section "Gated Delta Product
+    (GDP)") draw n_h key, value and beta rows per token (substep-major, i.e.
+    k [B, T n_h, H, d]) where the others draw one; q, the initial state and g
+    keep one row per token;
   * variable-length batches draw 32 lengths with ``numpy.random.default_rng(seed)``
     log-uniformly in [ln 128, ln 32768], L = floor(exp(u)), packed in draw order.
 """
@@ -51,6 +55,7 @@ class Workload:
     seqlens: Optional[tuple] = None   # varlen: per-sequence lengths (B == 1)
     chunk: int = 64
     gated: bool = False               # Gated DeltaNet: draw the log decay g
+    nh: int = 1                       # Gated Delta Product: writes per token (gated)
 
     @property
     def n_seq(self) -> int:
@@ -84,6 +89,8 @@ def _workloads() -> dict:
         "varlen_32": Workload("varlen_32", 1, sum(vl), 16, 128, 128, torch.bfloat16, True, vl),
         "gdn_1p3b": Workload("gdn_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False, gated=True),
         "gdn_65k": Workload("gdn_65k", 1, 65536, 16, 128, 128, torch.bfloat16, True, gated=True),
+        "gdp_1p3b": Workload("gdp_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False,
+                             gated=True, nh=2),
     }
 
 
@@ -91,11 +98,13 @@ WORKLOADS = _workloads()
 
 
 def custom(B, T, H, dk, dv, dtype=torch.bfloat16, init_state=False, seqlens=None,
-           name="custom", gated=False) -> Workload:
+           name="custom", gated=False, nh=1) -> Workload:
     if seqlens is not None:
         seqlens = tuple(int(x) for x in seqlens)
         B, T = 1, sum(seqlens)
-    return Workload(name, B, T, H, dk, dv, dtype, init_state, seqlens, gated=gated)
+    if nh > 1 and not gated:
+        raise ValueError("several writes per token is the gated product")
+    return Workload(name, B, T, H, dk, dv, dtype, init_state, seqlens, gated=gated, nh=nh)
 
 
 def _draw_tokens(gen, B, T, H, d, dtype, normalise):
@@ -118,10 +127,11 @@ def generate(w: Workload, seed: int = 0, beta_mode: str = "sigmoid") -> dict:
     """
     gen = torch.Generator("cpu")
     gen.manual_seed(seed)
+    Tw = w.T * w.nh                   # rows of k, v, beta
     q = _draw_tokens(gen, w.B, w.T, w.H, w.dk, w.dtype, True)
-    k = _draw_tokens(gen, w.B, w.T, w.H, w.dk, w.dtype, True)
-    v = _draw_tokens(gen, w.B, w.T, w.H, w.dv, w.dtype, False)
-    beta = torch.sigmoid(torch.randn((w.B, w.T, w.H), generator=gen, dtype=torch.float32))
+    k = _draw_tokens(gen, w.B, Tw, w.H, w.dk, w.dtype, True)
+    v = _draw_tokens(gen, w.B, Tw, w.H, w.dv, w.dtype, False)
+    beta = torch.sigmoid(torch.randn((w.B, Tw, w.H), generator=gen, dtype=torch.float32))
     if beta_mode == "zero":
         beta = torch.zeros_like(beta)
     elif beta_mode == "one":

@@ -10,7 +10,8 @@ Two independent float64 statements of the method:
 * ``token_recurrence`` -- the plain definition, a C float64 token-serial loop
   ("Linear Attention, Visualized", DeltaNet, "Recurrent form"), threaded over
   (sequence, head); with a gate ``g`` = ln a_t it runs the Gated DeltaNet
-  recurrence of the same page (section "Gated DeltaNet (GDN)").  Built from
+  recurrence of the same page (section "Gated DeltaNet (GDN)"), and with
+  ``n_sub`` > 1 the Gated Delta Product (section "Gated Delta Product (GDP)").  Built from
   ``deltanet_oracle.c`` with gcc.
 * ``chunkwise`` (module) -- numpy float64 statements of the chunk form, the
   WY transition product, the segment composition and the full-sequence closed
@@ -52,13 +53,13 @@ def _load():
     with _lock:
         if _lib is None:
             lib = ctypes.CDLL(build())
-            f = lib.gdn_oracle_fwd
+            f = lib.gdp_oracle_fwd
             f.restype = ctypes.c_int
             f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                           ctypes.c_int64,
                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-                          ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                          ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
             _lib = lib
     return _lib
@@ -70,12 +71,15 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
                      heads=None, out_dtype=torch.float64, want_out=True,
-                     n_threads: Optional[int] = None, g=None):
+                     n_threads: Optional[int] = None, g=None, n_sub: int = 1):
     """Run the float64 token recurrence on CPU tensors.
 
     q, k: [B, T, H, dk]; v: [B, T, H, dv] (fp32, bf16 or fp64); beta: [B, T, H]
     fp32; initial_state: [N, H, dk, dv] or None; cu_seqlens: int32 [N+1] or None;
     g: [B, T, H] fp32 log decay (Gated DeltaNet) or None (plain DeltaNet).
+    n_sub > 1: Gated Delta Product with n_sub writes per token; k, v, beta then
+    hold [B, T * n_sub, H, .] rows (substep-major within a token) while q, g, out
+    and cu_seqlens count tokens.
     ``heads``: (h_begin, h_end) to compute a subset of heads (others are NaN).
     Returns (out [B, T, H, dv] in ``out_dtype`` or None, final_state [N, H, dk, dv]
     float64).
@@ -85,6 +89,9 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
     beta = beta.to(torch.float32).contiguous()
     gate = None if g is None else g.to(torch.float32).contiguous()
     B, T, H, dk = q.shape
+    if n_sub < 1 or tuple(k.shape) != (B, T * n_sub, H, dk) or v.shape[:3] != (B, T * n_sub, H) \
+            or tuple(beta.shape) != (B, T * n_sub, H):
+        raise ValueError("k, v, beta must hold n_sub rows per token of q")
     dv = v.shape[-1]
     codes = {torch.float32: 0, torch.bfloat16: 1, torch.float64: 2}
     if not (q.dtype == k.dtype == v.dtype) or q.dtype not in codes:
@@ -104,10 +111,10 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
     fs = torch.full((n_seq, H, dk, dv), float("nan"), dtype=torch.float64)
     if n_threads is None:
         n_threads = os.cpu_count() or 1
-    if gate is not None and tuple(gate.shape) != tuple(beta.shape):
-        raise ValueError("g must have the shape of beta")
-    rc = lib.gdn_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta), _ptr(gate),
-                            _ptr(s0), _ptr(cu), n_seq, B, T, H, dk, dv, h0, h1,
+    if gate is not None and tuple(gate.shape) != (B, T, H):
+        raise ValueError("g must have one value per (token, head)")
+    rc = lib.gdp_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta), _ptr(gate),
+                            _ptr(s0), _ptr(cu), n_seq, B, T, H, dk, dv, int(n_sub), h0, h1,
                             _ptr(out), 0 if out_dtype == torch.float32 else 2,
                             _ptr(fs), int(n_threads))
     if rc != 0:

@@ -275,3 +275,43 @@ def decayed_linear_attention(Q, K, V, a):
         for s in range(t + 1):
             D[t, s] = lam(s + 2, t + 1)
     return ((Q @ K.T) * D) @ V
+
+
+# --- Gated Delta Product ("Linear Attention, Visualized", section "Gated Delta Product (GDP)") ---
+
+def gdp_virtual_sequence(Q, K, V, beta, a, n_h: int):
+    """The page's "GDP as GDN over a virtual sequence": token t's n_h substeps
+    become virtual steps m = n_h (t - 1) + j; k, v, beta move over unchanged,
+    the decay sits on the first substep (1 elsewhere) and the query on the last
+    (0 elsewhere).  K, V, beta hold n_h rows per token (substep-major), Q and a
+    one per token.  Returns (Qv, Kv, Vv, beta_v, a_v)."""
+    n = Q.shape[0]
+    Qv = np.zeros((n * n_h, Q.shape[1]))
+    Qv[n_h - 1::n_h] = Q
+    av = np.ones(n * n_h)
+    av[0::n_h] = a
+    return Qv, K, V, beta, av
+
+
+def gdp_chunkwise(Q, K, V, beta, a, n_h: int, S0=None, C: int = 64):
+    """GDP evaluated as the GDN chunk algorithm over the virtual sequence,
+    keeping every n_h-th output.  Returns (O [n, d_v], S_final)."""
+    Qv, Kv, Vv, bv, av = gdp_virtual_sequence(Q, K, V, beta, a, n_h)
+    Ov, S = gated_chunkwise(Qv, Kv, Vv, bv, av, S0, C)
+    return Ov[n_h - 1::n_h], S
+
+
+def gdp_substeps(Q, K, V, beta, a, n_h: int, S0):
+    """GDP's token update as the page writes it, with explicit d_k x d_k
+    matrices: S_{t,0} = a_t S_{t-1}, S_{t,j} = A_{t,j} S_{t,j-1} + X_{t,j}
+    (A = I - beta k^T k, X = beta k^T v), o_t = q_t S_{t,n_h}."""
+    S = S0.copy()
+    O = np.zeros((Q.shape[0], V.shape[1]))
+    for t in range(Q.shape[0]):
+        S = a[t] * S
+        for j in range(n_h):
+            m = t * n_h + j
+            A = np.eye(K.shape[1]) - beta[m] * np.outer(K[m], K[m])
+            S = A @ S + beta[m] * np.outer(K[m], V[m])
+        O[t] = Q[t] @ S
+    return O, S

@@ -22,12 +22,22 @@
  * so with a gate the loop first decays the state, S <- a_t S_{t-1}, and then
  * makes the same prediction, correction and write from the decayed state.
  * The gate arrives as g_t = ln a_t (fp32 [B, T, H]); a_t = exp(g_t) in float64.
+ *
+ * Gated Delta Product (same page, section "Gated Delta Product (GDP)") makes
+ * n_sub delta-rule writes per token, each with its own key, value and beta,
+ * after one decay of the state and before the token's readout:
+ *     S_{t,0} = a_t S_{t-1};  S_{t,j} = (I - b_{t,j} k_{t,j}^T k_{t,j}) S_{t,j-1}
+ *     + b_{t,j} k_{t,j}^T v_{t,j} for j = 1..n_sub;  S_t = S_{t,n_sub};  o_t = q_t S_t.
+ * k, v and beta then hold n_sub rows per token, substep-major within the token
+ * (row t * n_sub + j - 1, i.e. [B, T * n_sub, H, .]); q, gate and out keep one
+ * row per token.  n_sub = 1 is (Gated) DeltaNet.
  * S starts from the caller's initial state (or zero) at the first token of each
  * sequence.  No query scaling is applied.  Inputs stored as bf16 are widened
  * exactly to float64; every sum is accumulated in float64.
  *
  * Layouts (contiguous, row-major):
- *   q, k   [B, T, H, dk]     v, out [B, T, H, dv]     beta, gate [B, T, H] (fp32)
+ *   q [B, T, H, dk]  out [B, T, H, dv]  gate [B, T, H] (fp32)
+ *   k [B, T n_sub, H, dk]  v [B, T n_sub, H, dv]  beta [B, T n_sub, H] (fp32)
  *   init_state, final_state [N, H, dk, dv]
  * With cu_seqlens (host int32 [N+1]) B must be 1 and sequence n covers tokens
  * cu[n] .. cu[n+1]-1; without it N = B and sequence n is batch row n.
@@ -61,6 +71,7 @@ typedef struct {
     const double* init_state;   /* float64 copy or NULL */
     const int32_t* cu;
     int64_t n_seq, B, T, H, dk, dv, h_begin, h_end;
+    int64_t n_sub;              /* delta-rule writes per token (1 for DeltaNet / GDN) */
     void* out;
     int out_dtype;
     double* final_state;        /* may be NULL */
@@ -70,9 +81,9 @@ typedef struct {
 } oracle_ctx;
 
 static void run_job(oracle_ctx* c, int64_t job, double* S, double* kt, double* qt, double* u) {
-    const int64_t nh = c->h_end - c->h_begin;
-    const int64_t n = job / nh;
-    const int64_t h = c->h_begin + job % nh;
+    const int64_t n_heads = c->h_end - c->h_begin;
+    const int64_t n = job / n_heads;
+    const int64_t h = c->h_begin + job % n_heads;
     const int64_t dk = c->dk, dv = c->dv, H = c->H;
     int64_t row0, len;
     if (c->cu) {
@@ -88,34 +99,37 @@ static void run_job(oracle_ctx* c, int64_t job, double* S, double* kt, double* q
 
     for (int64_t t = 0; t < len; ++t) {
         const int64_t tok = row0 + t;                 /* flattened (b, t) row */
-        const int64_t qk_off = (tok * H + h) * dk;
-        const int64_t v_off = (tok * H + h) * dv;
-        const double b = (double)c->beta[tok * H + h];
+        const int64_t q_off = (tok * H + h) * dk;
+        const int64_t o_off = (tok * H + h) * dv;
         if (c->gate) {
             /* decay first: the prediction below reads a_t S_{t-1} */
             const double a = exp((double)c->gate[tok * H + h]);
             for (int64_t e = 0; e < dk * dv; ++e) S[e] *= a;
         }
-        for (int64_t a = 0; a < dk; ++a) {
-            kt[a] = load_elt(c->k, c->in_dtype, qk_off + a);
-            qt[a] = load_elt(c->q, c->in_dtype, qk_off + a);
+        for (int64_t sub = 0; sub < c->n_sub; ++sub) {
+            const int64_t row = tok * c->n_sub + sub;  /* this write's k, v, beta row */
+            const int64_t k_off = (row * H + h) * dk;
+            const int64_t v_off = (row * H + h) * dv;
+            const double b = (double)c->beta[row * H + h];
+            for (int64_t a = 0; a < dk; ++a) kt[a] = load_elt(c->k, c->in_dtype, k_off + a);
+            /* vhat = k S ; u = beta (v - vhat) */
+            for (int64_t j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int64_t a = 0; a < dk; ++a) acc += kt[a] * S[a * dv + j];
+                u[j] = b * (load_elt(c->v, c->in_dtype, v_off + j) - acc);
+            }
+            /* S += k^T u */
+            for (int64_t a = 0; a < dk; ++a)
+                for (int64_t j = 0; j < dv; ++j) S[a * dv + j] += kt[a] * u[j];
         }
-        /* vhat = k S ; u = beta (v - vhat) */
-        for (int64_t j = 0; j < dv; ++j) {
-            double acc = 0.0;
-            for (int64_t a = 0; a < dk; ++a) acc += kt[a] * S[a * dv + j];
-            u[j] = b * (load_elt(c->v, c->in_dtype, v_off + j) - acc);
-        }
-        /* S += k^T u */
-        for (int64_t a = 0; a < dk; ++a)
-            for (int64_t j = 0; j < dv; ++j) S[a * dv + j] += kt[a] * u[j];
-        /* o = q S (after the write) */
+        /* o = q S (after the writes) */
         if (c->out) {
+            for (int64_t a = 0; a < dk; ++a) qt[a] = load_elt(c->q, c->in_dtype, q_off + a);
             for (int64_t j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int64_t a = 0; a < dk; ++a) acc += qt[a] * S[a * dv + j];
-                if (c->out_dtype == OR_F64) ((double*)c->out)[v_off + j] = acc;
-                else ((float*)c->out)[v_off + j] = (float)acc;
+                if (c->out_dtype == OR_F64) ((double*)c->out)[o_off + j] = acc;
+                else ((float*)c->out)[o_off + j] = (float)acc;
             }
         }
     }
@@ -140,14 +154,16 @@ static void* worker(void* arg) {
 }
 
 /* Returns 0 on success, -1 on a bad argument, -2 on allocation failure.
- * gate may be NULL (plain DeltaNet). */
-int gdn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+ * gate may be NULL (no decay); n_sub >= 1 writes per token (T counts tokens,
+ * cu_seqlens token offsets). */
+int gdp_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
                    const float* beta, const float* gate, const double* init_state,
                    const int32_t* cu_seqlens, int64_t n_seq,
-                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t n_sub,
                    int64_t h_begin, int64_t h_end,
                    void* out, int out_dtype, double* final_state, int n_threads) {
     if ((B * T > 0) && (!q || !k || !v || !beta)) return -1;
+    if (n_sub < 1) return -1;
     if (in_dtype != OR_F32 && in_dtype != OR_BF16 && in_dtype != OR_F64) return -1;
     if (out_dtype != OR_F32 && out_dtype != OR_F64) return -1;
     if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
@@ -164,7 +180,7 @@ int gdn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     c.q = q; c.k = k; c.v = v; c.in_dtype = in_dtype; c.beta = beta; c.gate = gate;
     c.init_state = init_state; c.cu = cu_seqlens; c.n_seq = n_seq;
     c.B = B; c.T = T; c.H = H; c.dk = dk; c.dv = dv;
-    c.h_begin = h_begin; c.h_end = h_end;
+    c.h_begin = h_begin; c.h_end = h_end; c.n_sub = n_sub;
     c.out = out; c.out_dtype = out_dtype; c.final_state = final_state;
     c.n_jobs = n_seq * (h_end - h_begin);
     c.next_job = 0;
@@ -183,6 +199,17 @@ int gdn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     free(th);
     pthread_mutex_destroy(&c.lock);
     return 0;
+}
+
+/* Gated DeltaNet: one write per token (gate may be NULL: plain DeltaNet). */
+int gdn_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+                   const float* beta, const float* gate, const double* init_state,
+                   const int32_t* cu_seqlens, int64_t n_seq,
+                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                   int64_t h_begin, int64_t h_end,
+                   void* out, int out_dtype, double* final_state, int n_threads) {
+    return gdp_oracle_fwd(q, k, v, in_dtype, beta, gate, init_state, cu_seqlens, n_seq, B, T, H,
+                          dk, dv, 1, h_begin, h_end, out, out_dtype, final_state, n_threads);
 }
 
 /* Plain DeltaNet: the gated loop with every a_t = 1 (no decay step at all). */

@@ -48,3 +48,13 @@ def test_gate_recipe():
     med = float(a["g"].exp().median())
     assert 0.97 < med < 0.99
     assert wl.WORKLOADS["gdn_65k"].gated and not wl.WORKLOADS["long_65k"].gated
+
+
+def test_gdp_recipe():
+    """Gated Delta Product workloads draw n_h key/value/beta rows per token."""
+    w = wl.custom(2, 100, 3, 64, 32, torch.bfloat16, gated=True, nh=3)
+    x = wl.generate(w, seed=6)
+    assert x["q"].shape == (2, 100, 3, 64) and x["k"].shape == (2, 300, 3, 64)
+    assert x["v"].shape == (2, 300, 3, 32) and x["beta"].shape == (2, 300, 3)
+    assert x["g"].shape == (2, 100, 3)
+    assert wl.WORKLOADS["gdp_1p3b"].nh == 2
