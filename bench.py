@@ -3,7 +3,8 @@
 
 One step = one deltanet_fwd call over the whole workload (every step of the
 path: WY/UT factors, segment summaries, segment scan, boundary pass with
-output); for the Gated DeltaNet workloads (gdn_*) one gated_deltanet_fwd call.  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
+output); for the Gated DeltaNet workloads (gdn_*) one gated_deltanet_fwd call, for
+the Gated Delta Product workloads (gdp_*) one gated_deltaproduct_fwd call.  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
 d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 beta, zero initial state, fp32
 final state), synthetic seeded inputs.  Inputs (q, k, v: 201 MB) exceed the
 126 MB L2, so no flush is needed between steps.
@@ -54,7 +55,8 @@ def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
     DeltaNet), initial state read if given, final state written."""
     es = 2 if w.dtype == torch.bfloat16 else 4
     th = w.tokens * w.H
-    b = th * (es * (2 * w.dk + 2 * w.dv) + 4 + (4 if w.gated else 0))
+    # Gated Delta Product: k, v and beta have nh rows per token
+    b = th * (es * ((1 + w.nh) * w.dk + (w.nh + 1) * w.dv) + 4 * w.nh + (4 if w.gated else 0))
     st = w.n_seq * w.H * w.dk * w.dv * 4
     if w.init_state:
         b += st
@@ -201,9 +203,10 @@ def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0):
     sl = lambda t: t[b:b + 1, :tokens].contiguous()
     s0 = None if x["initial_state"] is None else x["initial_state"][b:b + 1].contiguous()
     gate = None if x.get("g") is None else sl(x["g"])
+    slw = lambda t: t[b:b + 1, :tokens * w.nh].contiguous()   # nh rows per token
     t0 = time.perf_counter()
-    oracle.token_recurrence(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["beta"]), s0,
-                            n_threads=n_threads, g=gate)
+    oracle.token_recurrence(sl(x["q"]), slw(x["k"]), slw(x["v"]), slw(x["beta"]), s0,
+                            n_threads=n_threads, g=gate, n_sub=w.nh)
     return time.perf_counter() - t0, min(n_threads, w.H)
 
 
@@ -257,7 +260,11 @@ def run_b200(args, w: wl.Workload):
     stream = torch.cuda.current_stream(device)
 
     def call(d, o, f):
-        if w.gated:
+        if w.nh > 1:
+            dn.gated_deltaproduct_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], w.nh,
+                                      d["initial_state"], d["cu_seqlens"], out=o, final_state=f,
+                                      stream=stream)
+        elif w.gated:
             dn.gated_deltanet_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["initial_state"],
                                   d["cu_seqlens"], out=o, final_state=f, stream=stream)
         else:
@@ -302,7 +309,9 @@ def run_b200(args, w: wl.Workload):
     tokens = w.tokens
     value = ws * tokens / (ms / 1e3)
     th = w.tokens * w.H
-    tflops = ws * th * flops_per_token_head(w.dk, w.dv) / (ms / 1e3) / 1e12
+    # the algorithmic FLOPs of the chunk algorithm per write (nh writes per token)
+    fpt = w.nh * flops_per_token_head(w.dk, w.dv)
+    tflops = ws * th * fpt / (ms / 1e3) / 1e12
     hbm_peak, tc_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(w)
     tc_path = not w.gated and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
@@ -325,12 +334,11 @@ def run_b200(args, w: wl.Workload):
                 "kernel": "k_tc_chain (boundary pass)" if tc_kernel else "k_boundary",
                 "kernel_ms": kernel_ms, "algorithmic_bytes_per_launch": kernel_bytes}
     # the whole path against its roofline: slower of FLOPs at the bf16 peak and bytes at HBM
-    t_roof = max(th * flops_per_token_head(w.dk, w.dv) / (tc_peak * 1e12),
-                 alg_bytes / (hbm_peak * 1e9))
-    roofline_step = {"bound": "hbm" if alg_bytes / hbm_peak > th * flops_per_token_head(w.dk, w.dv) / tc_peak / 1e3 else "tensor",
+    t_roof = max(th * fpt / (tc_peak * 1e12), alg_bytes / (hbm_peak * 1e9))
+    roofline_step = {"bound": "hbm" if alg_bytes / hbm_peak > th * fpt / tc_peak / 1e3 else "tensor",
                      "roofline_ms": t_roof * 1e3, "step_ms": ms_local,
                      "frac": t_roof * 1e3 / ms_local, "algorithmic_bytes": alg_bytes,
-                     "algorithmic_flops": th * flops_per_token_head(w.dk, w.dv),
+                     "algorithmic_flops": th * fpt,
                      "peaks": {"hbm_gbs": hbm_peak, "bf16_tflops": tc_peak, "kind": peak_kind}}
 
     # end to end through the public call with host buffers.  Every step copies its
@@ -421,7 +429,8 @@ def run_b200(args, w: wl.Workload):
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
                    "chunk": CHUNK, "segments_per_chain": G, "chunks_per_segment": s,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}",
-                   "variant": "gated DeltaNet" if w.gated else "DeltaNet"},
+                   "variant": (f"gated delta product, n_h = {w.nh}" if w.nh > 1 else
+                               "gated DeltaNet" if w.gated else "DeltaNet")},
         "tflops": tflops,
         "tflops_unit": "algorithmic TFLOP/s (6Cd^2 + 5C^2d + C^3/3 per chunk-head)",
         "roofline": roofline,

@@ -22,7 +22,7 @@ DN_OK, DN_ERR_INVALID_ARG, DN_ERR_UNSUPPORTED, DN_ERR_ALIAS, DN_ERR_CUDA, \
 DN_F32, DN_BF16, DN_I32 = 0, 1, 2
 
 EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "gated_deltanet_fwd", "gated_deltanet_fwd_ex",
-            "deltanet_status_string",
+            "gated_deltaproduct_fwd", "gated_deltaproduct_fwd_ex", "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
             "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events")
 
@@ -70,6 +70,13 @@ def load(path: Optional[str] = None):
         lib.gated_deltanet_fwd_ex.restype = ctypes.c_int
         lib.gated_deltanet_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P,
                                               ctypes.c_void_p, ctypes.c_int]
+        lib.gated_deltaproduct_fwd.restype = ctypes.c_int
+        lib.gated_deltaproduct_fwd.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                               P, P, ctypes.c_void_p]
+        lib.gated_deltaproduct_fwd_ex.restype = ctypes.c_int
+        lib.gated_deltaproduct_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int,
+                                                  ctypes.c_int, P, P, ctypes.c_void_p,
+                                                  ctypes.c_int]
         lib.deltanet_fwd_noalloc.restype = ctypes.c_int
         lib.deltanet_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
         lib.deltanet_status_string.restype = ctypes.c_char_p
@@ -198,6 +205,42 @@ def gated_deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: 
         final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     st = call_gated(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     _stream_handle(q.device, stream), seg_chunks)
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state
+
+
+def gated_deltaproduct_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           beta: torch.Tensor, g: torch.Tensor, n_h: int,
+                           initial_state: Optional[torch.Tensor] = None,
+                           cu_seqlens: Optional[torch.Tensor] = None, chunk_size: int = 64,
+                           out: Optional[torch.Tensor] = None,
+                           final_state: Optional[torch.Tensor] = None,
+                           output_final_state: bool = True, stream=None, seg_chunks: int = 0):
+    """Gated Delta Product forward on CUDA tensors through the C ABI.
+
+    q [B, T, H, d_k]; k [B, T * n_h, H, d_k], v [B, T * n_h, H, d_v] and beta
+    [B, T * n_h, H] with the n_h writes of each token on consecutive rows; g
+    [B, T, H] (ln a, one per token); cu_seqlens counts tokens.  Returns
+    (out [B, T, H, d_v], final_state or None).
+    """
+    if not q.is_cuda:
+        raise ValueError("gated_deltaproduct_fwd runs on CUDA tensors only")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    ds = [describe(t) for t in (q, k, v, beta, g, initial_state, cu_seqlens, out, final_state)]
+    args = [_ref(x) for x in ds[:7]] + [int(n_h), int(chunk_size)] + [_ref(x) for x in ds[7:]]
+    lib = load()
+    stream_h = _stream_handle(q.device, stream)
+    if seg_chunks:
+        st = lib.gated_deltaproduct_fwd_ex(*args, stream_h, int(seg_chunks))
+    else:
+        st = lib.gated_deltaproduct_fwd(*args, stream_h)
     if st != DN_OK:
         raise DeltaNetError(st, status_string(st))
     return out, final_state

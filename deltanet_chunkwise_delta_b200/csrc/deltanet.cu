@@ -366,7 +366,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         sc.cu = cu;
         sc.N = (int)d.N;
         k_schedule<<<1, 1024, 0, stream>>>(
-            cu, (int)d.N, (int)d.T, (int)d.H, forced_s, forced_s > 0 ? kMaxSlots : kAutoMaxSlots,
+            cu, p.nh > 1 ? p.nh : 1, (int)d.N, (int)d.T, (int)d.H, forced_s, forced_s > 0 ? kMaxSlots : kAutoMaxSlots,
             sms, model, reinterpret_cast<Item*>(base + off_items),
             reinterpret_cast<Item*>(base + off_A), reinterpret_cast<Item*>(base + off_S),
             reinterpret_cast<int*>(base), reinterpret_cast<int*>(base + off_nc),
@@ -448,18 +448,23 @@ dn_status dispatch(Params& p, const Dims& d, int dev, int sms, cudaStream_t stre
 }
 
 // gate: Gated DeltaNet's log decay [B, T, H] fp32, or null for DeltaNet.
+// nh: delta-rule writes per token (Gated Delta Product; 1 otherwise): k, v and beta hold
+// T * nh rows, q, gate and out T rows, cu_seqlens counts tokens.
 dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                    const dn_tensor* beta, const dn_tensor* gate, const dn_tensor* s0,
                    const dn_tensor* cu, int chunk, dn_tensor* out, dn_tensor* sT,
-                   void* stream_ptr, int forced_s) {
+                   void* stream_ptr, int forced_s, int nh = 1) {
     if (!q || !k || !v || !beta || !out) return DN_ERR_INVALID_ARG;
     if (q->ndim != 4 || k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return DN_ERR_INVALID_ARG;
-    if (forced_s < 0) return DN_ERR_INVALID_ARG;
+    if (forced_s < 0 || nh < 1 || (nh > 1 && !gate)) return DN_ERR_INVALID_ARG;
     const int64_t B = q->shape[0], T = q->shape[1], H = q->shape[2], dk = q->shape[3];
     const int64_t dv = v->shape[3];
     if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1) return DN_ERR_INVALID_ARG;
-    const int64_t kd[4] = {B, T, H, dk}, vd[4] = {B, T, H, dv}, bd[3] = {B, T, H};
-    if (!shape_eq(k, 4, kd) || !shape_eq(v, 4, vd) || !shape_eq(out, 4, vd) ||
+    if (nh > 1024 || T * nh >= (int64_t(1) << 31)) return DN_ERR_INVALID_ARG;
+    const int64_t Tw = T * nh;  // rows of k, v, beta
+    const int64_t kd[4] = {B, Tw, H, dk}, vd[4] = {B, Tw, H, dv}, bd[3] = {B, Tw, H};
+    const int64_t od[4] = {B, T, H, dv}, gd[3] = {B, T, H};
+    if (!shape_eq(k, 4, kd) || !shape_eq(v, 4, vd) || !shape_eq(out, 4, od) ||
         !shape_eq(beta, 3, bd))
         return DN_ERR_INVALID_ARG;
     const int32_t dt = q->dtype;
@@ -473,13 +478,13 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     if (numel(beta) > 0 && (!beta->data || (reinterpret_cast<uintptr_t>(beta->data) & 3)))
         return DN_ERR_INVALID_ARG;
     if (gate) {
-        if (!shape_eq(gate, 3, bd) || gate->dtype != DN_F32) return DN_ERR_INVALID_ARG;
+        if (!shape_eq(gate, 3, gd) || gate->dtype != DN_F32) return DN_ERR_INVALID_ARG;
         for (int i = 0; i < 3; ++i)
             if (gate->stride[i] < 0) return DN_ERR_INVALID_ARG;
         if (numel(gate) > 0 && (!gate->data || (reinterpret_cast<uintptr_t>(gate->data) & 3)))
             return DN_ERR_INVALID_ARG;
     }
-    if (B * T >= (int64_t(1) << 31) || H >= 65536) return DN_ERR_INVALID_ARG;
+    if (B * Tw >= (int64_t(1) << 31) || H >= 65536) return DN_ERR_INVALID_ARG;
 
     int64_t N = B;
     const bool varlen = cu != nullptr;
@@ -532,7 +537,8 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     if (s0) { p.s0_sn = s0->stride[0]; p.s0_sh = s0->stride[1]; }
     if (sT) { p.sT_sn = sT->stride[0]; p.sT_sh = sT->stride[1]; }
 
-    Dims d{B, T, H, dk, dv, N, varlen};
+    p.nh = nh;
+    Dims d{B, Tw, H, dk, dv, N, varlen};  // items count k/v/beta rows
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     const int* cup = varlen ? static_cast<const int*>(cu->data) : nullptr;
     if (gate) return dispatch<true>(p, d, dev, sms, stream, forced_s, cup, dt);
@@ -577,6 +583,26 @@ dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn
     if (!g) return DN_ERR_INVALID_ARG;
     return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     stream, seg_chunks);
+}
+
+dn_status gated_deltaproduct_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                 const dn_tensor* beta, const dn_tensor* g,
+                                 const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                 int n_h, int chunk_size, dn_tensor* out,
+                                 dn_tensor* final_state, void* stream) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, 0, n_h);
+}
+
+dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                    const dn_tensor* beta, const dn_tensor* g,
+                                    const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                    int n_h, int chunk_size, dn_tensor* out,
+                                    dn_tensor* final_state, void* stream, int seg_chunks) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, seg_chunks, n_h);
 }
 
 const char* deltanet_status_string(dn_status s) {

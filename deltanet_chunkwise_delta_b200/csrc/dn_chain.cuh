@@ -256,6 +256,8 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     E* og = static_cast<E*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
     const float* bg = p.beta + it.b * p.b_sb + it.head * p.b_sh;
     const float* gg = GATED ? p.g + it.b * p.g_sb + it.head * p.g_sh : nullptr;
+    // Gated Delta Product: item token ranges count virtual steps, nsub per token
+    const int nsub = (GATED && p.nh > 1) ? p.nh : 1;
 
     const int ntok = it.tok1 - it.tok0;
     const int nchunks = (ntok + kChunk - 1) / kChunk;
@@ -263,7 +265,23 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     auto issue_load = [&](int r, int stg) {
         const int t0 = it.tok0 + r * kChunk;
         const int rows = min(kChunk, it.tok1 - t0);
-        if (HAS_Q) load_tile<E, DK>(Qs + stg * (L::Q_BYTES / L::ES), qg + t0 * p.q_st, p.q_st, rows);
+        if (HAS_Q) {
+            if (GATED && nsub > 1) {
+                // the query of token m / nsub sits on its last step; other steps read zeros
+                constexpr int V = 16 / sizeof(E);
+                constexpr int CPR = DK / V;
+                E* dst = Qs + stg * (L::Q_BYTES / L::ES);
+                for (int idx = tid; idx < kChunk * CPR; idx += kThreads) {
+                    const int r = idx / CPR, c = idx % CPR;
+                    const int m = t0 + r;
+                    const bool ok = r < rows && m % nsub == nsub - 1;
+                    const E* src = ok ? qg + (int64_t)(m / nsub) * p.q_st + c * V : qg;
+                    cp_async16(smem_addr(dst + SW::template off<DK>(r, c * V)), src, ok ? 16 : 0);
+                }
+            } else {
+                load_tile<E, DK>(Qs + stg * (L::Q_BYTES / L::ES), qg + t0 * p.q_st, p.q_st, rows);
+            }
+        }
         load_tile<E, DK>(Ks + stg * (L::K_BYTES / L::ES), kg + t0 * p.k_st, p.k_st, rows);
         if (HAS_V) load_tile<E, NX>(Vs + stg * (L::V_BYTES / L::ES), vg + t0 * p.v_st, p.v_st, rows);
         if (tid < kChunk) {
@@ -276,10 +294,12 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
             // wait, with no barrier); rows past the run read g = 0, an identity step
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                // the decay of token m / nsub sits on its first step; other steps read g = 0
                 const int i = 2 * lane + h;
-                const bool ok = i < rows;
-                cp_async4(smem_addr(gates + stg * kChunk + i), ok ? gg + (t0 + i) * p.g_st : gg,
-                          ok ? 4 : 0);
+                const int m = t0 + i;
+                const bool ok = i < rows && m % nsub == 0;
+                cp_async4(smem_addr(gates + stg * kChunk + i),
+                          ok ? gg + (int64_t)(m / nsub) * p.g_st : gg, ok ? 4 : 0);
             }
         }
         cp_async_commit();
@@ -453,8 +473,10 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
             const int rows = min(kChunk, it.tok1 - t0);
             for (int idx = tid; idx < kChunk * CPR; idx += kThreads) {
                 const int rr = idx / CPR, c = idx % CPR;
-                if (rr < rows)
-                    *reinterpret_cast<int4*>(og + (t0 + rr) * p.o_st + c * V) =
+                const int m = t0 + rr;
+                // one output row per token: the last of its nsub steps
+                if (rr < rows && m % nsub == nsub - 1)
+                    *reinterpret_cast<int4*>(og + (int64_t)(m / nsub) * p.o_st + c * V) =
                         *reinterpret_cast<const int4*>(Os + SW::template off<NX>(rr, c * V));
             }
         }

@@ -76,6 +76,10 @@ struct Params {
     int64_t o_sb, o_st, o_sh;
     int64_t b_sb, b_st, b_sh;
     int64_t g_sb, g_st, g_sh;
+    // Gated Delta Product: delta-rule writes per token (<= 1: one).  Token ranges of the
+    // items then count virtual steps m (k, v, beta rows); q, g and o rows are tokens
+    // m / nh, read (q) and written (o) at the last step of a token, g at its first.
+    int nh;
     int64_t s0_sn, s0_sh;
     int64_t sT_sn, sT_sh;
     float* wsP;          // [slots][d_k][d_k]

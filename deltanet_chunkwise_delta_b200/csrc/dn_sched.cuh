@@ -65,8 +65,10 @@ inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots
 // Also numbers the chunks of all sequences in input order (cumchunks[N + 1],
 // counts[3] = total) for the UT pre-pass.
 // Scratch: nc[N], order[N], offs[N][4].
-__global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, int N, int T,
-                                                   int H, int forced_s, int max_slots,
+// cu_mul: token ranges are cu[n] * cu_mul (Gated Delta Product: cu counts tokens, the
+// items count virtual steps, cu_mul per token); T counts the same units as the items.
+__global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, int cu_mul, int N,
+                                                   int T, int H, int forced_s, int max_slots,
                                                    int slots, CostModel m, Item* itemsC,
                                                    Item* itemsA, Item* itemsScan, int* counts,
                                                    int* nc, int* order, int4* offs, int* cumchunks,
@@ -85,11 +87,11 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
         s_carry = make_int4(0, 0, 0, 0);
     }
     __syncthreads();
-    if (N > 0 && tid == 0 && (cu[0] != 0 || cu[N] != T)) s_err = 1;
+    if (N > 0 && tid == 0 && (cu[0] != 0 || (long long)cu[N] * cu_mul != T)) s_err = 1;
     for (int n = tid; n < N; n += blockDim.x) {
-        const int a = cu[n], e = cu[n + 1];
-        if (e < a || a < 0 || e > T) atomicOr(&s_err, 1);
-        const int L = e > a ? e - a : 0;
+        const long long a64 = (long long)cu[n] * cu_mul, e64 = (long long)cu[n + 1] * cu_mul;
+        if (e64 < a64 || a64 < 0 || e64 > T) atomicOr(&s_err, 1);
+        const int L = e64 > a64 && e64 <= T && a64 >= 0 ? (int)(e64 - a64) : 0;
         const int c = (L + kChunk - 1) / kChunk;
         nc[n] = c;
         atomicMax(&s_lmax, c);
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(1024) k_schedule(const int* __restrict__ cu, i
         const int c = nc[n];
         const int G = c > 0 ? (c + s - 1) / s : 1;
         const int4 o = offs[pos];
-        const int a = cu[n], e = cu[n + 1];
+        const int a = cu[n] * cu_mul, e = cu[n + 1] * cu_mul;  // validated above
         for (int h = 0; h < H; ++h) {
             const int slot = o.w + h * (G - 1);
             for (int g = 0; g < G; ++g) {

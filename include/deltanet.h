@@ -142,6 +142,50 @@ dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn
                                 void* stream, int seg_chunks);
 
 /*
+ * gated_deltaproduct_fwd -- Gated Delta Product forward pass ("Linear
+ * Attention, Visualized", section "Gated Delta Product (GDP)"): each token makes
+ * n_h delta-rule writes, each with its own key, value and beta, after one decay
+ * of the state and before the token's readout:
+ *
+ *     S_{t,0} = a_t S_{t-1},
+ *     S_{t,j} = (I - beta_{t,j} k_{t,j}^T k_{t,j}) S_{t,j-1} + beta_{t,j} k_{t,j}^T v_{t,j}
+ *               for j = 1 .. n_h,
+ *     S_t = S_{t,n_h},  o_t = q_t S_t.
+ *
+ * Evaluated as that section's "GDP as GDN over a virtual sequence": the writes
+ * are the steps m = n_h (t - 1) + j of a sequence n_h times longer, with the
+ * decay on each token's first step and the query on its last; the kernels read
+ * the query, the decay and write the output through that index map, so nothing
+ * of the virtual sequence is materialised.
+ *
+ *   q             [B, T, H, d_k]        one row per token
+ *   k             [B, T * n_h, H, d_k]  n_h rows per token, substep-major: row
+ *                                       (t * n_h + j - 1) is write j of token t
+ *                                       (the [B, T, n_h, H, d] layout, flattened)
+ *   v             [B, T * n_h, H, d_v]
+ *   beta          [B, T * n_h, H] fp32
+ *   g             [B, T, H] fp32        ln a_t, one per token (as gated_deltanet_fwd)
+ *   cu_seqlens    token offsets (not write offsets), or NULL
+ *   n_h           writes per token, 1 .. 1024 (1 is gated_deltanet_fwd)
+ *   out           [B, T, H, d_v]        one row per token
+ *   other arguments, layouts, ownership, aliasing and errors as gated_deltanet_fwd;
+ *   B * T * n_h must stay below 2^31.
+ */
+dn_status gated_deltaproduct_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                 const dn_tensor* beta, const dn_tensor* g,
+                                 const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                 int n_h, int chunk_size, dn_tensor* out,
+                                 dn_tensor* final_state, void* stream);
+
+/* gated_deltaproduct_fwd with the seg_chunks override of deltanet_fwd_ex (runs
+ * count chunks of the virtual sequence). */
+dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                                    const dn_tensor* beta, const dn_tensor* g,
+                                    const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                                    int n_h, int chunk_size, dn_tensor* out,
+                                    dn_tensor* final_state, void* stream, int seg_chunks);
+
+/*
  * deltanet_fwd_noalloc -- the forward pass without any device allocation.
  * (No counterpart on the pages: this is a deployment variant of deltanet_fwd.)
  *
@@ -196,7 +240,8 @@ int deltanet_last_launches(void);
 
 /*
  * deltanet_set_kernel_events -- profiling hook.  While set (non-NULL), every
- * deltanet_fwd / gated_deltanet_fwd (and _ex) call on this thread records start_event on
+ * deltanet_fwd / gated_deltanet_fwd / gated_deltaproduct_fwd (and _ex) call on this
+ * thread records start_event on
  * its stream right before launching the boundary-pass kernel (the output
  * kernel, which dominates the call) and stop_event right after it, so that
  * cudaEventElapsedTime gives that kernel's device time.  The caller owns the

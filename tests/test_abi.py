@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "deltanet.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b((?:gated_)?deltanet_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:gated_)?delta(?:net|product)_\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -159,3 +159,29 @@ def test_gated_rejects_bad_gate(lib):
     r = lambda x: ctypes.byref(x)
     assert lib.gated_deltanet_fwd_ex(r(q), r(k), r(v), r(beta), None, None, None, 64, r(out),
                                      None, None, 2) == L.DN_ERR_INVALID_ARG
+
+
+def test_gdp_rejects_bad_rows(lib):
+    """Gated Delta Product: k, v and beta hold n_h rows per token of q; g and out
+    one; n_h >= 1; the gate is required."""
+    r = lambda x: None if x is None else ctypes.byref(x)
+    base = 0x100000000
+    q = desc([2, 50, 3, 128], L.DN_BF16, base)
+    k = desc([2, 100, 3, 128], L.DN_BF16, base + 1 * 2**28)
+    v = desc([2, 100, 3, 64], L.DN_BF16, base + 2 * 2**28)
+    beta = desc([2, 100, 3], L.DN_F32, base + 3 * 2**28)
+    out = desc([2, 50, 3, 64], L.DN_BF16, base + 4 * 2**28)
+    g = desc([2, 50, 3], L.DN_F32, base + 7 * 2**28)
+    f = lambda qq, kk, vv, bb, gg, nh, oo: lib.gated_deltaproduct_fwd(
+        r(qq), r(kk), r(vv), r(bb), r(gg), None, None, nh, 64, r(oo), None, None)
+    assert f(q, k, v, beta, None, 2, out) == L.DN_ERR_INVALID_ARG
+    assert f(q, k, v, beta, g, 0, out) == L.DN_ERR_INVALID_ARG
+    assert f(q, k, v, beta, g, 3, out) == L.DN_ERR_INVALID_ARG          # k has 2 rows per token
+    g_rows = desc([2, 100, 3], L.DN_F32, g.data)
+    assert f(q, k, v, beta, g_rows, 2, out) == L.DN_ERR_INVALID_ARG     # g is per token
+    o_rows = desc([2, 100, 3, 64], L.DN_BF16, out.data)
+    assert f(q, k, v, beta, g, 2, o_rows) == L.DN_ERR_INVALID_ARG       # out is per token
+    b_tok = desc([2, 50, 3], L.DN_F32, beta.data)
+    assert f(q, k, v, b_tok, g, 2, out) == L.DN_ERR_INVALID_ARG         # beta is per write
+    assert lib.gated_deltaproduct_fwd(r(q), r(k), r(v), r(beta), r(g), None, None, 2, 32,
+                                      r(out), None, None) == L.DN_ERR_UNSUPPORTED
