@@ -22,7 +22,8 @@ DN_OK, DN_ERR_INVALID_ARG, DN_ERR_UNSUPPORTED, DN_ERR_ALIAS, DN_ERR_CUDA, \
 DN_F32, DN_BF16, DN_I32 = 0, 1, 2
 
 EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "gated_deltanet_fwd", "gated_deltanet_fwd_ex",
-            "gated_deltaproduct_fwd", "gated_deltaproduct_fwd_ex", "deltanet_status_string",
+            "gated_deltaproduct_fwd", "gated_deltaproduct_fwd_ex", "deltanet_fwd_states",
+            "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
             "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events")
 
@@ -77,6 +78,9 @@ def load(path: Optional[str] = None):
         lib.gated_deltaproduct_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int,
                                                   ctypes.c_int, P, P, ctypes.c_void_p,
                                                   ctypes.c_int]
+        lib.deltanet_fwd_states.restype = ctypes.c_int
+        lib.deltanet_fwd_states.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P, P,
+                                            ctypes.c_void_p, ctypes.c_int]
         lib.deltanet_fwd_noalloc.restype = ctypes.c_int
         lib.deltanet_fwd_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
         lib.deltanet_status_string.restype = ctypes.c_char_p
@@ -208,6 +212,47 @@ def gated_deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: 
     if st != DN_OK:
         raise DeltaNetError(st, status_string(st))
     return out, final_state
+
+
+def chunk_state_rows(B: int, T: int, cu_seqlens: Optional[torch.Tensor] = None,
+                     chunk_size: int = 64) -> int:
+    """Rows of the chunk-states buffer: B * ceil(T / C) for a dense batch; for packed
+    input ceil(T / C) + N, a bound on the sum of ceil(L_n / C)."""
+    n_c = (T + chunk_size - 1) // chunk_size
+    return B * n_c if cu_seqlens is None else n_c + cu_seqlens.numel() - 1
+
+
+def deltanet_fwd_states(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.Tensor,
+                        g: Optional[torch.Tensor] = None,
+                        initial_state: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, chunk_size: int = 64,
+                        out: Optional[torch.Tensor] = None,
+                        final_state: Optional[torch.Tensor] = None,
+                        chunk_states: Optional[torch.Tensor] = None, stream=None,
+                        seg_chunks: int = 0):
+    """DeltaNet (g None) or Gated DeltaNet forward that also returns the state
+    entering every chunk: chunk_states [rows, H, d_k, d_v] fp32 with row = global
+    chunk index (see ``chunk_state_rows``; allocated zeroed when not given).
+    Returns (out, final_state, chunk_states)."""
+    if not q.is_cuda:
+        raise ValueError("deltanet_fwd_states runs on CUDA tensors only")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    if chunk_states is None:
+        rows = chunk_state_rows(B, T, cu_seqlens, chunk_size)
+        chunk_states = torch.zeros((rows, H, dk, dv), dtype=torch.float32, device=q.device)
+    ds = [describe(t) for t in (q, k, v, beta, g, initial_state, cu_seqlens, out, final_state,
+                                chunk_states)]
+    args = [_ref(x) for x in ds[:7]] + [int(chunk_size)] + [_ref(x) for x in ds[7:]]
+    st = load().deltanet_fwd_states(*args, _stream_handle(q.device, stream), int(seg_chunks))
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state, chunk_states
 
 
 def gated_deltaproduct_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

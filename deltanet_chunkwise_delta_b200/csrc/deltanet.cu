@@ -242,9 +242,11 @@ template <typename E, int DK, int DV, int STAGES, bool GATED>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
     // bf16 DeltaNet with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels; Gated
-    // DeltaNet and the other shapes on the mma.sync chain kernels
-    constexpr bool kTc =
+    // DeltaNet, the other shapes and calls that keep the chunk-start states on the mma.sync
+    // chain kernels (which hold the state in registers)
+    constexpr bool kTcShape =
         !GATED && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
+    const bool use_tc = kTcShape && !p.cs;
     using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED>;
@@ -260,7 +262,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kPrep = k_ut_prep;
     constexpr int smemPrep = PrepSmem::TOTAL;
     dn_status st;
-    if (kTc) {
+    if (use_tc) {
         if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
         if ((st = set_smem(kAt, dev, tcs::SMEM_BYTES)) != DN_OK) return st;
         if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
@@ -275,7 +277,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     if ((st = set_smem(kS8, dev, smemS8)) != DN_OK) return st;
     if ((st = set_smem(kS16, dev, smemS16)) != DN_OK) return st;
     CUtensorMap tq, tk, tv, to;
-    if (kTc) {
+    if (use_tc) {
         const int64_t Bq = d.varlen ? 1 : d.B;
         if ((st = make_token_map(&tq, p.q, Bq, d.T, d.H, p.q_sb, p.q_st, p.q_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tk, p.k, Bq, d.T, d.H, p.k_sb, p.k_st, p.k_sh)) != DN_OK) return st;
@@ -294,7 +296,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         if (forced_s > 0) {
             s = forced_s;
         } else {
-            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, kTc);
+            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, use_tc);
             s = ch.s;
         }
         G = n_c_max > 0 ? (int)((n_c_max + s - 1) / s) : 1;
@@ -303,7 +305,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         nC = chains * G;
         // tensor-core path: run 0 of a split chain is computed once, by its boundary item,
         // next to the summary pass (which then has no end-state items)
-        e_in_c = kTc && G >= 2;
+        e_in_c = use_tc && G >= 2;
         nA = G >= 2 ? chains * (G - 1 - (e_in_c ? 1 : 0)) : 0;
         nScan = G >= 2 ? chains : 0;
     } else {
@@ -331,7 +333,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     // UT factors of every (chunk, head): chunks <= ceil(T / C) per row (+1 per sequence)
     const int64_t chunk_ub = d.varlen ? n_c_max + d.N : d.B * n_c_max;
     const size_t off_T = off_SS + up256((size_t)slots * DK * DV * 4);
-    bytes = off_T + (kTc ? (size_t)chunk_ub * d.H * kUnitBytes : 0);
+    bytes = off_T + (use_tc ? (size_t)chunk_ub * d.H * kUnitBytes : 0);
     StreamWs ws;
     if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
     char* base = ws.buf;
@@ -385,7 +387,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             kS16<<<dim3((unsigned)nScan, DV / 16), scan_threads<DK, 16>(), smemS16, stream>>>(tp, p);
     };
     int launches = d.varlen ? 1 : 0;
-    if (kTc) {
+    if (use_tc) {
         const int64_t units = chunk_ub * d.H;
         if (units > 0) {
             const int grid = (int)std::min<int64_t>(units, (int64_t)sms * kPrepCtasPerSm);
@@ -450,10 +452,11 @@ dn_status dispatch(Params& p, const Dims& d, int dev, int sms, cudaStream_t stre
 // gate: Gated DeltaNet's log decay [B, T, H] fp32, or null for DeltaNet.
 // nh: delta-rule writes per token (Gated Delta Product; 1 otherwise): k, v and beta hold
 // T * nh rows, q, gate and out T rows, cu_seqlens counts tokens.
+// cs: chunk-start states [rows, H, d_k, d_v] fp32, or null.
 dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                    const dn_tensor* beta, const dn_tensor* gate, const dn_tensor* s0,
                    const dn_tensor* cu, int chunk, dn_tensor* out, dn_tensor* sT,
-                   void* stream_ptr, int forced_s, int nh = 1) {
+                   void* stream_ptr, int forced_s, int nh = 1, dn_tensor* cs = nullptr) {
     if (!q || !k || !v || !beta || !out) return DN_ERR_INVALID_ARG;
     if (q->ndim != 4 || k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return DN_ERR_INVALID_ARG;
     if (forced_s < 0 || nh < 1 || (nh > 1 && !gate)) return DN_ERR_INVALID_ARG;
@@ -499,6 +502,16 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     const int64_t sd[4] = {N, H, dk, dv};
     if (s0 && (!shape_eq(s0, 4, sd) || !state_tensor_ok(s0, dv))) return DN_ERR_INVALID_ARG;
     if (sT && (!shape_eq(sT, 4, sd) || !state_tensor_ok(sT, dv))) return DN_ERR_INVALID_ARG;
+    if (cs) {
+        // one row per chunk: exactly B * ceil(T / C) for a dense batch; for packed input at
+        // least ceil(T / C) + N, which bounds the sum of ceil(L_n / C) over the sequences
+        const int64_t n_c = (Tw + kChunk - 1) / kChunk;
+        const int64_t need = varlen ? n_c + N : B * n_c;
+        if (cs->ndim != 4 || cs->shape[1] != H || cs->shape[2] != dk || cs->shape[3] != dv ||
+            !state_tensor_ok(cs, dv))
+            return DN_ERR_INVALID_ARG;
+        if (varlen ? cs->shape[0] < need : cs->shape[0] != need) return DN_ERR_INVALID_ARG;
+    }
 
     if (chunk != kChunk) return DN_ERR_UNSUPPORTED;
     const bool bf16_ok = (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
@@ -513,6 +526,11 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
             if (in && overlap(o, in)) return DN_ERR_ALIAS;
     }
     if (sT && overlap(out, sT)) return DN_ERR_ALIAS;
+    if (cs) {
+        for (const dn_tensor* in : ins)
+            if (in && overlap(cs, in)) return DN_ERR_ALIAS;
+        if (overlap(cs, out) || (sT && overlap(cs, sT))) return DN_ERR_ALIAS;
+    }
 
     int dev = 0, sms = 0;
     dn_status st = device_check(dev, sms);
@@ -538,6 +556,12 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     if (sT) { p.sT_sn = sT->stride[0]; p.sT_sh = sT->stride[1]; }
 
     p.nh = nh;
+    if (cs && numel(cs)) {
+        p.cs = static_cast<float*>(cs->data);
+        p.cs_sc = cs->stride[0];
+        p.cs_sh = cs->stride[1];
+        p.cs_rows = cs->shape[0];
+    }
     Dims d{B, Tw, H, dk, dv, N, varlen};  // items count k/v/beta rows
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     const int* cup = varlen ? static_cast<const int*>(cu->data) : nullptr;
@@ -583,6 +607,16 @@ dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn
     if (!g) return DN_ERR_INVALID_ARG;
     return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     stream, seg_chunks);
+}
+
+dn_status deltanet_fwd_states(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                              const dn_tensor* beta, const dn_tensor* g,
+                              const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                              int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                              dn_tensor* chunk_states, void* stream, int seg_chunks) {
+    if (!chunk_states) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, seg_chunks, 1, chunk_states);
 }
 
 dn_status gated_deltaproduct_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,

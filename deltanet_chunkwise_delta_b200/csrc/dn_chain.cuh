@@ -352,6 +352,25 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
             }
         }
 
+        if constexpr (HAS_Q) {
+            // the state entering chunk r, for a backward pass (row = global chunk index)
+            const int64_t row = (int64_t)it.cbase + r;
+            if (p.cs && row < p.cs_rows) {
+                float* dst = p.cs + row * p.cs_sc + it.head * p.cs_sh;
+#pragma unroll
+                for (int m = 0; m < MT_S; ++m)
+#pragma unroll
+                    for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int rr = s_r0 + 16 * m + g8 + 8 * h;
+                            const int c = x_c0 + 8 * nt + 2 * t4;
+                            *reinterpret_cast<float2*>(dst + rr * NX + c) =
+                                make_float2(s[m][nt][2 * h], s[m][nt][2 * h + 1]);
+                        }
+            }
+        }
+
         // (a) state -> operand copy
 #pragma unroll
         for (int m = 0; m < MT_S; ++m) store_frag<NT_X, NX>(Xb, s_r0 + 16 * m, x_c0, s[m], 1.f);

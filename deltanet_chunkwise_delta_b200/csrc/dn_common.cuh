@@ -80,6 +80,10 @@ struct Params {
     // items then count virtual steps m (k, v, beta rows); q, g and o rows are tokens
     // m / nh, read (q) and written (o) at the last step of a token, g at its first.
     int nh;
+    // Chunk-start states for a backward pass: the state entering every chunk, fp32
+    // [rows][H][d_k][d_v] at row (global chunk index), or null.
+    float* cs;
+    int64_t cs_sc, cs_sh, cs_rows;
     int64_t s0_sn, s0_sh;
     int64_t sT_sn, sT_sh;
     float* wsP;          // [slots][d_k][d_k]

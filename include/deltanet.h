@@ -142,6 +142,34 @@ dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn
                                 void* stream, int seg_chunks);
 
 /*
+ * deltanet_fwd_states -- the forward pass that also keeps the state entering
+ * every chunk, the chunk-boundary states S_[r] that a backward pass reuses
+ * ("Linear Attention, Visualized", section "Chunkwise algorithm": the chunk
+ * states are the only quantities carried between chunks).
+ *
+ *   g             NULL for DeltaNet, or Gated DeltaNet's log decay [B, T, H] fp32
+ *   chunk_states  [rows, H, d_k, d_v] fp32 (state layout rules): row = global
+ *                 chunk index, chunks numbered per sequence in input order
+ *                 (dense: b * ceil(T / 64) + r; packed: the chunks of earlier
+ *                 sequences first, ceil(L_n / 64) per sequence).  Dense batches
+ *                 need rows == B * ceil(T / 64); packed input rows >=
+ *                 ceil(T / 64) + N (rows past the total are not written).  Row r
+ *                 holds the state before chunk r's tokens (row 0 of a sequence is
+ *                 its initial state).
+ *   seg_chunks    as deltanet_fwd_ex (0: the library chooses)
+ *   other arguments, layouts, ownership and errors as deltanet_fwd /
+ *   gated_deltanet_fwd; chunk_states may not overlap any other tensor.
+ *
+ * These calls run on the mma.sync chain kernels, which keep the state in
+ * registers and store it at every chunk start.
+ */
+dn_status deltanet_fwd_states(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
+                              const dn_tensor* beta, const dn_tensor* g,
+                              const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                              int chunk_size, dn_tensor* out, dn_tensor* final_state,
+                              dn_tensor* chunk_states, void* stream, int seg_chunks);
+
+/*
  * gated_deltaproduct_fwd -- Gated Delta Product forward pass ("Linear
  * Attention, Visualized", section "Gated Delta Product (GDP)"): each token makes
  * n_h delta-rule writes, each with its own key, value and beta, after one decay
@@ -240,8 +268,8 @@ int deltanet_last_launches(void);
 
 /*
  * deltanet_set_kernel_events -- profiling hook.  While set (non-NULL), every
- * deltanet_fwd / gated_deltanet_fwd / gated_deltaproduct_fwd (and _ex) call on this
- * thread records start_event on
+ * deltanet_fwd / gated_deltanet_fwd / gated_deltaproduct_fwd (and _ex) /
+ * deltanet_fwd_states call on this thread records start_event on
  * its stream right before launching the boundary-pass kernel (the output
  * kernel, which dominates the call) and stop_event right after it, so that
  * cudaEventElapsedTime gives that kernel's device time.  The caller owns the

@@ -185,3 +185,19 @@ def test_gdp_rejects_bad_rows(lib):
     assert f(q, k, v, b_tok, g, 2, out) == L.DN_ERR_INVALID_ARG         # beta is per write
     assert lib.gated_deltaproduct_fwd(r(q), r(k), r(v), r(beta), r(g), None, None, 2, 32,
                                       r(out), None, None) == L.DN_ERR_UNSUPPORTED
+
+
+def test_states_rejects_bad_buffer(lib):
+    """deltanet_fwd_states: chunk_states is required, fp32 [rows, H, d_k, d_v] with
+    rows = B * ceil(T / 64) (dense), and may not overlap another tensor."""
+    r = lambda x: None if x is None else ctypes.byref(x)
+    q, k, v, beta, s0, out, sT = good()           # B = 2, T = 100: 2 chunks per row
+    cs = desc([4, 3, 128, 64], L.DN_F32, 0x100000000 + 8 * 2**28)
+    f = lambda c, o=out: lib.deltanet_fwd_states(r(q), r(k), r(v), r(beta), None, None, None,
+                                                 64, r(o), None, r(c), None, 0)
+    assert f(None) == L.DN_ERR_INVALID_ARG
+    assert f(desc([3, 3, 128, 64], L.DN_F32, cs.data)) == L.DN_ERR_INVALID_ARG
+    assert f(desc([4, 3, 128, 64], L.DN_BF16, cs.data)) == L.DN_ERR_INVALID_ARG
+    assert f(desc([4, 3, 64, 128], L.DN_F32, cs.data)) == L.DN_ERR_INVALID_ARG
+    assert f(desc([4, 3, 128, 64], L.DN_F32, q.data)) == L.DN_ERR_ALIAS
+    assert f(cs, desc([2, 100, 3, 64], L.DN_BF16, cs.data)) == L.DN_ERR_ALIAS
