@@ -11,7 +11,9 @@ Two independent float64 statements of the method:
   ("Linear Attention, Visualized", DeltaNet, "Recurrent form"), threaded over
   (sequence, head); with a gate ``g`` = ln a_t it runs the Gated DeltaNet
   recurrence of the same page (section "Gated DeltaNet (GDN)"), and with
-  ``n_sub`` > 1 the Gated Delta Product (section "Gated Delta Product (GDP)").  Built from
+  ``n_sub`` > 1 the Gated Delta Product (section "Gated Delta Product (GDP)");
+  with a gate per key channel, Kimi Delta Attention (section "Kimi Delta
+  Attention (KDA)").  Built from
   ``deltanet_oracle.c`` with gcc.
 * ``chunkwise`` (module) -- numpy float64 statements of the chunk form, the
   WY transition product, the segment composition and the full-sequence closed
@@ -53,11 +55,11 @@ def _load():
     with _lock:
         if _lib is None:
             lib = ctypes.CDLL(build())
-            f = lib.gdp_oracle_fwd
+            f = lib.delta_oracle_fwd
             f.restype = ctypes.c_int
             f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
-                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                          ctypes.c_int64,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                           ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
@@ -76,7 +78,8 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
 
     q, k: [B, T, H, dk]; v: [B, T, H, dv] (fp32, bf16 or fp64); beta: [B, T, H]
     fp32; initial_state: [N, H, dk, dv] or None; cu_seqlens: int32 [N+1] or None;
-    g: [B, T, H] fp32 log decay (Gated DeltaNet) or None (plain DeltaNet).
+    g: [B, T, H] fp32 log decay (Gated DeltaNet), [B, T, H, dk] one log decay per
+    key channel (Kimi Delta Attention), or None (plain DeltaNet).
     n_sub > 1: Gated Delta Product with n_sub writes per token; k, v, beta then
     hold [B, T * n_sub, H, .] rows (substep-major within a token) while q, g, out
     and cu_seqlens count tokens.
@@ -111,12 +114,13 @@ def token_recurrence(q, k, v, beta, initial_state=None, cu_seqlens=None,
     fs = torch.full((n_seq, H, dk, dv), float("nan"), dtype=torch.float64)
     if n_threads is None:
         n_threads = os.cpu_count() or 1
-    if gate is not None and tuple(gate.shape) != (B, T, H):
-        raise ValueError("g must have one value per (token, head)")
-    rc = lib.gdp_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta), _ptr(gate),
-                            _ptr(s0), _ptr(cu), n_seq, B, T, H, dk, dv, int(n_sub), h0, h1,
-                            _ptr(out), 0 if out_dtype == torch.float32 else 2,
-                            _ptr(fs), int(n_threads))
+    per_key = gate is not None and gate.dim() == 4
+    if gate is not None and tuple(gate.shape) not in ((B, T, H), (B, T, H, dk)):
+        raise ValueError("g must hold one value per (token, head) or per key channel")
+    rc = lib.delta_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), codes[q.dtype], _ptr(beta),
+                              _ptr(gate), int(per_key), _ptr(s0), _ptr(cu), n_seq, B, T, H, dk,
+                              dv, int(n_sub), h0, h1, _ptr(out),
+                              0 if out_dtype == torch.float32 else 2, _ptr(fs), int(n_threads))
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return out, fs

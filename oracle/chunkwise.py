@@ -315,3 +315,84 @@ def gdp_substeps(Q, K, V, beta, a, n_h: int, S0):
             S = A @ S + beta[m] * np.outer(K[m], V[m])
         O[t] = Q[t] @ S
     return O, S
+
+
+# --- Gated Linear Attention and Kimi Delta Attention ("Linear Attention, Visualized",
+#     sections "Gated Linear Attention (GLA)" and "Kimi Delta Attention (KDA)") ---
+#
+# Here the decay is a vector per token, A [n, d_k] with entries in (0, 1]: it
+# scales row c of the state (key channel c) by A[t, c].
+
+def channel_decay_products(A):
+    """lambda[i:j] = a_i o ... o a_j (elementwise, 1-based inclusive), the ones
+    vector when i > j."""
+    def lam(i, j):
+        return np.prod(A[i - 1:j], axis=0) if i <= j else np.ones(A.shape[1])
+    return lam
+
+
+def kda_chunk_factors(Qc, Kc, Vc, bc, Ac):
+    """The KDA "Complete per-chunk algorithm", quantities as the page defines them:
+      q<-_l = lambda[1:l] o q_l, k<-_l = lambda[1:l] o k_l, k->_l = lambda[l+1:C] o k_l;
+      A[l, m] = q_l (lambda[m+1:l] o k_m)^T for m <= l; L[l, m] = k_l (lambda[m+1:l] o k_m)^T
+      for m < l; (I + B L) T = B, U = T V, W<- = T K<-.
+    Qc may be None (no readout)."""
+    c = Kc.shape[0]
+    lam = channel_decay_products(Ac)
+    Ql = None if Qc is None else np.stack([lam(1, l + 1) * Qc[l] for l in range(c)])
+    Kl = np.stack([lam(1, l + 1) * Kc[l] for l in range(c)])
+    Kr = np.stack([lam(l + 2, c) * Kc[l] for l in range(c)])
+    Am = np.zeros((c, c))
+    L = np.zeros((c, c))
+    for l in range(c):
+        for m in range(l + 1):
+            km = lam(m + 2, l + 1) * Kc[m]
+            if Qc is not None:
+                Am[l, m] = Qc[l] @ km
+            if m < l:
+                L[l, m] = Kc[l] @ km
+    Bm = np.diag(bc)
+    T = solve_triangular(np.eye(c) + Bm @ L, Bm, lower=True, unit_diagonal=True)
+    return {"Ql": Ql, "Kl": Kl, "Kr": Kr, "A": Am, "L": L, "T": T,
+            "U": (T @ Vc if Vc is not None else None), "W": T @ Kl, "lamC": lam(1, c)}
+
+
+def kda_chunkwise(Q, K, V, beta, A, S0=None, C: int = 64):
+    """KDA threaded over the chunks: Z = U - W<- S, O = Q<- S + A Z,
+    S' = Diag(lambda[1:C]) S + K->^T Z.  Returns (O, S_final)."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    O = np.zeros((n, dv))
+    for s, e in chunk_bounds(n, C):
+        f = kda_chunk_factors(Q[s:e], K[s:e], V[s:e], beta[s:e], A[s:e])
+        Z = f["U"] - f["W"] @ S
+        O[s:e] = f["Ql"] @ S + f["A"] @ Z
+        S = f["lamC"][:, None] * S + f["Kr"].T @ Z
+    return O, S
+
+
+def kda_segment_map(K, V, beta, A, C: int = 64):
+    """S_end = P S_start + H of a run of chunks under KDA: one chunk is
+    S' = (Diag(lambda[1:C]) - K->^T W<-) S + K->^T U; chunks compose in order."""
+    dk = K.shape[1]
+    P = np.eye(dk)
+    H = np.zeros((dk, V.shape[1]))
+    for s, e in chunk_bounds(K.shape[0], C):
+        f = kda_chunk_factors(None, K[s:e], V[s:e], beta[s:e], A[s:e])
+        Lam = np.diag(f["lamC"]) - f["Kr"].T @ f["W"]
+        P, H = Lam @ P, Lam @ H + f["Kr"].T @ f["U"]
+    return P, H
+
+
+def gla_chunkwise(Q, K, V, A, S0=None, C: int = 64):
+    """GLA's chunk form: O = Q<- S + A V, S' = Diag(lambda[1:C]) S + K->^T V."""
+    n, dk = K.shape
+    dv = V.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    O = np.zeros((n, dv))
+    for s, e in chunk_bounds(n, C):
+        f = kda_chunk_factors(Q[s:e], K[s:e], V[s:e], np.zeros(e - s), A[s:e])
+        O[s:e] = f["Ql"] @ S + f["A"] @ V[s:e]
+        S = f["lamC"][:, None] * S + f["Kr"].T @ V[s:e]
+    return O, S

@@ -31,12 +31,19 @@
  * k, v and beta then hold n_sub rows per token, substep-major within the token
  * (row t * n_sub + j - 1, i.e. [B, T * n_sub, H, .]); q, gate and out keep one
  * row per token.  n_sub = 1 is (Gated) DeltaNet.
+ *
+ * Kimi Delta Attention (same page, section "Kimi Delta Attention (KDA)") decays
+ * every key channel of the state at its own rate before the delta correction:
+ *     S_t = Diag(a_t) S_{t-1} + beta_t k_t^T (v_t - k_t Diag(a_t) S_{t-1}),
+ * with a_t in (0, 1]^{d_k} scaling row c of S by a_{t,c}.  Its gate arrives as
+ * g [B, T, H, dk] (gate_per_key = 1); the loop scales row c by exp(g_{t,c})
+ * and then runs the same prediction, correction and write.
  * S starts from the caller's initial state (or zero) at the first token of each
  * sequence.  No query scaling is applied.  Inputs stored as bf16 are widened
  * exactly to float64; every sum is accumulated in float64.
  *
  * Layouts (contiguous, row-major):
- *   q [B, T, H, dk]  out [B, T, H, dv]  gate [B, T, H] (fp32)
+ *   q [B, T, H, dk]  out [B, T, H, dv]  gate [B, T, H] or [B, T, H, dk] (fp32)
  *   k [B, T n_sub, H, dk]  v [B, T n_sub, H, dv]  beta [B, T n_sub, H] (fp32)
  *   init_state, final_state [N, H, dk, dv]
  * With cu_seqlens (host int32 [N+1]) B must be 1 and sequence n covers tokens
@@ -72,6 +79,7 @@ typedef struct {
     const int32_t* cu;
     int64_t n_seq, B, T, H, dk, dv, h_begin, h_end;
     int64_t n_sub;              /* delta-rule writes per token (1 for DeltaNet / GDN) */
+    int gate_per_key;           /* 1: gate holds one log decay per key channel (KDA) */
     void* out;
     int out_dtype;
     double* final_state;        /* may be NULL */
@@ -101,7 +109,14 @@ static void run_job(oracle_ctx* c, int64_t job, double* S, double* kt, double* q
         const int64_t tok = row0 + t;                 /* flattened (b, t) row */
         const int64_t q_off = (tok * H + h) * dk;
         const int64_t o_off = (tok * H + h) * dv;
-        if (c->gate) {
+        if (c->gate && c->gate_per_key) {
+            /* channelwise decay first: row a of S by exp(g_{t,a}) */
+            const float* ga = c->gate + (tok * H + h) * dk;
+            for (int64_t a = 0; a < dk; ++a) {
+                const double f = exp((double)ga[a]);
+                for (int64_t j = 0; j < dv; ++j) S[a * dv + j] *= f;
+            }
+        } else if (c->gate) {
             /* decay first: the prediction below reads a_t S_{t-1} */
             const double a = exp((double)c->gate[tok * H + h]);
             for (int64_t e = 0; e < dk * dv; ++e) S[e] *= a;
@@ -154,14 +169,15 @@ static void* worker(void* arg) {
 }
 
 /* Returns 0 on success, -1 on a bad argument, -2 on allocation failure.
- * gate may be NULL (no decay); n_sub >= 1 writes per token (T counts tokens,
- * cu_seqlens token offsets). */
-int gdp_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
-                   const float* beta, const float* gate, const double* init_state,
-                   const int32_t* cu_seqlens, int64_t n_seq,
-                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t n_sub,
-                   int64_t h_begin, int64_t h_end,
-                   void* out, int out_dtype, double* final_state, int n_threads) {
+ * gate may be NULL (no decay), one log decay per (token, head) (gate_per_key 0)
+ * or one per key channel (gate_per_key 1); n_sub >= 1 writes per token (T counts
+ * tokens, cu_seqlens token offsets). */
+int delta_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+                     const float* beta, const float* gate, int gate_per_key,
+                     const double* init_state, const int32_t* cu_seqlens, int64_t n_seq,
+                     int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t n_sub,
+                     int64_t h_begin, int64_t h_end,
+                     void* out, int out_dtype, double* final_state, int n_threads) {
     if ((B * T > 0) && (!q || !k || !v || !beta)) return -1;
     if (n_sub < 1) return -1;
     if (in_dtype != OR_F32 && in_dtype != OR_BF16 && in_dtype != OR_F64) return -1;
@@ -180,7 +196,7 @@ int gdp_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     c.q = q; c.k = k; c.v = v; c.in_dtype = in_dtype; c.beta = beta; c.gate = gate;
     c.init_state = init_state; c.cu = cu_seqlens; c.n_seq = n_seq;
     c.B = B; c.T = T; c.H = H; c.dk = dk; c.dv = dv;
-    c.h_begin = h_begin; c.h_end = h_end; c.n_sub = n_sub;
+    c.h_begin = h_begin; c.h_end = h_end; c.n_sub = n_sub; c.gate_per_key = gate_per_key != 0;
     c.out = out; c.out_dtype = out_dtype; c.final_state = final_state;
     c.n_jobs = n_seq * (h_end - h_begin);
     c.next_job = 0;
@@ -199,6 +215,18 @@ int gdp_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
     free(th);
     pthread_mutex_destroy(&c.lock);
     return 0;
+}
+
+/* Gated Delta Product with a scalar gate per token. */
+int gdp_oracle_fwd(const void* q, const void* k, const void* v, int in_dtype,
+                   const float* beta, const float* gate, const double* init_state,
+                   const int32_t* cu_seqlens, int64_t n_seq,
+                   int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t n_sub,
+                   int64_t h_begin, int64_t h_end,
+                   void* out, int out_dtype, double* final_state, int n_threads) {
+    return delta_oracle_fwd(q, k, v, in_dtype, beta, gate, 0, init_state, cu_seqlens, n_seq, B,
+                            T, H, dk, dv, n_sub, h_begin, h_end, out, out_dtype, final_state,
+                            n_threads);
 }
 
 /* Gated DeltaNet: one write per token (gate may be NULL: plain DeltaNet). */
