@@ -201,3 +201,22 @@ def test_states_rejects_bad_buffer(lib):
     assert f(desc([4, 3, 64, 128], L.DN_F32, cs.data)) == L.DN_ERR_INVALID_ARG
     assert f(desc([4, 3, 128, 64], L.DN_F32, q.data)) == L.DN_ERR_ALIAS
     assert f(cs, desc([2, 100, 3, 64], L.DN_BF16, cs.data)) == L.DN_ERR_ALIAS
+
+
+def test_binding_host_logic():
+    """Row count of the chunk-states buffer, and the wrappers refuse CPU tensors
+    (there is no host implementation to fall back to)."""
+    import torch
+    import deltanet_chunkwise_delta_b200 as dn
+    assert dn.chunk_state_rows(8, 2048) == 8 * 32
+    assert dn.chunk_state_rows(3, 65) == 3 * 2
+    cu = torch.tensor([0, 1, 65, 65, 200], dtype=torch.int32)   # 1 + 1 + 0 + 3 = 5 chunks
+    assert dn.chunk_state_rows(1, 200, cu) == 4 + 4 >= 5
+    x = torch.zeros(1, 4, 1, 64)
+    b = torch.zeros(1, 4, 1)
+    with pytest.raises(ValueError):
+        dn.gated_deltanet_fwd(x, x, x, b, b)
+    with pytest.raises(ValueError):
+        dn.gated_deltaproduct_fwd(x, x, x, b, b, 1)
+    with pytest.raises(ValueError):
+        dn.deltanet_fwd_states(x, x, x, b)
