@@ -4,10 +4,16 @@
 One step = one deltanet_fwd call over the whole workload (every step of the
 path: WY/UT factors, segment summaries, segment scan, boundary pass with
 output); for the Gated DeltaNet workloads (gdn_*) one gated_deltanet_fwd call, for
-the Gated Delta Product workloads (gdp_*) one gated_deltaproduct_fwd call.  Default workload: the 1.3B-model layer shape (B=8, H=16, T=2048,
-d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 beta, zero initial state, fp32
-final state), synthetic seeded inputs.  Inputs (q, k, v: 201 MB) exceed the
-126 MB L2, so no flush is needed between steps.
+the Gated Delta Product workloads (gdp_*) one gated_deltaproduct_fwd call.
+Default workload: the 1M-token context (B=1, H=8, T=1048576, d_k=d_v=128,
+chunk 64, bf16 q/k/v, fp32 beta, zero initial state, fp32 final state), the
+largest single-GPU configuration, on synthetic seeded inputs.  Its inputs
+(q, k, v: 6.4 GB) exceed the 126 MB L2, so no flush is needed between steps;
+so do those of every other workload here (the 1.3B layer: 201 MB).
+
+The line also carries the parity of the timed call itself: its outputs on the
+CPU-baseline sample (the first tokens of the sequence, all heads) against the
+float64 oracle run on the same prefix, which yields the same outputs there.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
 oracle on a bounded sample of the same workload instead.
@@ -118,7 +124,7 @@ _REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown"
 class ClockSampler:
     """Samples SM clock and clock-event reasons with NVML while running."""
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.period = period_s
         self.samples = []
         self.reasons = 0
@@ -195,9 +201,9 @@ def barrier(ws: int):
 
 # ---- oracle timing (CPU baseline / reference arm) -----------------------------
 
-def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0):
+def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0, outputs: bool = False):
     """Runs the float64 oracle on tokens [0, tokens) of batch row b, all heads;
-    returns (seconds, threads)."""
+    returns (seconds, threads), and with ``outputs`` also the oracle's out."""
     import oracle
     n_threads = os.cpu_count() or 1
     sl = lambda t: t[b:b + 1, :tokens].contiguous()
@@ -205,9 +211,21 @@ def time_oracle(x, w: wl.Workload, tokens: int, b: int = 0):
     gate = None if x.get("g") is None else sl(x["g"])
     slw = lambda t: t[b:b + 1, :tokens * w.nh].contiguous()   # nh rows per token
     t0 = time.perf_counter()
-    oracle.token_recurrence(sl(x["q"]), slw(x["k"]), slw(x["v"]), slw(x["beta"]), s0,
-                            n_threads=n_threads, g=gate, n_sub=w.nh)
-    return time.perf_counter() - t0, min(n_threads, w.H)
+    res = oracle.token_recurrence(sl(x["q"]), slw(x["k"]), slw(x["v"]), slw(x["beta"]), s0,
+                                  out_dtype=torch.float32, n_threads=n_threads, g=gate,
+                                  n_sub=w.nh)
+    dt = time.perf_counter() - t0
+    if outputs:
+        return dt, min(n_threads, w.H), res[0]
+    return dt, min(n_threads, w.H)
+
+
+def cpu_sample_tokens(w: wl.Workload) -> int:
+    """Tokens of one batch row that the CPU baseline runs the oracle on: the whole
+    row up to 2^21 token-heads (about 10-20 s of float64 work on 8-16 cores)."""
+    if w.seqlens is not None:
+        return min(w.T, 4096)
+    return max(CHUNK, min(w.T, (1 << 21) // (w.H * w.nh)))
 
 
 def run_reference(args, w: wl.Workload):
@@ -410,16 +428,30 @@ def run_b200(args, w: wl.Workload):
                "pipelined": "upload / call / download on three streams, two buffer sets"}
 
     cpu = None
+    parity = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        sample = w.T if w.seqlens is None else min(w.T, 4096)
-        rows = w.B if w.seqlens is None else 1
+        sample = cpu_sample_tokens(w)
+        dense = w.seqlens is None
+        rows = min(w.B, max(1, (1 << 21) // (sample * w.H * w.nh))) if dense else 1
         total_s, threads = 0.0, 1
+        err, scale = 0.0, 0.0
+        out_h = out.float().cpu() if dense else None
         for b in range(rows):
-            dt, threads = time_oracle(x, w, sample, b)
+            dt, threads, ref_o = time_oracle(x, w, sample, b, outputs=True)
             total_s += dt
+            if dense:
+                # causal: the timed call's outputs on this prefix equal the oracle's on it
+                got = out_h[b:b + 1, :sample].double()
+                err = max(err, (got - ref_o.double()).abs().max().item())
+                scale = max(scale, ref_o.abs().max().item())
         cpu = {"value": rows * sample / total_s, "unit": "tokens/s", "cores": threads,
                "kind": "oracle",
                "sample": f"{rows} x {sample} tokens x {w.H} heads (float64 token recurrence)"}
+        if dense:
+            parity = {"out_rel_err": err / (scale if scale > 0 else 1.0),
+                      "bar": 1e-2 if w.dtype == torch.bfloat16 else 1e-4,
+                      "sample": f"outputs of the timed call on {rows} x {sample} tokens x {w.H} "
+                                "heads against the float64 oracle on the same prefix"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
@@ -438,6 +470,7 @@ def run_b200(args, w: wl.Workload):
         "clocks": clk.summary(),
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "parity": parity,
         "gpu_launches": launches_per_step * args.steps,
     }
     if rank == 0:
@@ -453,7 +486,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--config", default="layer_1p3b", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--config", default="ctx_1m", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=128,

@@ -7,9 +7,11 @@ draws synthetic inputs (``workloads``).
 """
 from ._lib import (DeltaNetError, chunk_state_rows, deltanet_fwd,  # noqa: F401
                    deltanet_fwd_noalloc, deltanet_fwd_states, gated_deltanet_fwd, gated_deltaproduct_fwd, get_error, last_launches,
-                   last_schedule, load, release_workspace, set_kernel_events, status_string)
+                   last_schedule, load, release_workspace, set_kernel_events, status_string,
+                   test_set_wait)
 
 __all__ = ["deltanet_fwd", "gated_deltanet_fwd", "gated_deltaproduct_fwd",
            "deltanet_fwd_states", "chunk_state_rows",
            "deltanet_fwd_noalloc", "get_error", "release_workspace", "last_schedule",
-           "last_launches", "set_kernel_events", "status_string", "DeltaNetError", "load"]
+           "last_launches", "set_kernel_events", "status_string", "test_set_wait",
+           "DeltaNetError", "load"]

@@ -25,7 +25,8 @@ EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "gated_deltanet_fwd", "gated_delt
             "gated_deltaproduct_fwd", "gated_deltaproduct_fwd_ex", "deltanet_fwd_states",
             "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
-            "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events")
+            "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events",
+            "deltanet_test_set_wait")
 
 
 class DnTensor(ctypes.Structure):
@@ -93,6 +94,8 @@ def load(path: Optional[str] = None):
         lib.deltanet_last_launches.argtypes = []
         lib.deltanet_set_kernel_events.restype = None
         lib.deltanet_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        lib.deltanet_test_set_wait.restype = None
+        lib.deltanet_test_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_int]
         lib.deltanet_last_schedule.restype = None
         lib.deltanet_last_schedule.argtypes = [ctypes.POINTER(ctypes.c_int),
                                                ctypes.POINTER(ctypes.c_int)]
@@ -315,6 +318,15 @@ def deltanet_fwd_noalloc(q, k, v, beta, initial_state=None, chunk_size: int = 64
 def get_error(stream=None, device=None) -> int:
     """Synchronise the stream and return (and clear) its device-side error flag."""
     return load().deltanet_get_error(_stream_handle(device, stream))
+
+
+def test_set_wait(wait_ns: int = 0, stall_chunk: int = 0) -> None:
+    """Test hook of the bounded device waits for the following calls on this
+    thread: their time-out (0: the default 2 s) and, with stall_chunk > 0, a
+    wait at chunk stall_chunk - 1 of every run that nothing completes
+    (deltanet_test_set_wait in include/deltanet.h).  test_set_wait() restores
+    normal calls."""
+    load().deltanet_test_set_wait(int(wait_ns), int(stall_chunk))
 
 
 def release_workspace() -> None:

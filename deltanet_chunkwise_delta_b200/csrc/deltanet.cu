@@ -22,9 +22,18 @@
 
 using namespace dn;
 
+// Shared with deltanet_noalloc.cu (not exported): this thread's bounded-wait settings
+// for the next calls, and the no-alloc scratch's error word of a device (read and
+// cleared; 0 when that entry point never ran on the device).
+__attribute__((visibility("hidden"))) void dn_wait_settings(unsigned long long* wait_ns, int* stall_chunk);
+__attribute__((visibility("hidden"))) int dn_noalloc_take_error(int dev, int* word);
+
 namespace {
 
 thread_local int g_last_G = 0, g_last_s = 0, g_last_launches = 0;
+// deltanet_test_set_wait: time-out of the bounded device waits (0: 2 s) and the test stall
+thread_local unsigned long long g_wait_ns = 0;
+thread_local int g_stall_chunk = 0;
 thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
 
 struct StreamWs {
@@ -539,6 +548,8 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
 
     Params p;
     std::memset(&p, 0, sizeof p);
+    p.wait_ns = g_wait_ns;
+    p.stall_chunk = g_stall_chunk;
     p.q = q->data; p.k = k->data; p.v = v->data; p.o = out->data;
     p.beta = static_cast<const float*>(beta->data);
     p.s0 = s0 && numel(s0) ? static_cast<const float*>(s0->data) : nullptr;
@@ -658,20 +669,39 @@ dn_status deltanet_get_error(void* stream_ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DN_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return DN_ERR_CUDA;
+    // the no-alloc entry point's error word (one per device), then this stream's flag
+    int h = 0;
+    if (dn_noalloc_take_error(dev, &h) != 0) return DN_ERR_CUDA;
     int* flag = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_ws.find(std::make_pair(dev, stream));
-        if (it == g_ws.end() || !it->second.flag) return DN_OK;
-        flag = it->second.flag;
+        if (it != g_ws.end()) flag = it->second.flag;
     }
-    int h = 0;
-    if (cudaMemcpy(&h, flag, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DN_ERR_CUDA;
-    if (h != 0 && cudaMemset(flag, 0, sizeof h) != cudaSuccess) return DN_ERR_CUDA;
+    if (flag) {
+        int f = 0;
+        if (cudaMemcpy(&f, flag, sizeof f, cudaMemcpyDeviceToHost) != cudaSuccess) return DN_ERR_CUDA;
+        if (f != 0 && cudaMemset(flag, 0, sizeof f) != cudaSuccess) return DN_ERR_CUDA;
+        if (h == 0) h = f;
+    }
     if (h == kErrSeqlens) return DN_ERR_SEQLENS;
     if (h == kErrTimeout) return DN_ERR_TIMEOUT;
     return DN_OK;
 }
+
+void deltanet_test_set_wait(unsigned long long wait_ns, int stall_chunk) {
+    g_wait_ns = wait_ns;
+    g_stall_chunk = stall_chunk > 0 ? stall_chunk : 0;
+}
+
+}  // extern "C"
+
+void dn_wait_settings(unsigned long long* wait_ns, int* stall_chunk) {
+    *wait_ns = g_wait_ns;
+    *stall_chunk = g_stall_chunk;
+}
+
+extern "C" {
 
 void deltanet_release_workspace(void) {
     std::lock_guard<std::mutex> lk(g_mu);

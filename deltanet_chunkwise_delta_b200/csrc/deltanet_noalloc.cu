@@ -21,6 +21,11 @@
 // make that first call before any stream capture.  All calls share the one
 // array and it keeps the last call's contents: calls that overlap on the GPU
 // (on different streams, or on different host threads) race on it.
+//
+// Device-side errors (a bounded wait that gave up) go to the error word at the
+// head of the array.  deltanet_get_error(stream) reads and clears it, after
+// synchronising `stream`: pass the stream of the no-alloc call.  Each call
+// clears the word when it starts.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -33,6 +38,9 @@
 #include "dn_common.cuh"
 #include "dn_prep.cuh"
 #include "dn_tc.cuh"
+
+// From deltanet.cu: this host thread's bounded-wait settings (deltanet_test_set_wait).
+__attribute__((visibility("hidden"))) void dn_wait_settings(unsigned long long* wait_ns, int* stall_chunk);
 
 namespace {
 
@@ -112,6 +120,28 @@ bool na_token_ok(const dn_tensor* t, int64_t B, int64_t T, int64_t H) {
     return true;
 }
 
+// Byte span [lo, hi) of a strided view (non-negative strides), and the overlap test
+// deltanet_fwd applies to its outputs against its inputs and each other.
+void na_span(const dn_tensor* t, uintptr_t& lo, uintptr_t& hi) {
+    lo = hi = 0;
+    if (!t || !t->data) return;
+    int64_t last = 0;
+    for (int i = 0; i < t->ndim; ++i) {
+        if (t->shape[i] == 0) return;
+        last += (t->shape[i] - 1) * t->stride[i];
+    }
+    const int64_t es = t->dtype == DN_BF16 ? 2 : 4;
+    lo = reinterpret_cast<uintptr_t>(t->data);
+    hi = lo + static_cast<uintptr_t>((last + 1) * es);
+}
+bool na_overlap(const dn_tensor* a, const dn_tensor* b) {
+    uintptr_t a0, a1, b0, b1;
+    na_span(a, a0, a1);
+    na_span(b, b0, b1);
+    if (a0 == a1 || b0 == b1) return false;
+    return a0 < b1 && b0 < a1;
+}
+
 bool na_state_ok(const dn_tensor* t, int64_t N, int64_t H) {
     if (!t) return true;
     return t->ndim == 4 && t->dtype == DN_F32 && t->shape[0] == N && t->shape[1] == H &&
@@ -140,6 +170,14 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
         beta->stride[2] < 0)
         return DN_ERR_INVALID_ARG;
     if (!na_state_ok(initial_state, B, H) || !na_state_ok(final_state, B, H)) return DN_ERR_INVALID_ARG;
+    // the same aliasing rules as deltanet_fwd: no output overlaps an input or the other output
+    const dn_tensor* ins[5] = {q, k, v, beta, initial_state};
+    for (const dn_tensor* o : {static_cast<const dn_tensor*>(out), static_cast<const dn_tensor*>(final_state)}) {
+        if (!o) continue;
+        for (const dn_tensor* in : ins)
+            if (in && na_overlap(o, in)) return DN_ERR_ALIAS;
+    }
+    if (final_state && na_overlap(out, final_state)) return DN_ERR_ALIAS;
     const int64_t n_c = (T + dn::kChunk - 1) / dn::kChunk;
     if (B * n_c * H > kNoAllocMaxUnits) return DN_ERR_WORKSPACE;
 
@@ -168,6 +206,7 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     if (initial_state) { p.s0_sn = initial_state->stride[0]; p.s0_sh = initial_state->stride[1]; }
     if (final_state) { p.sT_sn = final_state->stride[0]; p.sT_sh = final_state->stride[1]; }
     p.err = reinterpret_cast<int*>(scratch);
+    dn_wait_settings(&p.wait_ns, &p.stall_chunk);
     p.wsT = scratch + kNoAllocFlagBytes;
     dn::Sched& sc = p.sched;
     sc.list = 0;
@@ -204,3 +243,22 @@ extern "C" int dn_trace_copy_prep_na(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, dn::g_dn_trace_prep, sizeof(dn::g_dn_trace_prep)) == cudaSuccess ? 0 : 1;
 }
 #endif
+
+// For deltanet_get_error: the error word of device `dev`'s scratch, read and cleared
+// (0 when the no-alloc entry point has not run on that device).  Returns nonzero on a
+// CUDA error.  The caller has synchronised the stream of the call that wrote it.
+__attribute__((visibility("hidden"))) int dn_noalloc_take_error(int dev, int* word) {
+    *word = 0;
+    unsigned char* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_na_mu);
+        auto it = g_na_scratch.find(dev);
+        if (it == g_na_scratch.end()) return 0;
+        scratch = it->second;
+    }
+    int h = 0;
+    if (cudaMemcpy(&h, scratch, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return 1;
+    if (h != 0 && cudaMemset(scratch, 0, sizeof h) != cudaSuccess) return 1;
+    *word = h;
+    return 0;
+}

@@ -592,7 +592,8 @@ __global__ void __launch_bounds__(2 * DK) k_scan(const __grid_constant__ CUtenso
     auto Pm = [&](int b) { return smem + b * kPBytes; };    // DK/32 swizzled boxes of DK rows x 32 columns
     float* St = reinterpret_cast<float*>(smem + 2 * kPBytes);  // COLS x SLD
     uint64_t* bars = reinterpret_cast<uint64_t*>(St + COLS * SLD);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2);
+    sm100::WaitCtl* ctl = reinterpret_cast<sm100::WaitCtl*>(bars + 2);
+    volatile int* abort_flag = &ctl->abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
     const int ra = 16 * warp + gq;              // fragment rows ra, ra + 8
     const int c0 = blockIdx.y * COLS;
@@ -600,7 +601,7 @@ __global__ void __launch_bounds__(2 * DK) k_scan(const __grid_constant__ CUtenso
     if (tid == 0) {
         sm100::mbar_init(&bars[0], 1);
         sm100::mbar_init(&bars[1], 1);
-        *abort_flag = 0;
+        sm100::wait_ctl_init(ctl, p.wait_ns);
         sm100::mbar_fence_init();
     }
     __syncthreads();
@@ -713,7 +714,7 @@ __global__ void __launch_bounds__(2 * DK) k_scan(const __grid_constant__ CUtenso
     if (tid == 0) {
         volatile int drain = 0;
         for (int b = 0; b < 2; ++b)
-            if ((pending >> b) & 1u) sm100::mbar_wait(&bars[b], (phase >> b) & 1u, &drain, 200000000ull);
+            if ((pending >> b) & 1u) sm100::mbar_wait(&bars[b], (phase >> b) & 1u, &drain, sm100::kDrainWaitNs);
         if (*abort_flag) atomicExch(p.err, kErrTimeout);
     }
 }

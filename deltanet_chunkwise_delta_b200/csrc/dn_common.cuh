@@ -91,6 +91,12 @@ struct Params {
     float* wsS;          // [slots][d_k][d_v] start states of segments 1..G-1
     uint8_t* wsT;        // [chunks * H] UT factors T (bf16 64 x 64, 128-byte swizzled rows)
     int* err;            // device error flag
+    // Bounded waits: the time after which a wait gives up (0: 2 s).  stall_chunk > 0 makes
+    // the tensor-core boundary kernel's chain issuer wait, at chunk stall_chunk - 1 of each
+    // run, on a barrier that nothing completes, so that the time-out path (give up, drain,
+    // report DN_ERR_TIMEOUT) can be tested with no fault; 0 in normal calls.
+    unsigned long long wait_ns;
+    int stall_chunk;
     Sched sched;
 };
 

@@ -65,9 +65,9 @@ struct PrepSmem {
     static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N; before them the P tile
     static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 5 staging blocks of the off-diagonal solve
     static constexpr int OFF_BETA = 32768;                        // 2 x 64 step sizes
-    static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE
-    static constexpr int OFF_MISC = OFF_BAR + 16;                 // TMEM address, abort flag
-    static constexpr int USED = OFF_MISC + 16;
+    static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE, DRAIN
+    static constexpr int OFF_MISC = OFF_BAR + 24;                 // TMEM address, then the WaitCtl at + 8
+    static constexpr int USED = OFF_MISC + 24;
     static constexpr int TOTAL = USED + 1024;                     // slack for 1024-byte alignment
 };
 static_assert(PrepSmem::OFF_X + 5 * kBlkFloats * 4 <= PrepSmem::OFF_BETA, "solve blocks fit the q/k region");
@@ -133,9 +133,10 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
     float* Ablk = reinterpret_cast<float*>(smem + L::OFF_A);
     float* Nblk = reinterpret_cast<float*>(smem + L::OFF_N);
     float* Xs = reinterpret_cast<float*>(smem + L::OFF_X);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);  // [0] FULL, [1] GDONE
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);  // [0] FULL, [1] GDONE, [2] DRAIN
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
+    sm100::WaitCtl* ctl = reinterpret_cast<sm100::WaitCtl*>(smem + L::OFF_MISC + 8);
+    volatile int* abort_flag = &ctl->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.sched.H;
@@ -145,7 +146,8 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
     if (tid == 0) {
         sm100::mbar_init(&bars[0], 1);
         sm100::mbar_init(&bars[1], 1);
-        *abort_flag = 0;
+        sm100::mbar_init(&bars[2], 1);
+        sm100::wait_ctl_init(ctl, p.wait_ns);
         sm100::mbar_fence_init();
     }
     if (warp == 0) {
@@ -412,10 +414,13 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
     // a load issued for a unit this CTA then gave up on must land before exit
     if (in_flight) {
         volatile int drain = 0;
-        sm100::mbar_wait(&bars[0], it_ & 1, &drain, 200000000ull);
+        sm100::mbar_wait(&bars[0], it_ & 1, &drain, sm100::kDrainWaitNs);
     }
     cp_async_wait<0>();
-    if (tid == 0) sm100::bulk_wait0();  // the tile copies are complete
+    if (tid == 0) {
+        sm100::bulk_wait0();             // the tile copies are complete
+        sm100::umma_drain(&bars[2]);     // and the last Gram product (a wait for it may have given up)
+    }
     sm100::tc_fence_before();
     __syncthreads();
     if (warp == 0) {

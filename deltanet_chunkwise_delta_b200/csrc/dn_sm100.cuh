@@ -58,11 +58,29 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
     return ok != 0;
 }
 
-// Waits for the phase with the given parity.  Gives up after `limit_ns` (or
-// as soon as another thread has raised *abort) and returns false; the caller
-// then skips the rest of its work so that the CTA can drain and exit.
+// A CTA's abort state for its bounded waits: the flag that a wait which gave up
+// raises (every other wait of the CTA then gives up at once), followed by the
+// time after which a wait gives up.  Kernels keep one in shared memory and pass
+// &ctl->abort to the waits below.
+struct WaitCtl {
+    int abort;
+    int pad;
+    unsigned long long limit_ns;
+};
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+__device__ __forceinline__ void wait_ctl_init(WaitCtl* c, unsigned long long limit_ns) {
+    c->abort = 0;
+    c->limit_ns = limit_ns ? limit_ns : kDefaultWaitNs;
+}
+
+// Waits for the phase with the given parity.  Gives up after `limit_ns` (0: the
+// limit of the WaitCtl whose flag `abort` is), or as soon as another thread has
+// raised *abort, and returns false; the caller then skips the rest of its work
+// so that the CTA can drain and exit.  Drain waits pass a local flag and an
+// explicit limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns = 2000000000ull) {
+                                          uint64_t limit_ns = 0) {
+    if (limit_ns == 0) limit_ns = reinterpret_cast<volatile WaitCtl*>(abort)->limit_ns;
     // spin first (the common short waits on the state chain), then sleep-wait
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
@@ -76,6 +94,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             return false;
         }
     }
+}
+
+// Drain wait: at most 200 ms and independent of the abort flag, for copies or
+// products already issued, before the CTA exits or frees what they use.
+constexpr unsigned long long kDrainWaitNs = 200000000ull;
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+    volatile int local = 0;
+    mbar_wait(bar, parity, &local, kDrainWaitNs);
 }
 
 // Waits for two phases.  Both barriers are tested back to back first, so the
@@ -186,6 +212,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             saddr(bar))
         : "memory");
+}
+// Waits until every tensor-core product this thread has issued is complete: a
+// commit to `bar` (a barrier of count 1 used for nothing else, phase 0) and a
+// drain wait on it.  Issuers call it once before the CTA frees its tensor
+// memory, so that no product in flight writes freed columns or reads shared
+// memory after the CTA has left, also when a bounded wait gave up.
+__device__ __forceinline__ void umma_drain(uint64_t* bar) {
+    umma_commit(bar);
+    mbar_drain(bar, 0);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.

@@ -70,7 +70,7 @@ constexpr int B_STAGE = 24576, B_T = 16384;
 constexpr int OFF_PB = OFF_B + NB * B_STAGE;   // P rows, 2 x 8 KB
 constexpr int OFF_OB = OFF_PB + 2 * 8192;      // O staging
 constexpr int OFF_BAR = OFF_OB + 16384;
-constexpr int NBAR = 31;
+constexpr int NBAR = 34;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_USED = OFF_MISC + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -108,8 +108,10 @@ enum : int {
     B_OBFREE = 25,   // O staging buffer released by the chunk's store
     B_GAP2 = 26,     // +2: chain issuer: chunk's S^T update issued (one per chunk parity)
     B_UFULL = 28,    // U^T of the chunk ready in tensor memory
+    B_DRAIN = 31,    // +2: drain of the chain issuer's / the parallel issuer's products
+    B_STALL = 33,    // never completed: the wait of a test stall (Params::stall_chunk)
 };
-static_assert(B_OFREE + 1 < NBAR, "barrier count");
+static_assert(B_STALL < NBAR, "barrier count");
 
 // Optional timeline of CTA 0 (build with -DDN_TRACE): globaltimer stamps per
 // chunk and pipeline event, read back with dn_trace_copy().
@@ -178,7 +180,8 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
+    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + OFF_MISC + 8);
+    volatile int* abort_flag = &ctl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -208,7 +211,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         mbar_init(&bars[B_OFREE + 1], 4);
         mbar_init(&bars[B_OSTAGED], 4);
         mbar_init(&bars[B_OBFREE], 4);
-        *abort_flag = 0;
+        mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN + 1], 1);
+        mbar_init(&bars[B_STALL], 1);
+        wait_ctl_init(ctl, p.wait_ns);
         mbar_fence_init();
     }
     if (warp == kMmaWarp) {
@@ -253,7 +259,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             // the last loads issued must have landed before the CTA may exit (even after an abort)
             volatile int drain = 0;
             for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
-                mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, 200000000ull);
+                mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, kDrainWaitNs);
         }
     } else if (warp == kTmaBWarp) {
         // ------------------------------------------------------------ ring B: v, T
@@ -275,7 +281,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             }
             volatile int drain = 0;
             for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
-                mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, 200000000ull);
+                mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, kDrainWaitNs);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ state-chain products
@@ -294,6 +300,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int sa = r % NA, s = r & 1;
                 const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
                 DN_TR(true, r, 0);
+                if (r + 1 == p.stall_chunk && !mbar_wait(&bars[B_STALL], 0, abort_flag)) break;
                 const bool ready = mbar_wait4(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1,
                                               &bars[B_OFREE + s], (r >> 1) & 1, abort_flag);
                 if (!ready) break;
@@ -335,6 +342,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 umma_commit(&bars[B_EMPTYA + sa]);
                 DN_TR(true, r, 11);
             }
+            umma_drain(&bars[B_DRAIN]);
         }
     } else if (warp == kParMmaWarp) {
         // ------------------------------------------------------------ chunk-parallel products
@@ -396,6 +404,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 issue_u(r + 1);
                 DN_TR(true, r, 4);
             }
+            umma_drain(&bars[B_DRAIN + 1]);
         }
     } else if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ chunk-parallel epilogue
@@ -513,7 +522,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         if (lane == 0) {
             volatile int drain = 0;
             for (int c = p_issued - 2 < 0 ? 0 : p_issued - 2; c < p_issued; ++c)
-                mbar_wait(&bars[B_PFULL + (c & 1)], (c >> 1) & 1, &drain, 200000000ull);
+                mbar_wait(&bars[B_PFULL + (c & 1)], (c >> 1) & 1, &drain, kDrainWaitNs);
         }
         if (q == 0 && lane == 0) bulk_wait0();
     } else if (warp < 8) {

@@ -70,7 +70,7 @@ constexpr int OFF_Z = OFF_B + NB * B_STAGE;
 constexpr int Z_BYTES = 16384;
 constexpr int OFF_SP = OFF_Z + 2 * Z_BYTES;
 constexpr int OFF_BAR = OFF_SP + 32768;
-constexpr int NBAR = 26;
+constexpr int NBAR = 27;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM_USED = OFF_MISC + 64;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -112,8 +112,9 @@ enum : int {
     B_SBF = 19,     // +2: bf16 S_x^T written
     B_GAP1 = 21,    // +2: the chunk's first products are issued (one per chunk parity)
     B_GAP2 = 23,    // +2: chain H's state update is issued (one per chunk parity)
+    B_DRAIN = 25,   // +2: drain of the chain issuer's / the parallel issuer's products
 };
-static_assert(B_GAP2 + 2 <= NBAR, "barrier count");
+static_assert(B_DRAIN + 2 <= NBAR, "barrier count");
 
 // Optional timeline of CTA 1 (the first two-chain item of a split chain; build
 // with -DDN_TRACE): globaltimer stamps per chunk and pipeline event.
@@ -143,7 +144,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
+    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + OFF_MISC + 8);
+    volatile int* abort_flag = &ctl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -165,7 +167,9 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
         mbar_init(&bars[B_WUFULL], 1);
         mbar_init(&bars[B_WFULL], 4);
         mbar_init(&bars[B_UFULL], 1);
-        *abort_flag = 0;
+        mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN + 1], 1);
+        wait_ctl_init(ctl, p.wait_ns);
         mbar_fence_init();
     }
     if (warp == kMmaWarp) {
@@ -202,7 +206,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 // the last loads issued must have landed before the CTA may exit (even after an abort)
                 volatile int drain = 0;
                 for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
-                    mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, 200000000ull);
+                    mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, kDrainWaitNs);
             }
         } else if (warp == kTmaBWarp) {
             // ------------------------------------------------------------ ring B: v, T
@@ -222,7 +226,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 }
                 volatile int drain = 0;
                 for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
-                    mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, 200000000ull);
+                    mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, kDrainWaitNs);
             }
         } else if (warp == kMmaWarp) {
             // ------------------------------------------------------------ chain products
@@ -297,6 +301,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     // the chunk, complete before its -W rows were written)
                     umma_commit(&bars[B_EMPTYA + sa]);
                 }
+                umma_drain(&bars[B_DRAIN]);
             }
         } else if (warp == kParMmaWarp) {
             // ------------------------------------------------------------ chunk-parallel products
@@ -355,6 +360,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     tc_fence_after();
                     issue_u(r + 1);
                 }
+                umma_drain(&bars[B_DRAIN + 1]);
             }
         } else if (warp >= 8 && warp < 12) {
             // ------------------------------------------------------------ -W rows

@@ -230,8 +230,12 @@ dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, cons
  * bf16 q/k/v/out, d_k = d_v = 128, chunk_size 64, and
  * B * ceil(T / 64) * H <= 3072 (chunk, head) pairs; larger problems return
  * DN_ERR_WORKSPACE, other shapes or dtypes DN_ERR_UNSUPPORTED / _INVALID_ARG.
- * Outputs must not overlap inputs (not checked here).  Each (sequence, head)
- * runs as one run of chunks (no split across SMs).
+ * Aliasing as deltanet_fwd: an output that overlaps an input or the other
+ * output (final_state == initial_state included) returns DN_ERR_ALIAS.  Each
+ * (sequence, head) runs as one run of chunks (no split across SMs).
+ * Device-side errors (DN_ERR_TIMEOUT) go to the array's error word, which
+ * each call clears when it starts; deltanet_get_error(stream), called with
+ * the stream of the call, reads and clears it.
  * The first call on a device looks up the array's device address and sets
  * kernel attributes; make it before any stream capture.  All calls share the
  * array, which keeps the last call's contents, so calls that overlap on the
@@ -249,8 +253,25 @@ const char* deltanet_status_string(dn_status status);
  * deltanet_get_error -- synchronises `stream`, then returns and clears the
  * device-side error flag of the calls made on it (DN_OK, DN_ERR_SEQLENS or
  * DN_ERR_TIMEOUT), or DN_ERR_CUDA if the stream itself reports an error.
+ * It also reads and clears the error word of deltanet_fwd_noalloc's scratch
+ * on the current device (one per device, shared by all streams).
  */
 dn_status deltanet_get_error(void* stream);
+
+/*
+ * deltanet_test_set_wait -- test hook for the time-out path of the bounded
+ * device waits, for the calls made after it on this host thread.
+ * wait_ns: time after which a device wait gives up and the call reports
+ * DN_ERR_TIMEOUT through deltanet_get_error (0 restores the default, 2 s).
+ * stall_chunk > 0: in the tensor-core boundary kernel (bf16, d_k = d_v = 128),
+ * the thread that issues the state-chain products waits, at chunk
+ * stall_chunk - 1 of every run, on a barrier that nothing completes, so that
+ * the wait runs out: the kernel then gives up, waits for its copies and
+ * products in flight, frees its tensor memory, exits and reports the
+ * time-out.  The outputs of such a call are unspecified.  0 (the default):
+ * no stall.  deltanet_test_set_wait(0, 0) restores normal calls.
+ */
+void deltanet_test_set_wait(unsigned long long wait_ns, int stall_chunk);
 
 /* Frees every cached workspace (synchronises the device first). */
 void deltanet_release_workspace(void);

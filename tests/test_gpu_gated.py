@@ -37,7 +37,7 @@ def run_gpu(x, seg_chunks=0):
     return out.cpu(), fs.cpu()
 
 
-def check(w, x, seg_chunks=0, heads=None):
+def check(w, x, seg_chunks=0, heads=None, log=None, name=None):
     out, fs = run_gpu(x, seg_chunks)
     ref_o, ref_s = oracle.token_recurrence(x["q"], x["k"], x["v"], x["beta"],
                                            x["initial_state"], x["cu_seqlens"], heads=heads,
@@ -46,6 +46,8 @@ def check(w, x, seg_chunks=0, heads=None):
     eo = rel_err(out[:, :, h0:h1], ref_o[:, :, h0:h1])
     es = rel_err(fs[:, h0:h1], ref_s[:, h0:h1])
     tol = TOL[w.dtype]
+    if log is not None:
+        log.append((name or w.name, eo, es, tol))
     assert eo <= tol and es <= tol, (eo, es)
     return eo, es
 
@@ -157,12 +159,12 @@ def test_gated_strided_gate():
 # ---- full-size gated workloads: every output of a subset of heads ---------------
 
 @pytest.mark.slow
-def test_config_gdn_1p3b():
+def test_config_gdn_1p3b(margins):
     w = wl.WORKLOADS["gdn_1p3b"]
-    check(w, wl.generate(w, 0), heads=(0, 4))
+    check(w, wl.generate(w, 0), heads=(0, 4), log=margins, name="gdn_1p3b (heads 0-3)")
 
 
 @pytest.mark.slow
-def test_config_gdn_65k():
+def test_config_gdn_65k(margins):
     w = wl.WORKLOADS["gdn_65k"]
-    check(w, wl.generate(w, 0), heads=(0, 2))
+    check(w, wl.generate(w, 0), heads=(0, 2), log=margins, name="gdn_65k (heads 0-1)")

@@ -40,7 +40,7 @@ def run_gpu(x, seg_chunks=0, with_state=True):
     return out.cpu(), (fs.cpu() if fs is not None else None)
 
 
-def check(w, x, seg_chunks=0, heads=None):
+def check(w, x, seg_chunks=0, heads=None, log=None, name=None):
     out, fs = run_gpu(x, seg_chunks)
     ref_o, ref_s = oracle.token_recurrence(x["q"], x["k"], x["v"], x["beta"],
                                            x["initial_state"], x["cu_seqlens"], heads=heads)
@@ -48,6 +48,8 @@ def check(w, x, seg_chunks=0, heads=None):
     eo = rel_err(out[:, :, h0:h1], ref_o[:, :, h0:h1])
     es = rel_err(fs[:, h0:h1], ref_s[:, h0:h1])
     tol = TOL[w.dtype]
+    if log is not None:
+        log.append((name or w.name, eo, es, tol))
     assert eo <= tol and es <= tol, (eo, es)
     return eo, es
 
@@ -59,9 +61,9 @@ def _lib():
     dn.load()
 
 
-def test_tiny_fp32_config():
+def test_tiny_fp32_config(margins):
     w = wl.WORKLOADS["tiny_fp32"]
-    check(w, wl.generate(w, 0))
+    check(w, wl.generate(w, 0), log=margins)
 
 
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
@@ -187,29 +189,31 @@ def test_schedule_of_config_shapes():
 # ---- full-size configs: every output of a subset of heads ------------------
 
 @pytest.mark.slow
-def test_config_layer_1p3b():
+def test_config_layer_1p3b(margins):
     w = wl.WORKLOADS["layer_1p3b"]
-    check(w, wl.generate(w, 0), heads=(0, 4))
+    check(w, wl.generate(w, 0), heads=(0, 4), log=margins, name="layer_1p3b (heads 0-3)")
 
 
 @pytest.mark.slow
-def test_config_long_65k():
+def test_config_long_65k(margins):
     w = wl.WORKLOADS["long_65k"]
-    check(w, wl.generate(w, 0), heads=(0, 2))
+    check(w, wl.generate(w, 0), heads=(0, 2), log=margins, name="long_65k (heads 0-1)")
 
 
 @pytest.mark.slow
-def test_config_varlen_32():
+def test_config_varlen_32(margins):
     w = wl.WORKLOADS["varlen_32"]
-    check(w, wl.generate(w, 0), heads=(0, 2))
+    check(w, wl.generate(w, 0), heads=(0, 2), log=margins, name="varlen_32 (heads 0-1)")
 
 
 @pytest.mark.slow
-def test_config_ctx_1m():
+def test_config_ctx_1m(margins):
     w = wl.WORKLOADS["ctx_1m"]
     x = wl.generate(w, 0)
     out, fs = run_gpu(x)
     ref_o, ref_s = oracle.token_recurrence(x["q"], x["k"], x["v"], x["beta"], None,
                                            heads=(0, 1), out_dtype=torch.float32)
-    assert rel_err(out[:, :, 0:1], ref_o[:, :, 0:1]) <= 1e-2
-    assert rel_err(fs[:, 0:1], ref_s[:, 0:1]) <= 1e-2
+    eo = rel_err(out[:, :, 0:1], ref_o[:, :, 0:1])
+    es = rel_err(fs[:, 0:1], ref_s[:, 0:1])
+    margins.append(("ctx_1m (head 0, 1048576 tokens)", eo, es, 1e-2))
+    assert eo <= 1e-2 and es <= 1e-2, (eo, es)
