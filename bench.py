@@ -295,7 +295,7 @@ def run_b200(args, w: wl.Workload):
     step()
     if dn.get_error(stream) != 0:
         raise RuntimeError("device reported an error")
-    G, s = dn.last_schedule()
+    G, s, s0 = dn.last_schedule(with_first=True)
     launches_per_step = dn.last_launches()
     for _ in range(args.warmup):
         step()
@@ -341,7 +341,7 @@ def run_b200(args, w: wl.Workload):
         # the summary pass; the timed launch covers runs 1..G-1 (q, k, v, o of their
         # tokens and the final state)
         es = 2
-        th_b = w.B * (w.T - s * CHUNK) * w.H
+        th_b = w.B * (w.T - s0 * CHUNK) * w.H
         kernel_bytes = float(th_b * es * (2 * w.dk + 2 * w.dv) + w.n_seq * w.H * w.dk * w.dv * 4)
     achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9
     tc_kernel = tc_path
@@ -460,6 +460,7 @@ def run_b200(args, w: wl.Workload):
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
                    "chunk": CHUNK, "segments_per_chain": G, "chunks_per_segment": s,
+                   "chunks_first_segment": s0,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}",
                    "variant": (f"gated delta product, n_h = {w.nh}" if w.nh > 1 else
                                "gated DeltaNet" if w.gated else "DeltaNet")},

@@ -97,7 +97,7 @@ def load(path: Optional[str] = None):
         lib.deltanet_test_set_wait.restype = None
         lib.deltanet_test_set_wait.argtypes = [ctypes.c_ulonglong, ctypes.c_int]
         lib.deltanet_last_schedule.restype = None
-        lib.deltanet_last_schedule.argtypes = [ctypes.POINTER(ctypes.c_int),
+        lib.deltanet_last_schedule.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
                                                ctypes.POINTER(ctypes.c_int)]
         _lib = lib
         return lib
@@ -345,7 +345,9 @@ def set_kernel_events(start=None, stop=None) -> None:
                                       stop.cuda_event if stop is not None else None)
 
 
-def last_schedule():
-    g, s = ctypes.c_int(0), ctypes.c_int(0)
-    load().deltanet_last_schedule(ctypes.byref(g), ctypes.byref(s))
-    return g.value, s.value
+def last_schedule(with_first: bool = False):
+    """(segments per chain, chunks per segment) of the last dense call on this
+    thread; with ``with_first`` also the chunks of the first segment."""
+    g, s, s0 = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    load().deltanet_last_schedule(ctypes.byref(g), ctypes.byref(s), ctypes.byref(s0))
+    return (g.value, s.value, s0.value) if with_first else (g.value, s.value)

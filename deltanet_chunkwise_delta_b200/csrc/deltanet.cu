@@ -30,7 +30,7 @@ __attribute__((visibility("hidden"))) int dn_noalloc_take_error(int dev, int* wo
 
 namespace {
 
-thread_local int g_last_G = 0, g_last_s = 0, g_last_launches = 0;
+thread_local int g_last_G = 0, g_last_s = 0, g_last_s0 = 0, g_last_launches = 0;
 // deltanet_test_set_wait: time-out of the bounded device waits (0: 2 s) and the test stall
 thread_local unsigned long long g_wait_ns = 0;
 thread_local int g_stall_chunk = 0;
@@ -250,12 +250,12 @@ struct Dims {
 template <typename E, int DK, int DV, int STAGES, bool GATED>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
-    // bf16 DeltaNet with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels; Gated
-    // DeltaNet, the other shapes and calls that keep the chunk-start states on the mma.sync
-    // chain kernels (which hold the state in registers)
+    // bf16 DeltaNet with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels (with or
+    // without the chunk-start states); Gated DeltaNet and the other shapes on the mma.sync
+    // chain kernels
     constexpr bool kTcShape =
         !GATED && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
-    const bool use_tc = kTcShape && !p.cs;
+    const bool use_tc = kTcShape;
     using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED>;
@@ -297,18 +297,24 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
     const int64_t chains = d.N * d.H;
     CostModel model;
+    if (use_tc) model.a = kTcSummaryCost;
     size_t bytes = 0;
     int64_t slots = 0, nC = 0, nA = 0, nScan = 0;
-    int G = 1, s = 1;
+    int G = 1, s = 1, s0 = 0;
     bool e_in_c = false;
     if (!d.varlen) {
         if (forced_s > 0) {
-            s = forced_s;
+            s = forced_s & 0xffff;
+            s0 = (forced_s >> 16) & 0x7fff;
+            if (s < 1 || s0 > s) return DN_ERR_INVALID_ARG;
         } else {
             SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, use_tc);
             s = ch.s;
+            s0 = ch.s0;
         }
-        G = n_c_max > 0 ? (int)((n_c_max + s - 1) / s) : 1;
+        // run 0 has s0 chunks (s when s0 == 0), the others s
+        const int64_t first = s0 > 0 ? s0 : s;
+        G = n_c_max > first ? (int)(1 + (n_c_max - first + s - 1) / s) : 1;
         slots = chains * (G - 1);
         if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
         nC = chains * G;
@@ -319,6 +325,8 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         nScan = G >= 2 ? chains : 0;
     } else {
         if (forced_s > 0) {
+            forced_s &= 0xffff;
+            if (forced_s < 1) return DN_ERR_INVALID_ARG;
             slots = d.H * ((n_c_max + d.N) / forced_s);
             if (slots > kMaxSlots) return DN_ERR_WORKSPACE;
         } else {
@@ -362,8 +370,10 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         sc.G = G;
         sc.e_in_c = e_in_c ? 1 : 0;
         sc.s = s;
+        sc.s0 = G >= 2 ? s0 : 0;
         g_last_G = G;
         g_last_s = s;
+        g_last_s0 = G >= 2 && s0 > 0 ? s0 : s;
     } else {
         sc.list = 1;
         sc.B = 1;
@@ -385,6 +395,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             reinterpret_cast<int*>(base + off_cum), ws.flag);
         g_last_G = -1;
         g_last_s = -1;
+        g_last_s0 = -1;
     }
     CUtensorMap tp;
     if ((st = make_p_map(&tp, p.wsP, slots * DK, DK)) != DN_OK) return st;
@@ -724,15 +735,16 @@ int dn_trace_copy(unsigned long long* host) {
 int dn_trace_copy_prep(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_dn_trace_prep, sizeof(g_dn_trace_prep)) == cudaSuccess ? 0 : 1;
 }
-int dn_trace_copy_scan(unsigned long long* host) {
-    return cudaMemcpyFromSymbol(host, g_dn_trace_scan, sizeof(g_dn_trace_scan)) == cudaSuccess ? 0 : 1;
-}
 int dn_trace_copy_sum(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, tcs::g_dn_trace_sum, sizeof(tcs::g_dn_trace_sum)) == cudaSuccess ? 0 : 1;
 }
+int dn_trace_copy_scan(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_dn_trace_scan, sizeof(g_dn_trace_scan)) == cudaSuccess ? 0 : 1;
+}
 #endif
 
-void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment) {
+void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment, int* chunks_first_segment) {
+    if (chunks_first_segment) *chunks_first_segment = g_last_s0;
     if (segments_per_chain) *segments_per_chain = g_last_G;
     if (chunks_per_segment) *chunks_per_segment = g_last_s;
 }

@@ -49,7 +49,8 @@ enum SegMode : int {
 struct Sched {
     int list;           // 0 = dense, 1 = list
     int B, T, H;        // dense shape
-    int n_chunks, G, s; // dense segmentation
+    int n_chunks, G, s; // dense segmentation: G runs of s chunks (run 0: s0, see below)
+    int s0;             // dense: chunks of run 0 (0: s); the last run takes the remainder
     int e_in_c;         // dense: run 0's end state comes from the boundary pass (no E items)
     int c_part;         // dense boundary items: 0 all runs, 1 run 0 only, 2 runs 1..G-1
     const Item* itemsC;     // list: boundary-pass items
@@ -108,12 +109,17 @@ __device__ __forceinline__ void dense_chain_item(const Sched& s, int chain, int 
     it.head = chain % s.H;
     it.G = s.G;
     it.g = g;
-    it.tok0 = g * s.s * kChunk;
-    int e = (g + 1) * s.s * kChunk;
-    it.tok1 = e < s.T ? e : s.T;
+    // run g covers chunks [c0, c1): run 0 the first s0, every later run s (the last one
+    // whatever remains)
+    const int s0 = s.s0 > 0 ? s.s0 : s.s;
+    const int c0 = g == 0 ? 0 : s0 + (g - 1) * s.s;
+    const int c1 = g == 0 ? s0 : s0 + g * s.s;
+    it.tok0 = c0 * kChunk;
+    const long long e = (long long)c1 * kChunk;
+    it.tok1 = e < s.T ? (int)e : s.T;
     if (g == s.G - 1) it.tok1 = s.T;
     it.slot = chain * (s.G - 1);
-    it.cbase = it.b * s.n_chunks + g * s.s;
+    it.cbase = it.b * s.n_chunks + c0;
 }
 
 __device__ __forceinline__ int count_C(const Sched& s) {

@@ -1,19 +1,24 @@
 // Segmentation of (sequence, head) chains into runs of chunks.
 //
-// A chain of n_c chunks is cut into G = ceil(n_c / s) runs of s chunks (the
-// last one shorter).  Run 0 starts from the true initial state; the others need
-// the maps (P_g, H_g) of every run before them ("Context Parallelism for
-// DeltaNet", section 3: the chunk update is affine in the incoming state, so
-// runs compose).  Work per call:
+// A chain of n_c chunks is cut into G runs: run 0 of s0 chunks, then runs of s
+// chunks (the last one possibly shorter).  Run 0 starts from the true initial
+// state; the others need the maps (P_g, H_g) of every run before them ("Context
+// Parallelism for DeltaNet", section 3: the chunk update is affine in the
+// incoming state, so runs compose).  Work per call:
 //   summary pass   run 0: end state; runs 1..G-2: H_g and P_g (one item each)
 //   segment scan   start states of runs 1..G-1
 //   boundary pass  every run from its start state: outputs, final state
-// The run length s minimises a simple model of the call's duration, with
-// costs per chunk relative to one boundary-pass chunk and one CTA per SM:
-//   dense input (equal runs):  c * s * waves(runs) + a * s * waves(summary items)
-//                              + scan * (G - 1),  waves(n) = ceil(n / SMs)
-//   packed input (unequal):    c * max(min(s, longest chain), chunk-heads / SMs)
-//                              + a * max(s, summary chunk-heads / SMs) + scan * (G_max - 1)
+// The run lengths minimise a simple model of the call's duration, with costs
+// per chunk relative to one boundary-pass chunk and one CTA per SM
+// (waves(n) = ceil(n / SMs)):
+//   dense, equal runs (s0 = s):     c * s * waves(runs) + a * s * waves(summary items)
+//                                   + scan * (G - 1)
+//   dense, run 0 on the boundary    phase 1, run 0 (c per chunk) next to the summary
+//   pass next to the summary        items (a per chunk): max(c * s0, a * s) * waves;
+//   pass (tensor-core path):        phase 2, runs 1..G-1: c * s * waves; + scan * (G - 1);
+//                                   s0 = (a / c) s, so that both parts of phase 1 end together
+//   packed input (unequal):         c * max(min(s, longest chain), chunk-heads / SMs)
+//                                   + a * max(s, summary chunk-heads / SMs) + scan * (G_max - 1)
 #pragma once
 
 #include "dn_common.cuh"
@@ -22,39 +27,59 @@ namespace dn {
 
 struct CostModel {
     float c = 1.0f;      // boundary pass, per chunk
-    float a = 1.25f;     // summary pass, per chunk (two chains, no output, no Q)
+    float a = 1.25f;     // summary pass, per chunk (mma.sync path: two chains, no output)
     float scan = 2.0f;   // one step of the segment scan
 };
+// Summary-pass chunk of the tensor-core path (two chains, k_tc_summary) relative to its
+// boundary-pass chunk (measured: 1.9 against 1.5 us per chunk).
+constexpr float kTcSummaryCost = 1.25f;
 
 struct SegChoice {
     int s;
     float cost;
+    int s0 = 0;          // chunks of run 0 (0: s)
 };
 
-// Cost of run length s for `chains` chains of equal length n_c (dense input).  With
-// e_in_c, run 0 of a split chain is computed once, by its boundary item, which runs
-// next to the summary items (so the summary phase has G - 1 items per chain, the
-// boundary phase after the scan G - 1 more).
+// Cost of equal runs of length s for `chains` chains of equal length n_c (dense input,
+// every run's end state from the summary pass).
 __host__ __device__ inline float dense_cost(const CostModel& m, int chains, int n_c, int s,
-                                            int slots, bool e_in_c = false) {
+                                            int slots) {
     const int G = n_c > 0 ? (n_c + s - 1) / s : 1;
-    const long long runs = (long long)chains * ((e_in_c && G >= 2) ? G - 1 : G);
+    const long long runs = (long long)chains * G;
     const long long summ = G >= 2 ? (long long)chains * (G - 1) : 0;
     const float wC = (float)((runs + slots - 1) / slots);
     const float wA = (float)((summ + slots - 1) / slots);
     return m.c * min(s, n_c) * wC + m.a * s * wA + m.scan * (G - 1);
 }
 
+// The run lengths for `chains` chains of n_c chunks.  With e_in_c, run 0 of a split
+// chain is computed once, by its boundary item, which runs next to the summary items
+// (G - 1 items per chain in each of the two phases).
 inline SegChoice choose_dense(const CostModel& m, int chains, int n_c, int slots,
                               int max_slots, bool e_in_c = false) {
-    SegChoice best{n_c > 0 ? n_c : 1, 3.0e38f};
     if (n_c <= 0) return {1, 0.f};
-    for (int G = 1; G <= 256 && G <= n_c; ++G) {
-        const int s = (n_c + G - 1) / G;
-        const int Gs = (n_c + s - 1) / s;
-        if ((long long)chains * (Gs - 1) > max_slots) break;
-        const float cst = dense_cost(m, chains, n_c, s, slots, e_in_c);
-        if (cst < best.cost) best = {s, cst};
+    const auto waves = [&](long long n) { return (float)((n + slots - 1) / slots); };
+    SegChoice best{n_c, m.c * n_c * waves(chains)};  // one run per chain
+    if (!e_in_c) {
+        for (int G = 2; G <= 256 && G <= n_c; ++G) {
+            const int s = (n_c + G - 1) / G;
+            const int Gs = (n_c + s - 1) / s;
+            if ((long long)chains * (Gs - 1) > max_slots) break;
+            const float cst = dense_cost(m, chains, n_c, s, slots);
+            if (cst < best.cost) best = {s, cst};
+        }
+        return best;
+    }
+    const float rho = fminf(1.f, m.a / m.c);
+    for (int G = 2; G <= 256 && G <= n_c; ++G) {
+        if ((long long)chains * (G - 1) > max_slots) break;
+        int s = (int)ceilf((float)n_c / ((float)(G - 1) + rho));
+        int s0 = n_c - (G - 1) * s;
+        if (s0 < 1) continue;
+        const float w = waves((long long)chains * (G - 1));
+        const float phase1 = fmaxf(m.c * s0, G >= 3 ? m.a * s : 0.f);
+        const float cst = phase1 * w + m.c * s * w + m.scan * (G - 1);
+        if (cst < best.cost) best = {s, cst, s0 < s ? s0 : 0};
     }
     return best;
 }

@@ -532,6 +532,16 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         const int wq = warp & 3, h = warp >> 2;
         const int d = 32 * wq + lane;  // d_v row of S^T, Z^T
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+        // the state entering chunk c of the run (for a backward pass): row = global chunk
+        // index; this thread's column d of key rows 64 h .. + 63 (a warp writes 128
+        // contiguous bytes of each row)
+        auto store_chunk_state = [&](int c, const uint32_t(&v)[64]) {
+            const int64_t row = (int64_t)it.cbase + c;
+            if (!p.cs || row >= p.cs_rows) return;
+            float* dst = p.cs + row * p.cs_sc + it.head * p.cs_sh + d;
+#pragma unroll
+            for (int cc = 0; cc < 64; ++cc) dst[(int64_t)(64 * h + cc) * D] = __uint_as_float(v[cc]);
+        };
         {
             uint32_t v[64];
 #pragma unroll
@@ -545,6 +555,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 if (x_out)
                     for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * h + c) * D + d] = __uint_as_float(v[c]);
             } else {
+                store_chunk_state(0, v);
                 tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
                 tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                 uint32_t pk[32];
@@ -597,6 +608,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                     for (int c = 0; c < 64; ++c)
                         x_out[(int64_t)(64 * h + c) * D + d] = __uint_as_float(v[c]);
                 }
+                if (r + 1 < nch) store_chunk_state(r + 1, v);
             }
         }
     }

@@ -90,12 +90,16 @@ dn_status deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* 
 
 /*
  * deltanet_fwd_ex -- deltanet_fwd with a scheduling override.
- * seg_chunks > 0 forces every sequence to be split into runs of seg_chunks
- * chunks (the last run of each sequence may be shorter), each run on its own
- * CTA, composed through the segment maps; 0 lets the library choose.  The
- * result is the same up to rounding for every value (the composition is
- * exact), which the tests exercise.  Returns DN_ERR_WORKSPACE if the forced
- * split needs more segment slots than the library's limit (4096).
+ * seg_chunks > 0 forces every sequence to be split into runs of
+ * (seg_chunks & 0xffff) chunks (the last run of each sequence may be shorter),
+ * each run on its own CTA, composed through the segment maps; 0 lets the
+ * library choose.  For dense batches, bits 16-30 may force a different length
+ * of the first run ((seg_chunks >> 16): its chunks, 1 .. the run length; 0:
+ * the same length).  The result is the same up to rounding for every value
+ * (the composition is exact), which the tests exercise.  Returns
+ * DN_ERR_WORKSPACE if the forced split needs more segment slots than the
+ * library's limit (4096), DN_ERR_INVALID_ARG for a first run longer than the
+ * others.
  */
 dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                           const dn_tensor* beta, const dn_tensor* initial_state,
@@ -279,10 +283,14 @@ void deltanet_release_workspace(void);
 /*
  * deltanet_last_schedule -- the segmentation chosen by the last successful
  * call on this thread for dense (cu_seqlens == NULL) batches: segments per
- * sequence-head chain and chunks per segment.  Varlen batches are scheduled on
- * the device and report -1 for both.  For tests and benchmarks.
+ * sequence-head chain, chunks per segment, and chunks of the first segment
+ * (which may be shorter: on the tensor-core path it runs next to the summary
+ * pass, which costs less per chunk).  Any pointer may be NULL.  Varlen batches
+ * are scheduled on the device and report -1 for all three.  For tests and
+ * benchmarks.
  */
-void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment);
+void deltanet_last_schedule(int* segments_per_chain, int* chunks_per_segment,
+                            int* chunks_first_segment);
 
 /* Number of kernels the last successful call on this thread enqueued. */
 int deltanet_last_launches(void);

@@ -83,6 +83,19 @@ def test_forced_segmentation_is_exact(seg):
     assert max(e_seg) <= 1e-2 and max(e_one) <= 1e-2
 
 
+@pytest.mark.parametrize("first", [1, 3])
+def test_split_with_a_shorter_first_run(first):
+    """Run 0 (on the tensor-core path computed by the boundary kernel next to the
+    summary items) may be shorter than the other runs, which the schedule uses
+    when a summary chunk is cheaper than a boundary chunk; the result equals the
+    serial pass."""
+    w = wl.custom(2, 64 * 13 - 5, 1, 128, 128, torch.bfloat16, init_state=True)
+    x = wl.generate(w, seed=16)
+    check(w, x, seg_chunks=5 | (first << 16))
+    G, s, s0 = dn.last_schedule(with_first=True)
+    assert (G, s, s0) == (1 + (13 - first + 4) // 5, 5, first), (G, s, s0)
+
+
 def test_segmentation_short_memory_case():
     """Short runs (1 chunk) with a slowly forgetting state: beta small so the
     transition products stay far from zero and the composition matters."""
@@ -182,8 +195,8 @@ def test_schedule_of_config_shapes():
     q = torch.zeros((1, 65536, 16, 128), dtype=torch.bfloat16, device=DEV)
     b = torch.zeros((1, 65536, 16), device=DEV)
     dn.deltanet_fwd(q, q, torch.zeros_like(q), b)
-    G, s = dn.last_schedule()
-    assert G >= 4 and G * s >= 1024
+    G, s, s0 = dn.last_schedule(with_first=True)
+    assert G >= 4 and s0 + (G - 1) * s >= 1024 and 1 <= s0 <= s
 
 
 # ---- full-size configs: every output of a subset of heads ------------------

@@ -93,3 +93,13 @@ def test_states_packed(gated):
     w = wl.custom(1, 0, 2, 64, 64, torch.bfloat16, init_state=True, seqlens=lens, gated=True)
     x = wl.generate(w, seed=61)
     check(w, x, gated, seg_chunks=1)
+
+
+@pytest.mark.parametrize("seg", [0, 1, 3])
+def test_states_packed_tensor_core_shape(seg):
+    """d_k = d_v = 128 bf16 DeltaNet: the tensor-core boundary kernel writes the
+    states, packed input with empty and 1-token sequences, split or not."""
+    lens = [0, 1, 64, 130, 0, 200, 700]
+    w = wl.custom(1, 0, 2, 128, 128, torch.bfloat16, init_state=True, seqlens=lens)
+    x = wl.generate(w, seed=62)
+    check(w, x, False, seg_chunks=seg)
