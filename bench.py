@@ -332,7 +332,9 @@ def run_b200(args, w: wl.Workload):
     tflops = ws * th * fpt / (ms / 1e3) / 1e12
     hbm_peak, tc_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(w)
-    tc_path = not w.gated and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+    # DeltaNet and Gated DeltaNet (one write per token) at d_k = d_v = 128 run on the
+    # tensor-core kernels
+    tc_path = w.nh == 1 and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
     # the tensor-core boundary kernel moves q, k, v, o and the states (beta is read by the
     # UT pre-pass); the mma.sync boundary kernel reads beta (and g) itself
     kernel_bytes = alg_bytes - (4.0 * w.tokens * w.H if tc_path else 0.0)

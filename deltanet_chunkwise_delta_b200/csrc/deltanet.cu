@@ -250,12 +250,11 @@ struct Dims {
 template <typename E, int DK, int DV, int STAGES, bool GATED>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
-    // bf16 DeltaNet with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels (with or
-    // without the chunk-start states); Gated DeltaNet and the other shapes on the mma.sync
-    // chain kernels
-    constexpr bool kTcShape =
-        !GATED && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
-    const bool use_tc = kTcShape;
+    // bf16 DeltaNet and Gated DeltaNet with d_k = d_v = 128 run on the tensor-core (tcgen05)
+    // kernels (with or without the chunk-start states); the Gated Delta Product (several
+    // writes per token) and the other shapes on the mma.sync chain kernels
+    constexpr bool kTcShape = std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
+    const bool use_tc = kTcShape && p.nh <= 1;
     using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED>;
@@ -266,14 +265,15 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kA = k_summary<E, DK, DV, STAGES, GATED>;
     auto* kS8 = k_scan<DK, DV, 8>;
     auto* kS16 = k_scan<DK, DV, 16>;
-    auto* kCt = tc::k_tc_chain;
-    auto* kAt = tcs::k_tc_summary;
-    auto* kPrep = k_ut_prep;
-    constexpr int smemPrep = PrepSmem::TOTAL;
+    auto* kCt = tc::k_tc_chain<GATED>;
+    auto* kAt = tcs::k_tc_summary<GATED>;
+    auto* kPrep = k_ut_prep<GATED>;
+    constexpr int smemPrep = PrepSmemT<GATED>::TOTAL;
+    constexpr int smemCt = tc::TcLay<GATED>::SMEM_BYTES, smemAt = tcs::SumLay<GATED>::SMEM_BYTES;
     dn_status st;
     if (use_tc) {
-        if ((st = set_smem(kCt, dev, tc::SMEM_BYTES)) != DN_OK) return st;
-        if ((st = set_smem(kAt, dev, tcs::SMEM_BYTES)) != DN_OK) return st;
+        if ((st = set_smem(kCt, dev, smemCt)) != DN_OK) return st;
+        if ((st = set_smem(kAt, dev, smemAt)) != DN_OK) return st;
         if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
         // several pre-pass CTAs share an SM: ask for the largest shared-memory carveout
         if (cudaFuncSetAttribute(kPrep, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -350,7 +350,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     // UT factors of every (chunk, head): chunks <= ceil(T / C) per row (+1 per sequence)
     const int64_t chunk_ub = d.varlen ? n_c_max + d.N : d.B * n_c_max;
     const size_t off_T = off_SS + up256((size_t)slots * DK * DV * 4);
-    bytes = off_T + (use_tc ? (size_t)chunk_ub * d.H * kUnitBytes : 0);
+    bytes = off_T + (use_tc ? (size_t)chunk_ub * d.H * unit_bytes(GATED) : 0);
     StreamWs ws;
     if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
     char* base = ws.buf;
@@ -410,7 +410,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     if (use_tc) {
         const int64_t units = chunk_ub * d.H;
         if (units > 0) {
-            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * kPrepCtasPerSm);
+            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * prep_ctas_per_sm<GATED>());
             kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
             ++launches;
         }
@@ -424,23 +424,23 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             if (cudaEventRecord(aux.fork, stream) != cudaSuccess ||
                 cudaStreamWaitEvent(aux.stream, aux.fork, 0) != cudaSuccess)
                 return DN_ERR_CUDA;
-            kCt<<<(unsigned)chains, tc::kThreadsTc, tc::SMEM_BYTES, aux.stream>>>(tq, tk, tv, to, p0);
+            kCt<<<(unsigned)chains, tc::kThreadsTc, smemCt, aux.stream>>>(tq, tk, tv, to, p0);
             ++launches;
             if (cudaEventRecord(aux.join, aux.stream) != cudaSuccess) return DN_ERR_CUDA;
-            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
+            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, smemAt, stream>>>(tk, tv, p); ++launches; }
             if (cudaStreamWaitEvent(stream, aux.join, 0) != cudaSuccess) return DN_ERR_CUDA;
             if (nScan > 0) { launch_scan(); ++launches; }
             Params p1 = p;
             p1.sched.c_part = 2;
             if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-            kCt<<<(unsigned)(chains * (G - 1)), tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p1);
+            kCt<<<(unsigned)(chains * (G - 1)), tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, p1);
             ++launches;
             if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
         } else {
-            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, tcs::SMEM_BYTES, stream>>>(tk, tv, p); ++launches; }
+            if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, smemAt, stream>>>(tk, tv, p); ++launches; }
             if (nScan > 0) { launch_scan(); ++launches; }
             if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-            if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, tc::SMEM_BYTES, stream>>>(tq, tk, tv, to, p); ++launches; }
+            if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, p); ++launches; }
             if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
         }
     } else {

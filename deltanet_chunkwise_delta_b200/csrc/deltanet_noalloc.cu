@@ -98,11 +98,11 @@ dn_status na_setup(int dev, unsigned char** scratch) {
     }
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DN_ERR_CUDA;
-    if (cudaFuncSetAttribute(dn::tc::k_tc_chain, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(dn::tc::k_tc_chain<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::tc::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(dn::k_ut_prep<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dn::PrepSmem::TOTAL) != cudaSuccess ||
-        cudaFuncSetAttribute(dn::k_ut_prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+        cudaFuncSetAttribute(dn::k_ut_prep<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return DN_ERR_CUDA;
     g_na_scratch[dev] = static_cast<unsigned char*>(ptr);
@@ -228,8 +228,8 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     const int64_t units = B * n_c * H;
     const int64_t cap = (int64_t)sms * dn::kPrepCtasPerSm;
     const int grid = (int)(units < cap ? units : cap);
-    dn::k_ut_prep<<<grid, dn::kPrepThreads, dn::PrepSmem::TOTAL, stream>>>(tq, tk, p);
-    dn::tc::k_tc_chain<<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
+    dn::k_ut_prep<false><<<grid, dn::kPrepThreads, dn::PrepSmem::TOTAL, stream>>>(tq, tk, p);
+    dn::tc::k_tc_chain<false><<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
         tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }

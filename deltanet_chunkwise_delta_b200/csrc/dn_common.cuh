@@ -14,8 +14,30 @@ constexpr int kChunk = 64;       // C
 constexpr int kThreads = 256;    // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 4096;  // segment-map slots (P, H, start state) per call
-// workspace bytes per (chunk, head) written by the UT pre-pass: T tile, then P tile
+// workspace bytes per (chunk, head) written by the UT pre-pass: T tile, then P tile, and for
+// Gated DeltaNet a third tile, T diag(lambda[1:l])
 constexpr int kUnitBytes = 16384;
+constexpr int kUnitBytesGated = 24576;
+__host__ __device__ constexpr int unit_bytes(bool gated) { return gated ? kUnitBytesGated : kUnitBytes; }
+
+// Gated DeltaNet: the log decays g of tokens [t, t + 64) of one (batch row, head), read
+// two per lane (tokens at or past `t_end` count as g = 0, a = 1), and their inclusive
+// prefix sums over the chunk: lane l gets c[2 l] and c[2 l + 1] (c_j = g_0 + ... + g_j).
+// Called by a whole warp.
+__device__ __forceinline__ float2 gate_prefix(const float* gbase, int64_t g_st, int t, int t_end) {
+    const int lane = threadIdx.x & 31;
+    const int j = 2 * lane;
+    float g0 = t + j < t_end ? gbase[(int64_t)(t + j) * g_st] : 0.f;
+    float g1 = t + j + 1 < t_end ? gbase[(int64_t)(t + j + 1) * g_st] : 0.f;
+    float s = g0 + g1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+    }
+    // s = c[2 lane + 1]; c[2 lane] = s - g1
+    return make_float2(s - g1, s);
+}
 constexpr int kAutoMaxSlots = 592;  // slots the automatic schedule may use (4 x 148)
 
 // Device error flag values (match dn_status).

@@ -19,8 +19,14 @@
 // A = B L; each diagonal block by forward substitution (one warp per block,
 // one column per lane, fp32), then N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj in
 // order of i - j with tf32 mma.sync, and T = N B.
-// One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM, so the
-// latency of the solve is hidden by parallelism across chunks.  A CTA's shared
+// Gated DeltaNet ("Linear Attention, Visualized", section "Gated DeltaNet
+// (GDN)", complete per-chunk algorithm): with the running sums c_l of the
+// chunk's log decays, Gamma[l][i] = lambda[i+1:l] = exp(c_l - c_i) multiplies
+// both halves of G (L = (K K^T o Gamma) o M_c^-, P = (Q K^T o Gamma) o M_c),
+// and a third tile T' = T diag(lambda[1:l]) = T diag(exp(c_l)) gives
+// W<- = T K<- = T' K to the chain kernels (24 KB per unit: T, P, T').
+// One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM (five when
+// gated), so the latency of the solve is hidden by parallelism across chunks.  A CTA's shared
 // memory is one 32 KB region that holds the unit's q/k tile until the product
 // has read it, and then the solve's blocks, the P tile (staged where N is
 // written later) and the T tile (staged where A was); the next unit's tile is
@@ -52,27 +58,35 @@ static __device__ unsigned long long g_dn_trace_prep[16 * 8];
 #endif
 
 constexpr int kPrepThreads = 128;
-constexpr int kPrepCtasPerSm = 6;
+template <bool GATED>
+constexpr int prep_ctas_per_sm() { return GATED ? 5 : 6; }
+constexpr int kPrepCtasPerSm = prep_ctas_per_sm<false>();
 constexpr int kBlkLd = 20;  // fp32 16 x 16 blocks, 16-byte aligned rows
 constexpr int kBlkFloats = 16 * kBlkLd;
 
 // Shared memory of the pre-pass (byte offsets from a 1024-aligned base).  The
 // region [0, 32 KB) holds [Q d0-63 | K d0-63 | Q d64-127 | K d64-127] while the
 // q/k tile is loaded and read by the product, then the blocks of the solve:
-struct PrepSmem {
+template <bool GATED>
+struct PrepSmemT {
     static constexpr int OFF_QK = 0;
     static constexpr int OFF_A = 0;                               // 10 blocks of A = B L; later the T tile
     static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N; before them the P tile
     static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 5 staging blocks of the off-diagonal solve
-    static constexpr int OFF_BETA = 32768;                        // 2 x 64 step sizes
-    static constexpr int OFF_BAR = OFF_BETA + 2 * kChunk * 4;     // FULL, GDONE, DRAIN
+    static constexpr int OFF_T2 = 32768;                          // gated: the T' tile
+    static constexpr int OFF_BETA = GATED ? 40960 : 32768;        // 2 x 64 step sizes
+    static constexpr int OFF_G = OFF_BETA + 2 * kChunk * 4;       // gated: 2 x 64 log decays
+    static constexpr int OFF_C = OFF_G + (GATED ? 2 * kChunk * 4 : 0);  // gated: 64 running sums
+    static constexpr int OFF_BAR = OFF_C + (GATED ? kChunk * 4 : 0);    // FULL, GDONE, DRAIN
     static constexpr int OFF_MISC = OFF_BAR + 24;                 // TMEM address, then the WaitCtl at + 8
     static constexpr int USED = OFF_MISC + 24;
     static constexpr int TOTAL = USED + 1024;                     // slack for 1024-byte alignment
 };
-static_assert(PrepSmem::OFF_X + 5 * kBlkFloats * 4 <= PrepSmem::OFF_BETA, "solve blocks fit the q/k region");
+using PrepSmem = PrepSmemT<false>;
+static_assert(PrepSmem::OFF_X + 5 * kBlkFloats * 4 <= 32768, "solve blocks fit the q/k region");
 static_assert(PrepSmem::OFF_N + 8192 <= PrepSmem::OFF_X, "P staging fits the N blocks");
-static_assert((PrepSmem::TOTAL + 1024) * kPrepCtasPerSm <= 228 * 1024, "pre-pass shared memory");
+static_assert((PrepSmemT<false>::TOTAL + 1024) * prep_ctas_per_sm<false>() <= 228 * 1024, "pre-pass shared memory");
+static_assert((PrepSmemT<true>::TOTAL + 1024) * prep_ctas_per_sm<true>() <= 228 * 1024, "pre-pass shared memory");
 
 __device__ __forceinline__ int blk_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
 
@@ -124,9 +138,11 @@ __device__ __forceinline__ void ld_blk(float (&acc)[2][4], const float* C) {
     }
 }
 
-static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
+template <bool GATED>
+static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>())
     k_ut_prep(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
-    using L = PrepSmem;
+    using L = PrepSmemT<GATED>;
+    constexpr int kUnit = unit_bytes(GATED);
     extern __shared__ uint8_t prep_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(prep_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -181,6 +197,11 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
             const bool ok = tid < t1 - t0;
             const float* src = p.beta + b * p.b_sb + (int64_t)(t0 + (ok ? tid : 0)) * p.b_st + head * p.b_sh;
             cp_async4(smem_addr(smem + L::OFF_BETA + (bb * kChunk + tid) * 4), src, ok ? 4 : 0);
+            if constexpr (GATED) {
+                // log decays of the chunk (0 past its end: the pad rows are identity steps)
+                const float* gsrc = p.g + b * p.g_sb + (int64_t)(t0 + (ok ? tid : 0)) * p.g_st + head * p.g_sh;
+                cp_async4(smem_addr(smem + L::OFF_G + (bb * kChunk + tid) * 4), gsrc, ok ? 4 : 0);
+            }
         }
         cp_async_commit();
     };
@@ -198,6 +219,14 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         if (__syncthreads_or(!got)) break;
         in_flight = false;
         DN_TRP(it_, 1);
+        if constexpr (GATED) {
+            // running sums c_l of the chunk's log decays (read after the next barrier)
+            if (warp == 1) {
+                const float2 c = gate_prefix(reinterpret_cast<const float*>(smem + L::OFF_G) + bb * kChunk, 1, 0,
+                                             kChunk);
+                reinterpret_cast<float2*>(smem + L::OFF_C)[lane] = c;
+            }
+        }
         // G = [Q; K] K^T into 64 tensor-memory columns: lanes 0-63 Q K^T, 64-127 K K^T
         if (tid == 0) {
             sm100::tc_fence_after();
@@ -213,9 +242,16 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         if (__syncthreads_or(!gdone)) break;
         sm100::tc_fence_after();
         const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + bb * kChunk;
+        const float* cs = reinterpret_cast<const float*>(smem + L::OFF_C);  // gated: running sums
         {
             const int i = 32 * (warp & 1) + lane;  // row of Q K^T (warps 0, 1) or K K^T (warps 2, 3)
             const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+            // gated: Gamma[i][j] = exp(c_i - c_j) for j <= i (c falls with j, so <= 1)
+            const float ci = GATED ? cs[i] : 0.f;
+            auto gam = [&](int j) -> float {
+                if constexpr (GATED) return expf(ci - cs[j]);
+                else return 1.f;
+            };
             if (warp >= 2) {
                 // A = B L, blocked: row i of block row bi; blocks left of the diagonal
                 // row-major, the diagonal block transposed (for the column sweeps)
@@ -233,17 +269,19 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                         if (bj < bi) {
 #pragma unroll
                             for (int q4 = 0; q4 < 4; ++q4) {
+                                const int j = 16 * bj + 4 * q4;
                                 float4 f;
-                                f.x = bta * __uint_as_float(v[16 * bh + 4 * q4 + 0]);
-                                f.y = bta * __uint_as_float(v[16 * bh + 4 * q4 + 1]);
-                                f.z = bta * __uint_as_float(v[16 * bh + 4 * q4 + 2]);
-                                f.w = bta * __uint_as_float(v[16 * bh + 4 * q4 + 3]);
+                                f.x = bta * gam(j) * __uint_as_float(v[16 * bh + 4 * q4 + 0]);
+                                f.y = bta * gam(j + 1) * __uint_as_float(v[16 * bh + 4 * q4 + 1]);
+                                f.z = bta * gam(j + 2) * __uint_as_float(v[16 * bh + 4 * q4 + 2]);
+                                f.w = bta * gam(j + 3) * __uint_as_float(v[16 * bh + 4 * q4 + 3]);
                                 *reinterpret_cast<float4*>(blk + ri * kBlkLd + 4 * q4) = f;
                             }
                         } else {
 #pragma unroll
                             for (int c = 0; c < 16; ++c)
-                                blk[c * kBlkLd + ri] = c < ri ? bta * __uint_as_float(v[16 * bh + c]) : 0.f;
+                                blk[c * kBlkLd + ri] =
+                                    c < ri ? bta * gam(16 * bj + c) * __uint_as_float(v[16 * bh + c]) : 0.f;
                         }
                     }
                 }
@@ -260,7 +298,8 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                         const int col = 32 * hc + 8 * c8;
                         float x[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = (col + e <= i) ? __uint_as_float(v[8 * c8 + e]) : 0.f;
+                        for (int e = 0; e < 8; ++e)
+                            x[e] = (col + e <= i) ? gam(col + e) * __uint_as_float(v[8 * c8 + e]) : 0.f;
                         uint4 w;
                         w.x = sm100::pack_bf16(x[0], x[1]);
                         w.y = sm100::pack_bf16(x[2], x[3]);
@@ -275,7 +314,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         sm100::tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes + 8192, smem + L::OFF_N, 8192);
+            sm100::bulk_store(p.wsT + (size_t)u * kUnit + 8192, smem + L::OFF_N, 8192);
             sm100::bulk_commit();
         }
         DN_TRP(it_, 2);
@@ -360,6 +399,8 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                 mm16_tf32(y30, A_(3, 2), N_(2, 0));
                 finish_block(Nblk, X, 3, 0, y30);
             }
+            // gated: the previous unit's T' copy has read its staging, rewritten below
+            if (GATED && tid == 0) sm100::bulk_wait_read0();
             __syncthreads();
         }
         DN_TRP(it_, 4);
@@ -377,6 +418,7 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                 const float4 b1 = *reinterpret_cast<const float4*>(betas + j0 + 4);
                 const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
                 float vals[8];
+                (void)cs;
                 if (bj <= bi) {
                     const float* nr = Nblk + blk_index(bi, bj) * kBlkFloats + (i & 15) * kBlkLd + (j0 & 15);
                     const float4 f0 = *reinterpret_cast<const float4*>(nr);
@@ -394,6 +436,18 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
                 w.z = sm100::pack_bf16(vals[4], vals[5]);
                 w.w = sm100::pack_bf16(vals[6], vals[7]);
                 *reinterpret_cast<uint4*>(tg + sm100::swz128(i, j0)) = w;
+                if constexpr (GATED) {
+                    // T' = T diag(lambda[1:j]), lambda[1:j] = exp(c_j) <= 1
+                    float l8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) l8[e] = vals[e] * expf(cs[j0 + e]);
+                    uint4 w2;
+                    w2.x = sm100::pack_bf16(l8[0], l8[1]);
+                    w2.y = sm100::pack_bf16(l8[2], l8[3]);
+                    w2.z = sm100::pack_bf16(l8[4], l8[5]);
+                    w2.w = sm100::pack_bf16(l8[6], l8[7]);
+                    *reinterpret_cast<uint4*>(smem + L::OFF_T2 + sm100::swz128(i, j0)) = w2;
+                }
             }
             sm100::fence_async_smem();
         }
@@ -402,7 +456,8 @@ static __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
         // staging once the copy has read it)
         const int un = u + gridDim.x;
         if (tid == 0) {
-            sm100::bulk_store(p.wsT + (size_t)u * kUnitBytes, smem + L::OFF_A, 8192);
+            sm100::bulk_store(p.wsT + (size_t)u * kUnit, smem + L::OFF_A, 8192);
+            if constexpr (GATED) sm100::bulk_store(p.wsT + (size_t)u * kUnit + 16384, smem + L::OFF_T2, 8192);
             sm100::bulk_commit();
         }
         if (un < units) {

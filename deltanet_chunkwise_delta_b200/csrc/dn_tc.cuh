@@ -60,21 +60,29 @@ constexpr int kTmaBWarp = 15;
 //           one U^T / Z^T block between two O^T buffers.
 //   ring B: 2 stages of [V d0-63 | V d64-127 | T]
 //   2 P tiles (chunk r's in buffer r % 2); O staging (two 64-column boxes of token rows)
-constexpr int NA = 3, NB = 2;
+// Gated DeltaNet: ring B stages also hold T' = T diag(lambda[1:l]) (the W<- factor), and ring
+// A has two stages, so that the layout fits.
+constexpr int NB = 2;
 constexpr int A_STAGE = 49152;
 constexpr int A_K = 32768;  // + 8192 for d 64-127; -W and Q at 0 / 8192 (+ 16384 for d 64-127)
 __host__ __device__ constexpr int a_w(int c) { return (c & 1) ? 8192 : 0; }  // -W rows of chunk c
 __host__ __device__ constexpr int a_q(int c) { return (c & 1) ? 0 : 8192; }  // Q rows of chunk c
-constexpr int OFF_B = NA * A_STAGE;
-constexpr int B_STAGE = 24576, B_T = 16384;
-constexpr int OFF_PB = OFF_B + NB * B_STAGE;   // P rows, 2 x 8 KB
-constexpr int OFF_OB = OFF_PB + 2 * 8192;      // O staging
-constexpr int OFF_BAR = OFF_OB + 16384;
+constexpr int B_T = 16384, B_T2 = 24576;
 constexpr int NBAR = 34;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM_USED = OFF_MISC + 64;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+template <bool GATED>
+struct TcLay {
+    static constexpr int NA = GATED ? 2 : 3;
+    static constexpr int OFF_B = NA * A_STAGE;
+    static constexpr int B_STAGE = GATED ? 32768 : 24576;  // V, T (, T')
+    static constexpr int OFF_PB = OFF_B + NB * B_STAGE;    // P rows, 2 x 8 KB
+    static constexpr int OFF_OB = OFF_PB + 2 * 8192;       // O staging
+    static constexpr int OFF_BAR = OFF_OB + 16384;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+};
+static_assert(TcLay<false>::SMEM_BYTES <= 232448 && TcLay<true>::SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int SMEM_BYTES = TcLay<false>::SMEM_BYTES;
 
 // tensor-memory columns (512 allocated): S^T fp32, [O^T (odd chunks) | U^T/Z^T |
 // O^T (even chunks)] (one product of N = 128 writes Z^T and the chunk's O^T), W^T,
@@ -167,9 +175,44 @@ __device__ __forceinline__ void store_token_rows(const RowFrags& f, int q, uint8
                           pack_bf16(scale * __uint_as_float(f.hi[g][2]), scale * __uint_as_float(f.hi[g][3])));
 }
 
+// bf16 pair * f, rounded to nearest-even.
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float f) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+    return pack_bf16(lo * f, hi * f);
+}
+// Gated DeltaNet: token rows 16 q .. 16 q + 15 of a chunk tile (two 64-column boxes of
+// 128-byte rows, at box0 and box0 + box_stride) multiplied in place by one factor per
+// row: lane l holds the factor of row 16 q + (l & 15).  A whole warp; the caller fences
+// the writes for the tensor cores.
+__device__ __forceinline__ void scale_token_rows(uint8_t* box0, uint32_t box_stride, int q, float f) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int id = lane + 32 * i;  // 256 pieces of 16 bytes: 16 rows x 2 boxes x 8
+        const int piece = id & 7, lr = (id >> 3) & 15, box = id >> 7;
+        const float fr = __shfl_sync(0xffffffffu, f, lr);
+        uint4* ptr = reinterpret_cast<uint4*>(box0 + box * box_stride + (16 * q + lr) * 128 + piece * 16);
+        uint4 w = *ptr;
+        w.x = scale_bf16x2(w.x, fr);
+        w.y = scale_bf16x2(w.y, fr);
+        w.z = scale_bf16x2(w.z, fr);
+        w.w = scale_bf16x2(w.w, fr);
+        *ptr = w;
+    }
+}
+// Gated DeltaNet: lambda[1:C] = exp(c_C) of chunk c of a run (a whole warp).
+__device__ __forceinline__ float chunk_decay(const Params& p, const Item& it, int c) {
+    const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
+    const float2 cc = gate_prefix(gb, p.g_st, it.tok0 + c * kChunk, it.tok1);
+    return expf(__shfl_sync(0xffffffffu, cc.y, 31));
+}
+
+template <bool GATED>
 static __global__ void __launch_bounds__(kThreadsTc, 1)
     k_tc_chain(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
+    using L = TcLay<GATED>;
+    constexpr int kUnit = unit_bytes(GATED);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -178,15 +221,15 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
     if ((int)blockIdx.x >= n_items) return;
     const Item it = item_C(p.sched, blockIdx.x);
 
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + OFF_MISC + 8);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + L::OFF_MISC + 8);
     volatile int* abort_flag = &ctl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NA; ++s) {
+        for (int s = 0; s < L::NA; ++s) {
             mbar_init(&bars[B_FULLA + s], 1);
             mbar_init(&bars[B_EMPTYA + s], 1);
         }
@@ -243,8 +286,8 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t bytes = 32768u;
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
-                const int s = r % NA;
-                if (r >= NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / NA) - 1) & 1, abort_flag)) break;
+                const int s = r % L::NA;
+                if (r >= L::NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / L::NA) - 1) & 1, abort_flag)) break;
                 mbar_expect_tx(&bars[B_FULLA + s], bytes);
                 uint8_t* st = smem + s * A_STAGE;
                 const int t0 = it.tok0 + r * kChunk;
@@ -258,25 +301,26 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             }
             // the last loads issued must have landed before the CTA may exit (even after an abort)
             volatile int drain = 0;
-            for (int r = issued - NA < 0 ? 0 : issued - NA; r < issued; ++r)
-                mbar_wait(&bars[B_FULLA + (r % NA)], (r / NA) & 1, &drain, kDrainWaitNs);
+            for (int r = issued - L::NA < 0 ? 0 : issued - L::NA; r < issued; ++r)
+                mbar_wait(&bars[B_FULLA + (r % L::NA)], (r / L::NA) & 1, &drain, kDrainWaitNs);
         }
     } else if (warp == kTmaBWarp) {
         // ------------------------------------------------------------ ring B: v, T
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = 16384u + 8192u;
+            const uint32_t bytes = 16384u + 8192u + (GATED ? 8192u : 0u);
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
                 const int s = r & 1;
                 if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
                 mbar_expect_tx(&bars[B_FULLB + s], bytes);
-                uint8_t* st = smem + OFF_B + s * B_STAGE;
+                uint8_t* st = smem + L::OFF_B + s * L::B_STAGE;
                 const int t0 = it.tok0 + r * kChunk;
 #pragma unroll
                 for (int a = 0; a < 2; ++a)
                     tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
-                bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnitBytes, 8192,
-                          &bars[B_FULLB + s]);
+                const uint8_t* unit = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit;
+                bulk_load(st + B_T, unit, 8192, &bars[B_FULLB + s]);
+                if constexpr (GATED) bulk_load(st + B_T2, unit + 16384, 8192, &bars[B_FULLB + s]);
                 issued = r + 1;
             }
             volatile int drain = 0;
@@ -295,9 +339,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t i_o = idesc_bf16(128, 64, false, false);
             const uint64_t dWQ = sdesc(sb, 16, 1024);           // [-W; Q] / [Q; -W] token rows, K-major
             const uint64_t dK = sdesc(sb + A_K, 8192, 1024);    // K, MN-major
-            const uint64_t dP = sdesc(sb + OFF_PB, 16, 1024);   // P^T, K-major (+ 8 KB for odd chunks)
+            const uint64_t dP = sdesc(sb + L::OFF_PB, 16, 1024);   // P^T, K-major (+ 8 KB for odd chunks)
             for (int r = 0; r < nch; ++r) {
-                const int sa = r % NA, s = r & 1;
+                const int sa = r % L::NA, s = r & 1;
                 const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
                 DN_TR(true, r, 0);
                 if (r + 1 == p.stall_chunk && !mbar_wait(&bars[B_STALL], 0, abort_flag)) break;
@@ -355,21 +399,23 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t sb = saddr(smem);
             const uint32_t i_tt = idesc_bf16(128, 64, true, false);
             const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
-            const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
-            const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
+            const uint64_t dVT = sdesc(sb + L::OFF_B, 8192, 1024);        // V^T, MN-major
+            const uint64_t dT = sdesc(sb + L::OFF_B + B_T, 16, 1024);     // T^T, K-major
+            // W = T K, or for Gated DeltaNet W<- = T' K with T' = T diag(lambda[1:l])
+            const uint64_t dTw = GATED ? sdesc(sb + L::OFF_B + B_T2, 16, 1024) : dT;
             auto issue_w = [&](int c) {
-                const uint64_t sta = (uint64_t)(((c % NA) * A_STAGE) >> 4);
-                const uint64_t stb = (uint64_t)(((c & 1) * B_STAGE) >> 4);
+                const uint64_t sta = (uint64_t)(((c % L::NA) * A_STAGE) >> 4);
+                const uint64_t stb = (uint64_t)(((c & 1) * L::B_STAGE) >> 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     umma_bf16(tmem + TM_WT, dKT + sta + (uint64_t)((j * 2048) >> 4),
-                              dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                              dTw + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 umma_commit(&bars[B_WUFULL]);
             };
             // U^T of chunk c; its ring-B stage is consumed after it (W^T came first)
             auto issue_u = [&](int c) {
                 const int s = c & 1;
-                const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
+                const uint64_t stb = (uint64_t)((s * L::B_STAGE) >> 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     umma_bf16(tmem + TM_ZU, dVT + stb + (uint64_t)((j * 2048) >> 4),
@@ -378,7 +424,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 umma_commit(&bars[B_EMPTYB + s]);
             };
             auto wait_data = [&](int c) -> bool {
-                return mbar_wait2(&bars[B_FULLA + c % NA], (c / NA) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
+                return mbar_wait2(&bars[B_FULLA + c % L::NA], (c / L::NA) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
                                   abort_flag);
             };
             bool ok = wait_data(0);
@@ -415,8 +461,8 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         auto issue_p = [&](int c) {
             ++p_issued;
             mbar_expect_tx(&bars[B_PFULL + (c & 1)], 8192u);
-            bulk_load(smem + OFF_PB + (c & 1) * 8192,
-                      p.wsT + ((size_t)(it.cbase + c) * p.sched.H + it.head) * kUnitBytes + 8192, 8192,
+            bulk_load(smem + L::OFF_PB + (c & 1) * 8192,
+                      p.wsT + ((size_t)(it.cbase + c) * p.sched.H + it.head) * kUnit + 8192, 8192,
                       &bars[B_PFULL + (c & 1)]);
         };
         // O^T of chunk c -> out: read out of tensor memory (and zeroed for the next
@@ -424,7 +470,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         // TMA box layout of out) and written by one TMA store per box; a chunk that
         // ends inside the run's last 64 tokens is written with bounded 16-byte stores.
         __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
-        uint8_t* ob = smem + OFF_OB;
+        uint8_t* ob = smem + L::OFF_OB;
         auto store_o = [&](int c) -> bool {
             // read out and zero the columns first: the next chunk's first product waits
             // for them
@@ -482,10 +528,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             }
         }
         for (int r = 0; r < nch; ++r) {
-            uint8_t* stage = smem + (r % NA) * A_STAGE;
+            uint8_t* stage = smem + (r % L::NA) * A_STAGE;
             // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's q/k stage,
             // once the stage holds the chunk (its previous chunk's products are done)
-            if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
+            if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % L::NA], (r / L::NA) & 1,
                                                     abort_flag)))
                 break;
             DN_TR(q == 0, r, 13);
@@ -497,6 +543,19 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_WTFREE]);
                 store_token_rows(f, q, stage + a_w(r), 16384, -1.f);
+            }
+            if constexpr (GATED) {
+                // W^T has read K: the chunk's Q rows become Q<- (lambda[1:l] q_l, read by the
+                // output product) and its K rows K-> (lambda[l+1:C] k_l, read by the state
+                // update), with lambda[1:l] = exp(c_l) and lambda[l+1:C] = exp(c_C - c_l)
+                const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
+                const float2 c = gate_prefix(gb, p.g_st, it.tok0 + r * kChunk, it.tok1);
+                const int t = 16 * q + (lane & 15);
+                const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1), cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
+                const float cC = __shfl_sync(0xffffffffu, c.y, 31);
+                const float ct = (t & 1) ? cy : cx;
+                scale_token_rows(stage + a_q(r), 16384, q, expf(ct));
+                scale_token_rows(stage + A_K, 8192, q, expf(cC - ct));
             }
             fence_async_smem();
             __syncwarp();
@@ -556,17 +615,25 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                     for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * h + c) * D + d] = __uint_as_float(v[c]);
             } else {
                 store_chunk_state(0, v);
-                tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
-                tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                 uint32_t pk[32];
                 pack_pairs<64>(v, pk);
                 tmem_st32(tmem + lane_base + TM_SBF + 32 * h, pk);
+                if constexpr (GATED) {
+                    // Gated DeltaNet: the update of chunk 0 adds K->^T Z to lambda[1:C] S
+                    const float lam = chunk_decay(p, it, 0);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
+                }
+                tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
             }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[B_SBF]);
         for (int r = 0; r < nch; ++r) {
+            // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
+            const float lam_next = (GATED && r + 1 < nch) ? chunk_decay(p, it, r + 1) : 1.f;
             // Z^T -> bf16 (A operand of the S^T update and of O^T += Z^T P^T), once the
             // previous chunk's O^T += Z^T P^T has read the previous one
             DN_TR(warp == 0, r, 27);
@@ -609,6 +676,15 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                         x_out[(int64_t)(64 * h + c) * D + d] = __uint_as_float(v[c]);
                 }
                 if (r + 1 < nch) store_chunk_state(r + 1, v);
+                if (GATED && r + 1 < nch) {
+                    // S^T <- lambda[1:C] S^T before the next chunk's update accumulates into
+                    // it (complete before this warp's next Z^T arrival, which that update
+                    // waits for); the bf16 copy above stays unscaled
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
+                    tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+                    tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                }
             }
         }
     }

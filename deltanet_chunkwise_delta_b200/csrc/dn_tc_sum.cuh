@@ -61,20 +61,26 @@ constexpr int kTmaBWarp = 15;
 //   ring B: 2 stages of [V d0-63 | V d64-127 | T]
 //   Z^T bf16 of chain H and of chain P: d_v rows x 64 tokens, 128-byte swizzled
 //   S_P^T bf16: d_v rows x [d_k 0-63 | d_k 64-127], 128-byte swizzled
+//   (Gated DeltaNet: ring B stages also hold T' = T diag(lambda[1:l]), the W<- factor)
 constexpr int NA = 3, NB = 2;
 constexpr int A_STAGE = 32768;
 constexpr int A_K = 16384;
 constexpr int OFF_B = NA * A_STAGE;
-constexpr int B_STAGE = 24576, B_T = 16384;
-constexpr int OFF_Z = OFF_B + NB * B_STAGE;
+constexpr int B_T = 16384, B_T2 = 24576;
 constexpr int Z_BYTES = 16384;
-constexpr int OFF_SP = OFF_Z + 2 * Z_BYTES;
-constexpr int OFF_BAR = OFF_SP + 32768;
 constexpr int NBAR = 27;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM_USED = OFF_MISC + 64;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+template <bool GATED>
+struct SumLay {
+    static constexpr int B_STAGE = GATED ? 32768 : 24576;
+    static constexpr int OFF_Z = OFF_B + NB * B_STAGE;
+    static constexpr int OFF_SP = OFF_Z + 2 * Z_BYTES;
+    static constexpr int OFF_BAR = OFF_SP + 32768;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 64;
+    static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+};
+static_assert(SumLay<false>::SMEM_BYTES <= 232448 && SumLay<true>::SMEM_BYTES <= 232448, "shared memory budget");
+constexpr int SMEM_BYTES = SumLay<false>::SMEM_BYTES;
 
 // 32 consecutive 32-bit tensor-memory columns of this thread's lane, without
 // waiting: follow with tmem_wait_st() before the columns are signalled as written.
@@ -131,8 +137,11 @@ static __device__ unsigned long long g_dn_trace_sum[64 * 32];
     } while (0)
 #endif
 
+template <bool GATED>
 static __global__ void __launch_bounds__(kThreadsSum, 1)
     k_tc_summary(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, Params p) {
+    using L = SumLay<GATED>;
+    constexpr int kUnit = unit_bytes(GATED);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -142,9 +151,9 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
     int mode = kModeEnd;
     const Item it = item_A(p.sched, blockIdx.x, mode);
 
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + OFF_MISC + 8);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    WaitCtl* ctl = reinterpret_cast<WaitCtl*>(smem + L::OFF_MISC + 8);
     volatile int* abort_flag = &ctl->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -215,13 +224,14 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 for (int r = 0; r < nch; ++r) {
                     const int s = r & 1;
                     if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
-                    mbar_expect_tx(&bars[B_FULLB + s], 16384u + 8192u);
-                    uint8_t* st = smem + OFF_B + s * B_STAGE;
+                    mbar_expect_tx(&bars[B_FULLB + s], 16384u + 8192u + (GATED ? 8192u : 0u));
+                    uint8_t* st = smem + OFF_B + s * L::B_STAGE;
                     const int t0 = it.tok0 + r * kChunk;
     #pragma unroll
                     for (int a = 0; a < 2; ++a) tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
-                    bulk_load(st + B_T, p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnitBytes, 8192,
-                              &bars[B_FULLB + s]);
+                    const uint8_t* unit = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit;
+                    bulk_load(st + B_T, unit, 8192, &bars[B_FULLB + s]);
+                    if constexpr (GATED) bulk_load(st + B_T2, unit + 16384, 8192, &bars[B_FULLB + s]);
                     issued = r + 1;
                 }
                 volatile int drain = 0;
@@ -241,8 +251,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
                 const uint64_t dW = sdesc(sb, 16, 1024);             // -W token rows, K-major
                 const uint64_t dK = sdesc(sb + A_K, 8192, 1024);     // K, MN-major
-                const uint64_t dZ = sdesc(sb + OFF_Z, 16, 1024);     // Z^T rows, K-major (+ Z_BYTES for P)
-                const uint64_t dSP = sdesc(sb + OFF_SP, 16, 1024);   // S_P^T bf16 rows, K-major
+                const uint64_t dZ = sdesc(sb + L::OFF_Z, 16, 1024);     // Z^T rows, K-major (+ Z_BYTES for P)
+                const uint64_t dSP = sdesc(sb + L::OFF_SP, 16, 1024);   // S_P^T bf16 rows, K-major
                 for (int r = 0; r < nch; ++r) {
                     const int sa = r % NA;
                     const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
@@ -316,19 +326,21 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
                 const uint64_t dVT = sdesc(sb + OFF_B, 8192, 1024);        // V^T, MN-major
                 const uint64_t dT = sdesc(sb + OFF_B + B_T, 16, 1024);     // T^T, K-major
+                // W = T K, or for Gated DeltaNet W<- = T' K with T' = T diag(lambda[1:l])
+                const uint64_t dTw = GATED ? sdesc(sb + OFF_B + B_T2, 16, 1024) : dT;
                 auto issue_w = [&](int c) {
                     const uint64_t sta = (uint64_t)(((c % NA) * A_STAGE) >> 4);
-                    const uint64_t stb = (uint64_t)(((c & 1) * B_STAGE) >> 4);
+                    const uint64_t stb = (uint64_t)(((c & 1) * L::B_STAGE) >> 4);
     #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         umma_bf16(tmem + TM_WT, dKT + sta + (uint64_t)((j * 2048) >> 4),
-                                  dT + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
+                                  dTw + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                     umma_commit(&bars[B_WUFULL]);
                 };
                 // U^T of chunk c; its ring-B stage is consumed after it (W^T came first)
                 auto issue_u = [&](int c) {
                     const int s = c & 1;
-                    const uint64_t stb = (uint64_t)((s * B_STAGE) >> 4);
+                    const uint64_t stb = (uint64_t)((s * L::B_STAGE) >> 4);
     #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         umma_bf16(tmem + tm_zu(0), dVT + stb + (uint64_t)((j * 2048) >> 4),
@@ -381,6 +393,17 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     tc_fence_before();
                     store_token_rows(f, q, stage, 8192, -1.f);
                 }
+                if constexpr (GATED) {
+                    // W^T has read K: the chunk's K rows become K-> = lambda[l+1:C] k_l
+                    // (exp(c_C - c_l)), read by both state updates
+                    const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
+                    const float2 c = gate_prefix(gb, p.g_st, it.tok0 + r * kChunk, it.tok1);
+                    const int t = 16 * q + (lane & 15);
+                    const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1);
+                    const float cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
+                    const float cC = __shfl_sync(0xffffffffu, c.y, 31);
+                    tc::scale_token_rows(stage + A_K, 8192, q, expf(cC - ((t & 1) ? cy : cx)));
+                }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_WFULL]);
@@ -404,14 +427,14 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 } else {
                     x_out = p.wsH + (int64_t)(it.slot + it.g) * D * D;
                 }
-                uint8_t* zs = smem + OFF_Z + x * Z_BYTES;
+                uint8_t* zs = smem + L::OFF_Z + x * Z_BYTES;
                 // bf16 copy of S_x^T columns 64 hh .. + 63 of row d: chain H into tensor
                 // memory, chain P into K block hh of its shared-memory operand
                 auto store_sbf = [&](int xx, int hh, const uint32_t(&pk)[32]) {
                     if (xx == 0) {
                         tmem_st32_nowait(tmem + lane_base + TM_SBF + 32 * hh, pk);
                     } else {
-                        uint8_t* sp = smem + OFF_SP + hh * 16384;
+                        uint8_t* sp = smem + L::OFF_SP + hh * 16384;
     #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             *reinterpret_cast<uint4*>(sp + swz128(d, 8 * c)) =
@@ -432,11 +455,17 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     if (nch == 0) {
                         for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
                     } else {
-                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
-                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                         uint32_t pk[32];
                         pack_pairs<64>(v, pk);
                         store_sbf(x, hh, pk);
+                        if constexpr (GATED) {
+                            // the update of chunk 0 adds K->^T Z to lambda[1:C] S
+                            const float lam = tc::chunk_decay(p, it, 0);
+    #pragma unroll
+                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
+                        }
+                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+                        tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                     }
                 }
                 tmem_wait_st();  // the bf16 copy's tensor-memory stores
@@ -445,6 +474,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
                 for (int r = 0; r < nch; ++r) {
+                    // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
+                    const float lam_next = (GATED && r + 1 < nch) ? tc::chunk_decay(p, it, r + 1) : 1.f;
                     // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
                     // the state update)
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
@@ -479,6 +510,15 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                         if (r == nch - 1) {
     #pragma unroll
                             for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
+                        }
+                        if (GATED && r + 1 < nch) {
+                            // S_x^T <- lambda[1:C] S_x^T before the next chunk's update accumulates
+                            // into it (the bf16 copy above stays unscaled)
+    #pragma unroll
+                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
+                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32,
+                                      *reinterpret_cast<uint32_t(*)[32]>(v + 32));
                         }
                     }
                     tmem_wait_st();  // the bf16 copy's tensor-memory stores
