@@ -20,23 +20,36 @@ constexpr int kUnitBytes = 16384;
 constexpr int kUnitBytesGated = 24576;
 __host__ __device__ constexpr int unit_bytes(bool gated) { return gated ? kUnitBytesGated : kUnitBytes; }
 
-// Gated DeltaNet: the log decays g of tokens [t, t + 64) of one (batch row, head), read
-// two per lane (tokens at or past `t_end` count as g = 0, a = 1), and their inclusive
-// prefix sums over the chunk: lane l gets c[2 l] and c[2 l + 1] (c_j = g_0 + ... + g_j).
-// Called by a whole warp.
-__device__ __forceinline__ float2 gate_prefix(const float* gbase, int64_t g_st, int t, int t_end) {
+// Gated DeltaNet: the log decays g of tokens [t, t + 64) of one (batch row, head), two
+// per lane: lane l reads tokens t + 2 l and t + 2 l + 1 (tokens at or past `t_end` count
+// as g = 0, a = 1).
+__device__ __forceinline__ float2 gate_load(const float* gbase, int64_t g_st, int t, int t_end) {
+    const int j = 2 * (threadIdx.x & 31);
+    return make_float2(t + j < t_end ? gbase[(int64_t)(t + j) * g_st] : 0.f,
+                       t + j + 1 < t_end ? gbase[(int64_t)(t + j + 1) * g_st] : 0.f);
+}
+// Their inclusive prefix sums over the chunk: lane l gets c[2 l] and c[2 l + 1]
+// (c_j = g_0 + ... + g_j).  A whole warp.
+__device__ __forceinline__ float2 gate_scan(float2 g) {
     const int lane = threadIdx.x & 31;
-    const int j = 2 * lane;
-    float g0 = t + j < t_end ? gbase[(int64_t)(t + j) * g_st] : 0.f;
-    float g1 = t + j + 1 < t_end ? gbase[(int64_t)(t + j + 1) * g_st] : 0.f;
-    float s = g0 + g1;
+    float s = g.x + g.y;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, s, o);
         if (lane >= o) s += y;
     }
     // s = c[2 lane + 1]; c[2 lane] = s - g1
-    return make_float2(s - g1, s);
+    return make_float2(s - g.y, s);
+}
+// Their total c_63 on every lane.  A whole warp.
+__device__ __forceinline__ float gate_sum(float2 g) {
+    float s = g.x + g.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+__device__ __forceinline__ float2 gate_prefix(const float* gbase, int64_t g_st, int t, int t_end) {
+    return gate_scan(gate_load(gbase, g_st, t, t_end));
 }
 constexpr int kAutoMaxSlots = 592;  // slots the automatic schedule may use (4 x 148)
 

@@ -77,7 +77,8 @@ struct PrepSmemT {
     static constexpr int OFF_BETA = GATED ? 40960 : 32768;        // 2 x 64 step sizes
     static constexpr int OFF_G = OFF_BETA + 2 * kChunk * 4;       // gated: 2 x 64 log decays
     static constexpr int OFF_C = OFF_G + (GATED ? 2 * kChunk * 4 : 0);  // gated: 64 running sums
-    static constexpr int OFF_BAR = OFF_C + (GATED ? kChunk * 4 : 0);    // FULL, GDONE, DRAIN
+    static constexpr int OFF_LAM = OFF_C + (GATED ? kChunk * 4 : 0);    // gated: exp of those
+    static constexpr int OFF_BAR = OFF_LAM + (GATED ? kChunk * 4 : 0);  // FULL, GDONE, DRAIN
     static constexpr int OFF_MISC = OFF_BAR + 24;                 // TMEM address, then the WaitCtl at + 8
     static constexpr int USED = OFF_MISC + 24;
     static constexpr int TOTAL = USED + 1024;                     // slack for 1024-byte alignment
@@ -225,6 +226,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                 const float2 c = gate_prefix(reinterpret_cast<const float*>(smem + L::OFF_G) + bb * kChunk, 1, 0,
                                              kChunk);
                 reinterpret_cast<float2*>(smem + L::OFF_C)[lane] = c;
+                reinterpret_cast<float2*>(smem + L::OFF_LAM)[lane] = make_float2(expf(c.x), expf(c.y));
             }
         }
         // G = [Q; K] K^T into 64 tensor-memory columns: lanes 0-63 Q K^T, 64-127 K K^T
@@ -249,7 +251,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
             // gated: Gamma[i][j] = exp(c_i - c_j) for j <= i (c falls with j, so <= 1)
             const float ci = GATED ? cs[i] : 0.f;
             auto gam = [&](int j) -> float {
-                if constexpr (GATED) return expf(ci - cs[j]);
+                if constexpr (GATED) return __expf(ci - cs[j]);
                 else return 1.f;
             };
             if (warp >= 2) {
@@ -438,9 +440,10 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                 *reinterpret_cast<uint4*>(tg + sm100::swz128(i, j0)) = w;
                 if constexpr (GATED) {
                     // T' = T diag(lambda[1:j]), lambda[1:j] = exp(c_j) <= 1
+                    const float* lam = reinterpret_cast<const float*>(smem + L::OFF_LAM);
                     float l8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) l8[e] = vals[e] * expf(cs[j0 + e]);
+                    for (int e = 0; e < 8; ++e) l8[e] = vals[e] * lam[j0 + e];
                     uint4 w2;
                     w2.x = sm100::pack_bf16(l8[0], l8[1]);
                     w2.y = sm100::pack_bf16(l8[2], l8[3]);

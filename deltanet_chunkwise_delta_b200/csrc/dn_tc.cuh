@@ -200,11 +200,27 @@ __device__ __forceinline__ void scale_token_rows(uint8_t* box0, uint32_t box_str
         *ptr = w;
     }
 }
+// Gated DeltaNet: the log decays of chunk c of a run, two per lane (gate_load), or zeros
+// past the run's last chunk.
+__device__ __forceinline__ float2 chunk_gates(const Params& p, const Item& it, int c, int nch) {
+    if (c >= nch) return make_float2(0.f, 0.f);
+    return gate_load(p.g + it.b * p.g_sb + it.head * p.g_sh, p.g_st, it.tok0 + c * kChunk, it.tok1);
+}
 // Gated DeltaNet: lambda[1:C] = exp(c_C) of chunk c of a run (a whole warp).
 __device__ __forceinline__ float chunk_decay(const Params& p, const Item& it, int c) {
-    const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
-    const float2 cc = gate_prefix(gb, p.g_st, it.tok0 + c * kChunk, it.tok1);
-    return expf(__shfl_sync(0xffffffffu, cc.y, 31));
+    return expf(gate_sum(chunk_gates(p, it, c, c + 1)));
+}
+// Gated DeltaNet, a whole warp: from the chunk's log decays (gate_load), the factors of its
+// token row 16 q + (lane & 15): lambda[1:l] = exp(c_l) (-> .x) and lambda[l+1:C] =
+// exp(c_C - c_l) (-> .y).
+__device__ __forceinline__ float2 row_decays(float2 g, int q) {
+    const int lane = threadIdx.x & 31;
+    const float2 c = gate_scan(g);
+    const int t = 16 * q + (lane & 15);
+    const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1), cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
+    const float cC = __shfl_sync(0xffffffffu, c.y, 31);
+    const float ct = (t & 1) ? cy : cx;
+    return make_float2(expf(ct), expf(cC - ct));
 }
 
 template <bool GATED>
@@ -527,8 +543,12 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 mbar_arrive(&bars[B_OFREE + 1]);
             }
         }
+        // Gated DeltaNet: the chunk's log decays are loaded one chunk ahead
+        float2 g_next = GATED ? chunk_gates(p, it, 0, nch) : make_float2(0.f, 0.f);
         for (int r = 0; r < nch; ++r) {
             uint8_t* stage = smem + (r % L::NA) * A_STAGE;
+            const float2 g_cur = g_next;
+            if constexpr (GATED) g_next = chunk_gates(p, it, r + 1, nch);
             // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's q/k stage,
             // once the stage holds the chunk (its previous chunk's products are done)
             if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % L::NA], (r / L::NA) & 1,
@@ -548,14 +568,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 // W^T has read K: the chunk's Q rows become Q<- (lambda[1:l] q_l, read by the
                 // output product) and its K rows K-> (lambda[l+1:C] k_l, read by the state
                 // update), with lambda[1:l] = exp(c_l) and lambda[l+1:C] = exp(c_C - c_l)
-                const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
-                const float2 c = gate_prefix(gb, p.g_st, it.tok0 + r * kChunk, it.tok1);
-                const int t = 16 * q + (lane & 15);
-                const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1), cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
-                const float cC = __shfl_sync(0xffffffffu, c.y, 31);
-                const float ct = (t & 1) ? cy : cx;
-                scale_token_rows(stage + a_q(r), 16384, q, expf(ct));
-                scale_token_rows(stage + A_K, 8192, q, expf(cC - ct));
+                const float2 f = row_decays(g_cur, q);
+                scale_token_rows(stage + a_q(r), 16384, q, f.x);
+                scale_token_rows(stage + A_K, 8192, q, f.y);
             }
             fence_async_smem();
             __syncwarp();
@@ -631,9 +646,15 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[B_SBF]);
+        // Gated DeltaNet: the log decays of the chunk after next, loaded one iteration early
+        float2 g_pre = GATED ? chunk_gates(p, it, 1, nch) : make_float2(0.f, 0.f);
         for (int r = 0; r < nch; ++r) {
             // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
-            const float lam_next = (GATED && r + 1 < nch) ? chunk_decay(p, it, r + 1) : 1.f;
+            float lam_next = 1.f;
+            if constexpr (GATED) {
+                lam_next = expf(gate_sum(g_pre));
+                g_pre = chunk_gates(p, it, r + 2, nch);
+            }
             // Z^T -> bf16 (A operand of the S^T update and of O^T += Z^T P^T), once the
             // previous chunk's O^T += Z^T P^T has read the previous one
             DN_TR(warp == 0, r, 27);

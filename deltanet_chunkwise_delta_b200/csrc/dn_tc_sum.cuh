@@ -378,8 +378,12 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
             // ------------------------------------------------------------ -W rows
             const int q = warp - 8;
             const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+            // Gated DeltaNet: the chunk's log decays are loaded one chunk ahead
+            float2 g_next = GATED ? tc::chunk_gates(p, it, 0, nch) : make_float2(0.f, 0.f);
             for (int r = 0; r < nch; ++r) {
                 uint8_t* stage = smem + (r % NA) * A_STAGE;
+                const float2 g_cur = g_next;
+                if constexpr (GATED) g_next = tc::chunk_gates(p, it, r + 1, nch);
                 // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's k stage,
                 // once the stage holds the chunk (its previous chunk's products are done)
                 if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
@@ -396,13 +400,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 if constexpr (GATED) {
                     // W^T has read K: the chunk's K rows become K-> = lambda[l+1:C] k_l
                     // (exp(c_C - c_l)), read by both state updates
-                    const float* gb = p.g + it.b * p.g_sb + it.head * p.g_sh;
-                    const float2 c = gate_prefix(gb, p.g_st, it.tok0 + r * kChunk, it.tok1);
-                    const int t = 16 * q + (lane & 15);
-                    const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1);
-                    const float cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
-                    const float cC = __shfl_sync(0xffffffffu, c.y, 31);
-                    tc::scale_token_rows(stage + A_K, 8192, q, expf(cC - ((t & 1) ? cy : cx)));
+                    tc::scale_token_rows(stage + A_K, 8192, q, tc::row_decays(g_cur, q).y);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -473,9 +471,15 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
+                // Gated DeltaNet: the log decays of the chunk after next, loaded one iteration early
+                float2 g_pre = GATED ? tc::chunk_gates(p, it, 1, nch) : make_float2(0.f, 0.f);
                 for (int r = 0; r < nch; ++r) {
                     // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
-                    const float lam_next = (GATED && r + 1 < nch) ? tc::chunk_decay(p, it, r + 1) : 1.f;
+                    float lam_next = 1.f;
+                    if constexpr (GATED) {
+                        lam_next = expf(gate_sum(g_pre));
+                        g_pre = tc::chunk_gates(p, it, r + 2, nch);
+                    }
                     // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
                     // the state update)
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
