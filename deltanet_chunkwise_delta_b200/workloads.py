@@ -86,6 +86,9 @@ def _workloads() -> dict:
         "layer_1p3b": Workload("layer_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False),
         "long_65k": Workload("long_65k", 1, 65536, 16, 128, 128, torch.bfloat16, True),
         "ctx_1m": Workload("ctx_1m", 1, 1 << 20, 8, 128, 128, torch.bfloat16, False),
+        # the first 131,072 tokens of the 1M-token context: the same kernels at one eighth of
+        # the size, small enough for a profiler capture
+        "ctx_128k": Workload("ctx_128k", 1, 1 << 17, 8, 128, 128, torch.bfloat16, False),
         "varlen_32": Workload("varlen_32", 1, sum(vl), 16, 128, 128, torch.bfloat16, True, vl),
         "gdn_1p3b": Workload("gdn_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False, gated=True),
         "gdn_65k": Workload("gdn_65k", 1, 65536, 16, 128, 128, torch.bfloat16, True, gated=True),
