@@ -62,7 +62,8 @@ def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
     es = 2 if w.dtype == torch.bfloat16 else 4
     th = w.tokens * w.H
     # Gated Delta Product: k, v and beta have nh rows per token
-    b = th * (es * ((1 + w.nh) * w.dk + (w.nh + 1) * w.dv) + 4 * w.nh + (4 if w.gated else 0))
+    b = th * (es * ((1 + w.nh) * w.dk + (w.nh + 1) * w.dv) + 4 * w.nh + (4 if w.gated else 0)
+              + (4 * w.dk if w.kda else 0))
     st = w.n_seq * w.H * w.dk * w.dv * 4
     if w.init_state:
         b += st
@@ -279,7 +280,10 @@ def run_b200(args, w: wl.Workload):
     stream = torch.cuda.current_stream(device)
 
     def call(d, o, f):
-        if w.nh > 1:
+        if w.kda:
+            dn.kda_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["initial_state"],
+                       d["cu_seqlens"], out=o, final_state=f, stream=stream)
+        elif w.nh > 1:
             dn.gated_deltaproduct_fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], w.nh,
                                       d["initial_state"], d["cu_seqlens"], out=o, final_state=f,
                                       stream=stream)
@@ -335,7 +339,7 @@ def run_b200(args, w: wl.Workload):
     alg_bytes = algorithmic_bytes(w)
     # DeltaNet and Gated DeltaNet (one write per token) at d_k = d_v = 128 run on the
     # tensor-core kernels
-    tc_path = w.nh == 1 and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+    tc_path = w.nh == 1 and not w.kda and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
     # the tensor-core boundary kernel moves q, k, v, o and the states (beta is read by the
     # UT pre-pass); the mma.sync boundary kernel reads beta (and g) itself
     kernel_bytes = alg_bytes - (4.0 * w.tokens * w.H if tc_path else 0.0)
@@ -466,7 +470,8 @@ def run_b200(args, w: wl.Workload):
                    "chunks_first_segment": s0,
                    "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{ws}",
                    "variant": (f"gated delta product, n_h = {w.nh}" if w.nh > 1 else
-                               "gated DeltaNet" if w.gated else "DeltaNet")},
+                               "gated DeltaNet" if w.gated else
+                               "Kimi Delta Attention" if w.kda else "DeltaNet")},
         "tflops": tflops,
         "tflops_unit": "algorithmic TFLOP/s (6Cd^2 + 5C^2d + C^3/3 per chunk-head)",
         "roofline": roofline,

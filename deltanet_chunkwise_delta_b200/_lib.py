@@ -26,7 +26,7 @@ EXPORTED = ("deltanet_fwd", "deltanet_fwd_ex", "gated_deltanet_fwd", "gated_delt
             "deltanet_status_string",
             "deltanet_get_error", "deltanet_release_workspace", "deltanet_last_schedule",
             "deltanet_fwd_noalloc", "deltanet_last_launches", "deltanet_set_kernel_events",
-            "deltanet_test_set_wait")
+            "deltanet_test_set_wait", "kda_fwd", "kda_fwd_ex")
 
 
 class DnTensor(ctypes.Structure):
@@ -79,6 +79,11 @@ def load(path: Optional[str] = None):
         lib.gated_deltaproduct_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int,
                                                   ctypes.c_int, P, P, ctypes.c_void_p,
                                                   ctypes.c_int]
+        lib.kda_fwd.restype = ctypes.c_int
+        lib.kda_fwd.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p]
+        lib.kda_fwd_ex.restype = ctypes.c_int
+        lib.kda_fwd_ex.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_void_p,
+                                   ctypes.c_int]
         lib.deltanet_fwd_states.restype = ctypes.c_int
         lib.deltanet_fwd_states.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, P, P, P,
                                             ctypes.c_void_p, ctypes.c_int]
@@ -154,6 +159,17 @@ def call_gated(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, fin
     return lib.gated_deltanet_fwd(*args, stream)
 
 
+def call_kda(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+             stream, seg_chunks: int = 0) -> int:
+    """Raw Kimi Delta Attention call: returns the dn_status code (no exception)."""
+    lib = load()
+    ds = [describe(t) for t in (q, k, v, beta, g, initial_state, cu_seqlens, out, final_state)]
+    args = [_ref(x) for x in ds[:7]] + [int(chunk_size)] + [_ref(x) for x in ds[7:]]
+    if seg_chunks:
+        return lib.kda_fwd_ex(*args, stream, int(seg_chunks))
+    return lib.kda_fwd(*args, stream)
+
+
 def _stream_handle(device, stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -212,6 +228,32 @@ def gated_deltanet_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: 
         final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     st = call_gated(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     _stream_handle(q.device, stream), seg_chunks)
+    if st != DN_OK:
+        raise DeltaNetError(st, status_string(st))
+    return out, final_state
+
+
+def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.Tensor,
+            g: torch.Tensor, initial_state: Optional[torch.Tensor] = None,
+            cu_seqlens: Optional[torch.Tensor] = None, chunk_size: int = 64,
+            out: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+            output_final_state: bool = True, stream=None, seg_chunks: int = 0):
+    """Kimi Delta Attention forward on CUDA tensors through the C ABI.
+
+    As ``deltanet_fwd``, plus ``g`` [B, T, H, d_k] fp32: the decay of every key channel
+    as its natural log (the state update is S <- (I - beta k^T k) Diag(a) S + beta k^T v).
+    """
+    if not q.is_cuda:
+        raise ValueError("kda_fwd runs on CUDA tensors only")
+    B, T, H, _ = q.shape
+    dk, dv = q.shape[3], v.shape[3]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = call_kda(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                  _stream_handle(q.device, stream), seg_chunks)
     if st != DN_OK:
         raise DeltaNetError(st, status_string(st))
     return out, final_state

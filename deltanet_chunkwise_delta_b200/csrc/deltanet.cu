@@ -247,22 +247,25 @@ struct Dims {
     bool varlen;
 };
 
-template <typename E, int DK, int DV, int STAGES, bool GATED>
+template <typename E, int DK, int DV, int STAGES, bool GATED, bool KDA = false>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
     // bf16 DeltaNet and Gated DeltaNet with d_k = d_v = 128 run on the tensor-core (tcgen05)
     // kernels (with or without the chunk-start states); the Gated Delta Product (several
     // writes per token) and the other shapes on the mma.sync chain kernels
-    constexpr bool kTcShape = std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
+    // (Kimi Delta Attention, a decay per key channel, runs on the mma.sync chain kernels)
+    constexpr bool kTcShape = !KDA && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
     const bool use_tc = kTcShape && p.nh <= 1;
-    using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED>;
-    using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED>;
-    using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED>;
+    using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED, KDA>;
+    using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED, KDA>;
+    using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED, KDA>;
+    static_assert(LC::TOTAL <= 232448 && LH::TOTAL <= 232448 && LP::TOTAL <= 232448,
+                  "chain kernel shared memory");
     const int smemC = LC::TOTAL;
     const int smemA = LH::TOTAL > LP::TOTAL ? LH::TOTAL : LP::TOTAL;
     const int smemS8 = scan_smem_bytes<DK, 8>(), smemS16 = scan_smem_bytes<DK, 16>();
-    auto* kC = k_boundary<E, DK, DV, STAGES, GATED>;
-    auto* kA = k_summary<E, DK, DV, STAGES, GATED>;
+    auto* kC = k_boundary<E, DK, DV, STAGES, GATED, KDA>;
+    auto* kA = k_summary<E, DK, DV, STAGES, GATED, KDA>;
     auto* kS8 = k_scan<DK, DV, 8>;
     auto* kS16 = k_scan<DK, DV, 16>;
     auto* kCt = tc::k_tc_chain<GATED>;
@@ -455,6 +458,20 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     return DN_OK;
 }
 
+// Kimi Delta Attention (a log decay per key channel): bf16 only; one load stage at d_k = 128
+// (its per-channel gate tile takes the room of the second)
+dn_status dispatch_kda(Params& p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
+                       const int* cup) {
+    const int64_t dk = d.dk, dv = d.dv;
+    if (dk == 128 && dv == 128)
+        return launch<__nv_bfloat16, 128, 128, 1, false, true>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 128 && dv == 64)
+        return launch<__nv_bfloat16, 128, 64, 1, false, true>(p, d, dev, sms, stream, forced_s, cup);
+    if (dk == 64 && dv == 128)
+        return launch<__nv_bfloat16, 64, 128, 2, false, true>(p, d, dev, sms, stream, forced_s, cup);
+    return launch<__nv_bfloat16, 64, 64, 2, false, true>(p, d, dev, sms, stream, forced_s, cup);
+}
+
 template <bool GATED>
 dn_status dispatch(Params& p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                    const int* cup, int32_t dt) {
@@ -469,14 +486,16 @@ dn_status dispatch(Params& p, const Dims& d, int dev, int sms, cudaStream_t stre
     return launch<__nv_bfloat16, 64, 64, 2, GATED>(p, d, dev, sms, stream, forced_s, cup);
 }
 
-// gate: Gated DeltaNet's log decay [B, T, H] fp32, or null for DeltaNet.
+// gate: Gated DeltaNet's log decay [B, T, H] fp32, or null for DeltaNet; with kda, Kimi
+// Delta Attention's log decay per key channel [B, T, H, d_k] fp32.
 // nh: delta-rule writes per token (Gated Delta Product; 1 otherwise): k, v and beta hold
 // T * nh rows, q, gate and out T rows, cu_seqlens counts tokens.
 // cs: chunk-start states [rows, H, d_k, d_v] fp32, or null.
 dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                    const dn_tensor* beta, const dn_tensor* gate, const dn_tensor* s0,
                    const dn_tensor* cu, int chunk, dn_tensor* out, dn_tensor* sT,
-                   void* stream_ptr, int forced_s, int nh = 1, dn_tensor* cs = nullptr) {
+                   void* stream_ptr, int forced_s, int nh = 1, dn_tensor* cs = nullptr,
+                   bool kda = false) {
     if (!q || !k || !v || !beta || !out) return DN_ERR_INVALID_ARG;
     if (q->ndim != 4 || k->ndim != 4 || v->ndim != 4 || out->ndim != 4) return DN_ERR_INVALID_ARG;
     if (forced_s < 0 || nh < 1 || (nh > 1 && !gate)) return DN_ERR_INVALID_ARG;
@@ -500,7 +519,13 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
         if (beta->stride[i] < 0) return DN_ERR_INVALID_ARG;
     if (numel(beta) > 0 && (!beta->data || (reinterpret_cast<uintptr_t>(beta->data) & 3)))
         return DN_ERR_INVALID_ARG;
-    if (gate) {
+    if (kda) {
+        // one log decay per key channel, rows of d_k fp32 read in 16-byte pieces
+        const int64_t gk[4] = {B, T, H, dk};
+        if (!gate || nh != 1 || !shape_eq(gate, 4, gk) || gate->dtype != DN_F32) return DN_ERR_INVALID_ARG;
+        if (!token_tensor_ok(gate)) return DN_ERR_INVALID_ARG;
+        if (dt != DN_BF16) return DN_ERR_UNSUPPORTED;
+    } else if (gate) {
         if (!shape_eq(gate, 3, gd) || gate->dtype != DN_F32) return DN_ERR_INVALID_ARG;
         for (int i = 0; i < 3; ++i)
             if (gate->stride[i] < 0) return DN_ERR_INVALID_ARG;
@@ -587,6 +612,7 @@ dn_status fwd_impl(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
     Dims d{B, Tw, H, dk, dv, N, varlen};  // items count k/v/beta rows
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     const int* cup = varlen ? static_cast<const int*>(cu->data) : nullptr;
+    if (kda) return dispatch_kda(p, d, dev, sms, stream, forced_s, cup);
     if (gate) return dispatch<true>(p, d, dev, sms, stream, forced_s, cup, dt);
     return dispatch<false>(p, d, dev, sms, stream, forced_s, cup, dt);
 }
@@ -659,6 +685,23 @@ dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, cons
     if (!g) return DN_ERR_INVALID_ARG;
     return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
                     stream, seg_chunks, n_h);
+}
+
+dn_status kda_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v, const dn_tensor* beta,
+                  const dn_tensor* g, const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                  int chunk_size, dn_tensor* out, dn_tensor* final_state, void* stream) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, 0, 1, nullptr, true);
+}
+
+dn_status kda_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v, const dn_tensor* beta,
+                     const dn_tensor* g, const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                     int chunk_size, dn_tensor* out, dn_tensor* final_state, void* stream,
+                     int seg_chunks) {
+    if (!g) return DN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, beta, g, initial_state, cu_seqlens, chunk_size, out, final_state,
+                    stream, seg_chunks, 1, nullptr, true);
 }
 
 const char* deltanet_status_string(dn_status s) {

@@ -28,6 +28,21 @@
 // are done), the readout factor into the rows of Q S, and lambda[1:C] into the
 // state registers.
 //
+// Kimi Delta Attention (same page, section "Kimi Delta Attention (KDA)", its
+// complete per-chunk algorithm) decays every key channel c by its own a_t[c] =
+// exp(g_t[c]).  With G_l = g_1 + ... + g_l (per channel, within the chunk):
+//   L[l][m] = sum_c k_l[c] k_m[c] exp(G_l[c] - G_m[c])  (m < l),  A[l][m] the same
+//   with q_l (m <= l);  (I + B_r L) T_r = B_r,  U_r = T_r V_r,  W_r = T_r K<-_r,
+//   Z_r = U_r - W_r S_r,  O_r = Q<-_r S_r + A Z_r,  S_{r+1} = Diag(lambda[1:C]) S_r
+//   + K->_r^T Z_r,  with q<-_l = exp(G_l) o q_l, k<-_l = exp(G_l) o k_l,
+//   k->_l = exp(G_C - G_l) o k_l, lambda[1:C] = exp(G_C).
+// L and A are formed block by block of 16 rows against the block's first row s:
+// exp(G_l - G_m) = exp(G_l - G_s) exp(G_s - G_m), so each product takes the rows
+// k_l o exp(G_l - G_s) (q_l o exp(G_l - G_s)) and k_m o exp(G_s - G_m).  For rows
+// before the block both factors are products of decays (at most 1 for a_t <= 1);
+// inside the block the second one grows with at most 15 tokens' decay, which keeps
+// it in range for |g| < 5.8 per token and channel.
+//
 // The state stays in registers (fp32) for the whole run; W, U, Z, T and the
 // masked scores never leave shared memory.  Only q, k, v, beta are read and o
 // written per chunk.  Loads of chunk r+1 are issued before chunk r is computed.
@@ -41,7 +56,8 @@ namespace dn {
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false>
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false,
+          bool KDA = false>
 struct ChainSmem {
     static constexpr int ES = sizeof(E);
     static constexpr int Q_BYTES = kChunk * DK * ES;
@@ -56,16 +72,24 @@ struct ChainSmem {
     static constexpr int OFF_K = OFF_Q + (HAS_Q ? STAGES * Q_BYTES : 0);
     static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
     static constexpr int OFF_BETA = OFF_V + (HAS_V ? STAGES * V_BYTES : 0);
-    static constexpr int OFF_GATE = OFF_BETA + STAGES * kChunk * 4;  // g per stage
-    static constexpr int OFF_DECAY = OFF_GATE + (GATED ? STAGES * kChunk * 4 : 0);
-    static constexpr int OFF_SOLVE = OFF_DECAY + (GATED ? 4 * kChunk * 4 : 0);
+    // g per stage: one per token (GATED), or one per (token, key channel) as an fp32 tile
+    // of 64 rows x DK, row-major (KDA; made the chunk's running sums in place)
+    static constexpr int GATE_BYTES = KDA ? kChunk * DK * 4 : (GATED ? kChunk * 4 : 0);
+    static constexpr int OFF_GATE = OFF_BETA + STAGES * kChunk * 4;
+    static constexpr int OFF_DECAY = OFF_GATE + STAGES * GATE_BYTES;
+    // GATED: running sum, lambda[1:l], lambda[l+1:C], lambda[1:C]; KDA: lambda[1:C] per channel
+    static constexpr int OFF_SOLVE = OFF_DECAY + (GATED ? 4 * kChunk * 4 : (KDA ? DK * 4 : 0));
     static constexpr int OFF_T = align_up(OFF_SOLVE + UNION_BYTES, 128);
     static constexpr int OFF_W = OFF_T + kChunk * kChunk * ES;
     static constexpr int OFF_X = OFF_W + kChunk * DK * ES;
     static constexpr int OFF_Z = OFF_X + DK * NX * ES;
     static constexpr int OFF_P = OFF_Z + kChunk * NX * ES;
     static constexpr int OFF_T2 = OFF_P + (HAS_Q ? kChunk * kChunk * ES : 0);
-    static constexpr int TOTAL = OFF_T2 + (GATED ? kChunk * kChunk * ES : 0);
+    // KDA: scratch rows of K scaled by decay ratios (one 16-row block's operands at a time,
+    // later K<-), and the block's left operands [K rows; Q rows] (2 x 16 rows)
+    static constexpr int OFF_R = OFF_T2 + (GATED ? kChunk * kChunk * ES : 0);
+    static constexpr int OFF_LQ = OFF_R + (KDA ? kChunk * DK * ES : 0);
+    static constexpr int TOTAL = OFF_LQ + (KDA ? 2 * 16 * DK * ES : 0);
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -176,10 +200,12 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
 }
 
 // Runs one work item.  mode selects start state, output and destination.
-template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false>
+template <typename E, int DK, int NX, bool HAS_V, bool HAS_Q, int STAGES, bool GATED = false,
+          bool KDA = false>
 __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int mode,
                                             char* smem) {
-    using L = ChainSmem<E, DK, NX, HAS_V, HAS_Q, STAGES, GATED>;
+    using L = ChainSmem<E, DK, NX, HAS_V, HAS_Q, STAGES, GATED, KDA>;
+    static_assert(!(GATED && KDA), "one kind of gate");
     using SW = Swz<E>;
     constexpr int MT_S = DK / 64;  // 16-row tiles of the state per warp
     constexpr int NT_X = NX / 16;  // 8-column tiles per warp (NX / 2 columns)
@@ -196,6 +222,11 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     float* lam_r = lam_l + kChunk;
     float* lam_c = lam_r + kChunk;
     E* Ts2 = reinterpret_cast<E*>(smem + L::OFF_T2);
+    // KDA: the per-channel gate tile of each stage, lambda[1:C] per channel, scratch rows
+    float* gtile = reinterpret_cast<float*>(smem + L::OFF_GATE);
+    float* lamc_k = reinterpret_cast<float*>(smem + L::OFF_DECAY);
+    E* Rs = reinterpret_cast<E*>(smem + L::OFF_R);
+    E* LQs = reinterpret_cast<E*>(smem + L::OFF_LQ);
     float* Af = reinterpret_cast<float*>(smem + L::OFF_SOLVE);
     float* Nf = Af + kChunk * L::SOLVE_LD;
     float* Xt = Nf + kChunk * L::SOLVE_LD;
@@ -255,7 +286,7 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     const E* vg = static_cast<const E*>(p.v) + it.b * p.v_sb + it.head * p.v_sh;
     E* og = static_cast<E*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
     const float* bg = p.beta + it.b * p.b_sb + it.head * p.b_sh;
-    const float* gg = GATED ? p.g + it.b * p.g_sb + it.head * p.g_sh : nullptr;
+    const float* gg = (GATED || KDA) ? p.g + it.b * p.g_sb + it.head * p.g_sh : nullptr;
     // Gated Delta Product: item token ranges count virtual steps, nsub per token
     const int nsub = (GATED && p.nh > 1) ? p.nh : 1;
 
@@ -288,6 +319,18 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
             const bool ok = tid < rows;
             cp_async4(smem_addr(betas + stg * kChunk + tid), ok ? bg + (t0 + tid) * p.b_st : bg,
                       ok ? 4 : 0);
+        }
+        if constexpr (KDA) {
+            // the chunk's log decays per (token, key channel): 64 rows x DK, rows past the
+            // run read g = 0 (identity steps)
+            float* dst = gtile + stg * (L::GATE_BYTES / 4);
+            constexpr int CPR = DK / 4;
+            for (int idx = tid; idx < kChunk * CPR; idx += kThreads) {
+                const int rr = idx / CPR, c = idx % CPR;
+                const bool ok = rr < rows;
+                const float* src = ok ? gg + (int64_t)(t0 + rr) * p.g_st + 4 * c : gg;
+                cp_async16(smem_addr(dst + rr * DK + 4 * c), src, ok ? 16 : 0);
+            }
         }
         if (GATED && warp == 0) {
             // warp 0 loads all 64 gates (two per lane: it scans them itself after its own
@@ -376,6 +419,75 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         for (int m = 0; m < MT_S; ++m) store_frag<NT_X, NX>(Xb, s_r0 + 16 * m, x_c0, s[m], 1.f);
         __syncthreads();
 
+        if constexpr (KDA) {
+            float* G = gtile + stg * (L::GATE_BYTES / 4);
+            E* Kw = const_cast<E*>(Kc);
+            E* Qw = const_cast<E*>(Qc);
+            // (b1) the chunk's running sums per key channel, in place, and lambda[1:C]
+            for (int c = tid; c < DK; c += kThreads) {
+                float acc = 0.f;
+                for (int l = 0; l < kChunk; ++l) {
+                    acc += G[l * DK + c];
+                    G[l * DK + c] = acc;
+                }
+                lamc_k[c] = expf(acc);
+            }
+            __syncthreads();
+            // (b2) rows 16 b .. 16 b + 15 of A = B L (fp32, strict lower) and of the
+            // readout scores P (inclusive), against reference row s = 16 b
+#pragma unroll 1
+            for (int b = 0; b < 4; ++b) {
+                const int s = 16 * b, ncol = s + 16;
+                for (int idx = tid; idx < ncol * DK; idx += kThreads) {
+                    const int m = idx / DK, c = idx % DK;
+                    const int o = SW::template off<DK>(m, c);
+                    Rs[o] = to_e<E>(float(Kc[o]) * expf(G[s * DK + c] - G[m * DK + c]));
+                }
+                for (int idx = tid; idx < 16 * DK; idx += kThreads) {
+                    const int lr = idx / DK, c = idx % DK, l = s + lr;
+                    const float f = expf(G[l * DK + c] - G[s * DK + c]);
+                    const int o = SW::template off<DK>(l, c), ol = SW::template off<DK>(lr, c);
+                    LQs[ol] = to_e<E>(float(Kc[o]) * f);
+                    if (HAS_Q) LQs[16 * DK + ol] = to_e<E>(float(Qc[o]) * f);
+                }
+                // the block's rows right of its last column are zero in both
+                for (int idx = tid; idx < 16 * (kChunk - ncol); idx += kThreads) {
+                    const int row = s + idx / (kChunk - ncol), col = ncol + idx % (kChunk - ncol);
+                    Af[row * L::SOLVE_LD + col] = 0.f;
+                    if (HAS_Q) Ps[SW::template off<kChunk>(row, col)] = to_e<E>(0.f);
+                }
+                __syncthreads();
+                const int ntile = b + 1;
+                if (warp < (HAS_Q ? 2 : 1) * ntile) {
+                    const int mat = warp / ntile, j = warp % ntile;
+                    float acc[2][4];
+                    zero_frag(acc);
+                    warp_gemm<DK, 2, DK, false, DK, false>(acc, LQs + mat * 16 * DK, 0, Rs, 16 * j);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int row = s + g8 + 8 * (e >> 1);
+                            const int col = 16 * j + 8 * nt + 2 * t4 + (e & 1);
+                            if (mat == 0) Af[row * L::SOLVE_LD + col] = col < row ? bc[row] * acc[nt][e] : 0.f;
+                            else acc[nt][e] = col > row ? 0.f : acc[nt][e];
+                        }
+                    if (mat == 1) store_frag<2, kChunk>(Ps, s, 16 * j, acc, 1.f);
+                }
+                __syncthreads();
+            }
+            // (b3) K<- = exp(G) o K into the scratch rows (the W factor); K becomes K->
+            // (exp(G_C - G) o K, read by the state update) and Q becomes Q<- (exp(G) o Q)
+            for (int idx = tid; idx < kChunk * DK; idx += kThreads) {
+                const int l = idx / DK, c = idx % DK;
+                const int o = SW::template off<DK>(l, c);
+                const float gl = G[l * DK + c], gC = G[(kChunk - 1) * DK + c];
+                const float kv = float(Kc[o]);
+                Rs[o] = to_e<E>(kv * expf(gl));
+                Kw[o] = to_e<E>(kv * expf(gC - gl));
+                if (HAS_Q) Qw[o] = to_e<E>(float(Qc[o]) * expf(gl));
+            }
+        } else {
         // (b) A = B L (strict lower, fp32) and, with output, P = (Q K^T) o M_c
         {
             float acc[4][4];
@@ -417,6 +529,7 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
                 store_frag<4, kChunk>(Ps, 16 * mt, 32 * nh, acc, 1.f);
             }
         }
+        }
         __syncthreads();
 
         // (c) T = (I + B L)^{-1} B
@@ -430,8 +543,8 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
         {
             float w[NT_W][4];
             zero_frag(w);
-            warp_gemm<kChunk, NT_W, kChunk, false, DK, true>(w, GATED ? Ts2 : Ts, 16 * mt, Kc,
-                                                             nh * (DK / 2));
+            warp_gemm<kChunk, NT_W, kChunk, false, DK, true>(w, GATED ? Ts2 : Ts, 16 * mt,
+                                                             KDA ? Rs : Kc, nh * (DK / 2));
             store_frag<NT_W, DK>(Ws, 16 * mt, nh * (DK / 2), w, -1.f);
             if (HAS_V) warp_gemm<kChunk, NT_X, kChunk, false, NX, true>(z, Ts, 16 * mt, Vc, x_c0);
         }
@@ -470,6 +583,15 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
                 for (int nt = 0; nt < NT_X; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) s[m][nt][e] *= fc;
+        }
+        if constexpr (KDA) {
+            // the state's key rows decay by lambda[1:C] of their channel
+#pragma unroll
+            for (int m = 0; m < MT_S; ++m)
+#pragma unroll
+                for (int nt = 0; nt < NT_X; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[m][nt][e] *= lamc_k[s_r0 + 16 * m + g8 + 8 * (e >> 1)];
         }
         __syncthreads();
 
@@ -516,18 +638,18 @@ __device__ __forceinline__ void run_segment(const Params& p, const Item& it, int
     }
 }
 
-template <typename E, int DK, int DV, int STAGES, bool GATED>
+template <typename E, int DK, int DV, int STAGES, bool GATED, bool KDA = false>
 __global__ void __launch_bounds__(kThreads, 1) k_boundary(Params p) {
     extern __shared__ __align__(128) char smem[];
     const int n = count_C(p.sched);
     for (int i = blockIdx.x; i < n; i += gridDim.x) {
         const Item it = item_C(p.sched, i);
-        run_segment<E, DK, DV, true, true, STAGES, GATED>(p, it, kModeOut, smem);
+        run_segment<E, DK, DV, true, true, STAGES, GATED, KDA>(p, it, kModeOut, smem);
         __syncthreads();
     }
 }
 
-template <typename E, int DK, int DV, int STAGES, bool GATED>
+template <typename E, int DK, int DV, int STAGES, bool GATED, bool KDA = false>
 __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
     extern __shared__ __align__(128) char smem[];
     const int n = count_A(p.sched);
@@ -536,13 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_summary(Params p) {
         const Item it = item_A(p.sched, i, mode);
         if (mode == kModeHP) {
             // both maps of the segment, one after the other
-            run_segment<E, DK, DV, true, false, STAGES, GATED>(p, it, kModeH, smem);
+            run_segment<E, DK, DV, true, false, STAGES, GATED, KDA>(p, it, kModeH, smem);
             __syncthreads();
-            run_segment<E, DK, DK, false, false, STAGES, GATED>(p, it, kModeP, smem);
+            run_segment<E, DK, DK, false, false, STAGES, GATED, KDA>(p, it, kModeP, smem);
         } else if (mode == kModeP) {
-            run_segment<E, DK, DK, false, false, STAGES, GATED>(p, it, mode, smem);
+            run_segment<E, DK, DK, false, false, STAGES, GATED, KDA>(p, it, mode, smem);
         } else {
-            run_segment<E, DK, DV, true, false, STAGES, GATED>(p, it, mode, smem);
+            run_segment<E, DK, DV, true, false, STAGES, GATED, KDA>(p, it, mode, smem);
         }
         __syncthreads();
     }

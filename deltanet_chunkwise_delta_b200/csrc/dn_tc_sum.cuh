@@ -383,6 +383,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
             for (int r = 0; r < nch; ++r) {
                 uint8_t* stage = smem + (r % NA) * A_STAGE;
                 const float2 g_cur = g_next;
+                (void)g_cur;
                 if constexpr (GATED) g_next = tc::chunk_gates(p, it, r + 1, nch);
                 // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's k stage,
                 // once the stage holds the chunk (its previous chunk's products are done)

@@ -27,6 +27,9 @@ Recipe (all on the CPU, so every consumer sees bit-identical inputs):
     (GDP)") draw n_h key, value and beta rows per token (substep-major, i.e.
     k [B, T n_h, H, d]) where the others draw one; q, the initial state and g
     keep one row per token;
+  * Kimi Delta Attention workloads (same page, section "Kimi Delta Attention
+    (KDA)") draw one log decay per key channel instead, g = logsigmoid(z + 4),
+    z ~ N(0,1) in fp32, shape [B, T, H, d_k], after everything else;
   * variable-length batches draw 32 lengths with ``numpy.random.default_rng(seed)``
     log-uniformly in [ln 128, ln 32768], L = floor(exp(u)), packed in draw order.
 """
@@ -56,6 +59,7 @@ class Workload:
     chunk: int = 64
     gated: bool = False               # Gated DeltaNet: draw the log decay g
     nh: int = 1                       # Gated Delta Product: writes per token (gated)
+    kda: bool = False                 # Kimi Delta Attention: a log decay per key channel
 
     @property
     def n_seq(self) -> int:
@@ -94,6 +98,7 @@ def _workloads() -> dict:
         "gdn_65k": Workload("gdn_65k", 1, 65536, 16, 128, 128, torch.bfloat16, True, gated=True),
         "gdp_1p3b": Workload("gdp_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False,
                              gated=True, nh=2),
+        "kda_1p3b": Workload("kda_1p3b", 8, 2048, 16, 128, 128, torch.bfloat16, False, kda=True),
     }
 
 
@@ -101,13 +106,15 @@ WORKLOADS = _workloads()
 
 
 def custom(B, T, H, dk, dv, dtype=torch.bfloat16, init_state=False, seqlens=None,
-           name="custom", gated=False, nh=1) -> Workload:
+           name="custom", gated=False, nh=1, kda=False) -> Workload:
     if seqlens is not None:
         seqlens = tuple(int(x) for x in seqlens)
         B, T = 1, sum(seqlens)
     if nh > 1 and not gated:
         raise ValueError("several writes per token is the gated product")
-    return Workload(name, B, T, H, dk, dv, dtype, init_state, seqlens, gated=gated, nh=nh)
+    if kda and gated:
+        raise ValueError("one kind of gate")
+    return Workload(name, B, T, H, dk, dv, dtype, init_state, seqlens, gated=gated, nh=nh, kda=kda)
 
 
 def _draw_tokens(gen, B, T, H, d, dtype, normalise):
@@ -149,6 +156,9 @@ def generate(w: Workload, seed: int = 0, beta_mode: str = "sigmoid") -> dict:
     g = None
     if w.gated:
         z = torch.randn((w.B, w.T, w.H), generator=gen, dtype=torch.float32)
+        g = torch.nn.functional.logsigmoid(z + 4.0)
+    elif w.kda:
+        z = torch.randn((w.B, w.T, w.H, w.dk), generator=gen, dtype=torch.float32)
         g = torch.nn.functional.logsigmoid(z + 4.0)
     return {"q": q, "k": k, "v": v, "beta": beta, "initial_state": s0,
             "cu_seqlens": w.cu_seqlens(), "g": g}

@@ -218,6 +218,35 @@ dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, cons
                                     dn_tensor* final_state, void* stream, int seg_chunks);
 
 /*
+ * kda_fwd -- Kimi Delta Attention forward ("Linear Attention, Visualized",
+ * section "Kimi Delta Attention (KDA)"): every key channel c decays by its own
+ * a_t[c] before the delta-rule correction,
+ *   S_t = (I - beta_t k_t^T k_t) Diag(a_t) S_{t-1} + beta_t k_t^T v_t,  o_t = q_t S_t,
+ * evaluated with the section's complete per-chunk algorithm (decayed K<- / K->
+ * / Q<- rows, channel-decayed L and A, S' = Diag(lambda[1:C]) S + K->^T Z).
+ *
+ * Arguments as gated_deltanet_fwd, except
+ *   g   [B, T, H, d_k] fp32, g[b, t, h, c] = ln a_t[c] for head h (channel c of
+ *       the key), last dim contiguous, 16-byte aligned rows and strides (it is
+ *       read in 16-byte pieces); finite, and |g| < 5.8 per token and channel
+ *       (within a chunk the kernel forms decay ratios over up to 15 tokens from
+ *       running sums of g, which stay in range under that bound).
+ * Supported: bf16 q/k/v/out with d_k, d_v in {64, 128}, dense or packed
+ * (cu_seqlens), split across SMs like deltanet_fwd.  Runs on the mma.sync chain
+ * kernels.  Pad rows of a last partial chunk carry g = 0 (identity steps).
+ * Returns DN_ERR_UNSUPPORTED for fp32 inputs or other head sizes.
+ */
+dn_status kda_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v, const dn_tensor* beta,
+                  const dn_tensor* g, const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                  int chunk_size, dn_tensor* out, dn_tensor* final_state, void* stream);
+
+/* kda_fwd with the seg_chunks override of deltanet_fwd_ex. */
+dn_status kda_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v, const dn_tensor* beta,
+                     const dn_tensor* g, const dn_tensor* initial_state, const dn_tensor* cu_seqlens,
+                     int chunk_size, dn_tensor* out, dn_tensor* final_state, void* stream,
+                     int seg_chunks);
+
+/*
  * deltanet_fwd_noalloc -- the forward pass without any device allocation.
  * (No counterpart on the pages: this is a deployment variant of deltanet_fwd.)
  *

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "deltanet.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b((?:gated_)?delta(?:net|product)_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:gated_)?delta(?:net|product)_\w+|kda_\w+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -220,3 +220,31 @@ def test_binding_host_logic():
         dn.gated_deltaproduct_fwd(x, x, x, b, b, 1)
     with pytest.raises(ValueError):
         dn.deltanet_fwd_states(x, x, x, b)
+
+
+def call_kda(lib, q, k, v, beta, g, s0=None, cu=None, chunk=64, out=None, sT=None):
+    r = lambda x: None if x is None else ctypes.byref(x)
+    return lib.kda_fwd(r(q), r(k), r(v), r(beta), r(g), r(s0), r(cu), chunk, r(out), r(sT), None)
+
+
+def test_kda_rejects_bad_gates_and_types(lib):
+    """Kimi Delta Attention takes one log decay per key channel [B, T, H, d_k] fp32 with
+    16-byte aligned rows, bf16 inputs only; all checked before the device."""
+    q, k, v, beta, s0, out, sT = good(dk=128, dv=128)
+    g_ok = desc([2, 100, 3, 128], L.DN_F32, 0x100000000 + 7 * 2**28)
+    assert call_kda(lib, q, k, v, beta, None, out=out) == L.DN_ERR_INVALID_ARG
+    g_scalar = desc([2, 100, 3], L.DN_F32, 0x100000000 + 7 * 2**28)
+    assert call_kda(lib, q, k, v, beta, g_scalar, out=out) == L.DN_ERR_INVALID_ARG
+    g_bf16 = desc([2, 100, 3, 128], L.DN_BF16, 0x100000000 + 7 * 2**28)
+    assert call_kda(lib, q, k, v, beta, g_bf16, out=out) == L.DN_ERR_INVALID_ARG
+    g_odd = desc([2, 100, 3, 128], L.DN_F32, 0x100000000 + 7 * 2**28,
+                 strides=[100 * 3 * 130, 3 * 130, 130, 1])   # rows not 16-byte multiples
+    assert call_kda(lib, q, k, v, beta, g_odd, out=out) == L.DN_ERR_INVALID_ARG
+    g_mis = desc([2, 100, 3, 128], L.DN_F32, 0x100000000 + 7 * 2**28 + 4)
+    assert call_kda(lib, q, k, v, beta, g_mis, out=out) == L.DN_ERR_INVALID_ARG
+    qf, kf, vf, bf, s0f, outf, sTf = good(dk=64, dv=64, dtype=L.DN_F32)
+    gf = desc([2, 100, 3, 64], L.DN_F32, 0x100000000 + 7 * 2**28)
+    assert call_kda(lib, qf, kf, vf, bf, gf, out=outf) == L.DN_ERR_UNSUPPORTED
+    # an output over the gate is refused like any other aliasing
+    out_on_g = desc([2, 100, 3, 128], L.DN_BF16, 0x100000000 + 7 * 2**28)
+    assert call_kda(lib, q, k, v, beta, g_ok, out=out_on_g) == L.DN_ERR_ALIAS
