@@ -15,9 +15,12 @@ constexpr int kThreads = 256;    // 8 warps per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 4096;  // segment-map slots (P, H, start state) per call
 // workspace bytes per (chunk, head) written by the UT pre-pass: T tile, then P tile, and for
-// Gated DeltaNet a third tile, T diag(lambda[1:l])
+// Gated DeltaNet a third tile T' = T diag(lambda[1:l]) (at kUnitT2), the decayed queries
+// Q<- = diag(lambda[1:l]) Q as two 64-channel boxes (at kUnitQL) and the chunk's row factors
+// F (at kUnitF: lambda[l+1:C] for rows l = 0..63, then lambda[1:C]), padded to 1 KB
 constexpr int kUnitBytes = 16384;
-constexpr int kUnitBytesGated = 24576;
+constexpr int kUnitT2 = 16384, kUnitQL = 24576, kUnitF = 40960, kUnitFBytes = 512;
+constexpr int kUnitBytesGated = 41984;
 __host__ __device__ constexpr int unit_bytes(bool gated) { return gated ? kUnitBytesGated : kUnitBytes; }
 
 // Gated DeltaNet: the log decays g of tokens [t, t + 64) of one (batch row, head), two

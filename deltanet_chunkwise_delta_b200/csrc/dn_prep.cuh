@@ -24,7 +24,12 @@
 // chunk's log decays, Gamma[l][i] = lambda[i+1:l] = exp(c_l - c_i) multiplies
 // both halves of G (L = (K K^T o Gamma) o M_c^-, P = (Q K^T o Gamma) o M_c),
 // and a third tile T' = T diag(lambda[1:l]) = T diag(exp(c_l)) gives
-// W<- = T K<- = T' K to the chain kernels (24 KB per unit: T, P, T').
+// W<- = T K<- = T' K to the chain kernels.  The unit also carries what the chain
+// kernels would otherwise compute from the log decays next to the state chain: the
+// decayed queries Q<- = diag(lambda[1:l]) Q (the unit's q boxes scaled per token
+// row, in the layout the tensor cores read), and the row factors lambda[l+1:C] =
+// exp(c_C - c_l) and lambda[1:C] = exp(c_C) (K-> = diag(lambda[l+1:C]) K enters the
+// state update as diag(lambda[l+1:C]) Z, the state's decay as lambda[1:C]).
 // One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM (five when
 // gated), so the latency of the solve is hidden by parallelism across chunks.  A CTA's shared
 // memory is one 32 KB region that holds the unit's q/k tile until the product
@@ -90,6 +95,11 @@ static_assert((PrepSmemT<false>::TOTAL + 1024) * prep_ctas_per_sm<false>() <= 22
 static_assert((PrepSmemT<true>::TOTAL + 1024) * prep_ctas_per_sm<true>() <= 228 * 1024, "pre-pass shared memory");
 
 __device__ __forceinline__ int blk_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
+
+// bf16 pair * f, rounded to nearest-even.
+__device__ __forceinline__ uint32_t scale_pair(uint32_t w, float f) {
+    return sm100::pack_bf16(__uint_as_float(w << 16) * f, __uint_as_float(w & 0xffff0000u) * f);
+}
 
 // acc (16 x 16, two n8 tiles) += A (16 x 16) * B (16 x 16), tf32 inputs, fp32 accumulate.
 __device__ __forceinline__ void mm16_tf32(float (&acc)[2][4], const float* A, const float* B) {
@@ -227,6 +237,11 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                                              kChunk);
                 reinterpret_cast<float2*>(smem + L::OFF_C)[lane] = c;
                 reinterpret_cast<float2*>(smem + L::OFF_LAM)[lane] = make_float2(expf(c.x), expf(c.y));
+                // row factors F of the unit: lambda[l+1:C] per row, then lambda[1:C]
+                const float cC = __shfl_sync(0xffffffffu, c.y, 31);
+                float* F = reinterpret_cast<float*>(p.wsT + (size_t)u * kUnit + kUnitF);
+                reinterpret_cast<float2*>(F)[lane] = make_float2(expf(cC - c.x), expf(cC - c.y));
+                if (lane == 0) F[kChunk] = expf(cC);
             }
         }
         // G = [Q; K] K^T into 64 tensor-memory columns: lanes 0-63 Q K^T, 64-127 K K^T
@@ -243,6 +258,31 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         // the product has read the q/k tile: the region now takes the solve's blocks
         if (__syncthreads_or(!gdone)) break;
         sm100::tc_fence_after();
+        if constexpr (GATED) {
+            // Q<- = diag(lambda[1:l]) Q: the unit's two q boxes (128-byte rows, swizzled
+            // within the row) scaled per token row and written out unchanged in layout,
+            // before the solve's blocks overwrite them
+            const float* lam = reinterpret_cast<const float*>(smem + L::OFF_LAM);
+            uint8_t* dst = p.wsT + (size_t)u * kUnit + kUnitQL;
+            uint4 w[8];
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const int id = tid + kPrepThreads * k8, a = id >> 9, row = (id >> 3) & 63, pc = id & 7;
+                w[k8] = *reinterpret_cast<const uint4*>(smem + L::OFF_QK + a * 16384 + row * 128 + pc * 16);
+            }
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const int id = tid + kPrepThreads * k8, a = id >> 9, row = (id >> 3) & 63, pc = id & 7;
+                const float f = lam[row];
+                uint4 v = w[k8];
+                v.x = scale_pair(v.x, f);
+                v.y = scale_pair(v.y, f);
+                v.z = scale_pair(v.z, f);
+                v.w = scale_pair(v.w, f);
+                *reinterpret_cast<uint4*>(dst + a * 8192 + row * 128 + pc * 16) = v;
+            }
+            __syncthreads();
+        }
         const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + bb * kChunk;
         const float* cs = reinterpret_cast<const float*>(smem + L::OFF_C);  // gated: running sums
         {
@@ -460,7 +500,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         const int un = u + gridDim.x;
         if (tid == 0) {
             sm100::bulk_store(p.wsT + (size_t)u * kUnit, smem + L::OFF_A, 8192);
-            if constexpr (GATED) sm100::bulk_store(p.wsT + (size_t)u * kUnit + 16384, smem + L::OFF_T2, 8192);
+            if constexpr (GATED) sm100::bulk_store(p.wsT + (size_t)u * kUnit + kUnitT2, smem + L::OFF_T2, 8192);
             sm100::bulk_commit();
         }
         if (un < units) {

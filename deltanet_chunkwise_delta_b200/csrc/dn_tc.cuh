@@ -24,7 +24,8 @@
 //               chunk's P tile in
 //   warp 12     issues the state-chain products and the output product that
 //               reads the chain's operand, one thread; owns the tensor memory
-//   warp 13     TMA loads of q, k (3-stage ring), one thread
+//   warp 13     TMA loads of k (3-stage ring) and q (3-stage ring; Gated DeltaNet:
+//               bulk copies of the pre-pass's Q<- tile, 2 stages), one thread
 //   warp 14     issues the chunk-parallel products (U^T, W^T), one thread
 //   warp 15     TMA loads of v and bulk copies of T (2-stage ring), one thread
 // The tensor pipe runs products in issue order, and a waiting issuer thread
@@ -53,29 +54,35 @@ constexpr int kParMmaWarp = 14;
 constexpr int kTmaBWarp = 15;
 
 // shared memory (byte offsets from a 1024-aligned base)
-//   ring A: 3 stages of [-W d0-63 | Q d0-63 | -W d64-127 | Q d64-127 | K d0-63 | K d64-127]
-//           (-W rows written by the epilogue, q and k by TMA; [-W; Q] is one
-//           K-major operand of 128 token rows).  For odd chunks -W and Q swap
-//           places, so that the product's [Z^T | O^T] columns alternate around
-//           one U^T / Z^T block between two O^T buffers.
+//   ring Q: NQ stages of [-W d0-63 | Q d0-63 | -W d64-127 | Q d64-127] (-W rows
+//           written by the epilogue, q by TMA; [-W; Q] is one K-major operand of
+//           128 token rows).  For odd chunks -W and Q swap places, so that the
+//           product's [Z^T | O^T] columns alternate around one U^T / Z^T block
+//           between two O^T buffers.
+//   ring K: 3 stages of [K d0-63 | K d64-127] (TMA)
 //   ring B: 2 stages of [V d0-63 | V d64-127 | T]
 //   2 P tiles (chunk r's in buffer r % 2); O staging (two 64-column boxes of token rows)
-// Gated DeltaNet: ring B stages also hold T' = T diag(lambda[1:l]) (the W<- factor), and ring
-// A has two stages, so that the layout fits.
-constexpr int NB = 2;
-constexpr int A_STAGE = 49152;
-constexpr int A_K = 32768;  // + 8192 for d 64-127; -W and Q at 0 / 8192 (+ 16384 for d 64-127)
+// A chunk's ring-Q and ring-K stages are released together, by one commit after its
+// state update (B_EMPTY + r % 6; the producer waits for chunk r - 3 before loading k of
+// chunk r and for chunk r - NQ before its q).
+// Gated DeltaNet: ring Q holds Q<- = diag(lambda[1:l]) Q from the pre-pass and has two
+// stages, ring B stages also hold T' = T diag(lambda[1:l]) (the W<- factor), and each P
+// buffer is followed by the chunk's row factors (lambda[l+1:C] per row, lambda[1:C]).
+constexpr int NB = 2, NK = 3, NE = 6;
+constexpr int Q_STAGE = 32768, K_STAGE = 16384;
 __host__ __device__ constexpr int a_w(int c) { return (c & 1) ? 8192 : 0; }  // -W rows of chunk c
 __host__ __device__ constexpr int a_q(int c) { return (c & 1) ? 0 : 8192; }  // Q rows of chunk c
 constexpr int B_T = 16384, B_T2 = 24576;
-constexpr int NBAR = 34;
+constexpr int NBAR = 42;
 template <bool GATED>
 struct TcLay {
-    static constexpr int NA = GATED ? 2 : 3;
-    static constexpr int OFF_B = NA * A_STAGE;
+    static constexpr int NQ = GATED ? 2 : 3;
+    static constexpr int OFF_K = NQ * Q_STAGE;
+    static constexpr int OFF_B = OFF_K + NK * K_STAGE;
     static constexpr int B_STAGE = GATED ? 32768 : 24576;  // V, T (, T')
-    static constexpr int OFF_PB = OFF_B + NB * B_STAGE;    // P rows, 2 x 8 KB
-    static constexpr int OFF_OB = OFF_PB + 2 * 8192;       // O staging
+    static constexpr int PB_STRIDE = GATED ? 9216 : 8192;  // P tile (+ row factors)
+    static constexpr int OFF_PB = OFF_B + NB * B_STAGE;
+    static constexpr int OFF_OB = OFF_PB + 2 * PB_STRIDE;  // O staging
     static constexpr int OFF_BAR = OFF_OB + 16384;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
@@ -86,8 +93,10 @@ constexpr int SMEM_BYTES = TcLay<false>::SMEM_BYTES;
 
 // tensor-memory columns (512 allocated): S^T fp32, [O^T (odd chunks) | U^T/Z^T |
 // O^T (even chunks)] (one product of N = 128 writes Z^T and the chunk's O^T), W^T,
-// Z^T bf16 (64 tokens in 32 columns), S^T bf16 (128 d_k in 64 columns)
-constexpr uint32_t TM_S = 0, TM_O1 = 128, TM_ZU = 192, TM_O0 = 256, TM_WT = 320, TM_ZBF = 384, TM_SBF = 448;
+// Z^T bf16 (64 tokens in 32 columns), Gated DeltaNet: Z^T diag(lambda[l+1:C]) bf16 (the
+// state update's operand), S^T bf16 (128 d_k in 64 columns)
+constexpr uint32_t TM_S = 0, TM_O1 = 128, TM_ZU = 192, TM_O0 = 256, TM_WT = 320, TM_ZBF = 384, TM_ZBF2 = 416,
+                   TM_SBF = 448;
 __device__ __forceinline__ uint32_t tm_o(int c) { return (c & 1) ? TM_O1 : TM_O0; }   // O^T of chunk c
 __device__ __forceinline__ uint32_t tm_c1(int c) { return (c & 1) ? TM_O1 : TM_ZU; }  // first product's D
 
@@ -96,13 +105,13 @@ __device__ __forceinline__ uint32_t tm_c1(int c) { return (c & 1) ? TM_O1 : TM_Z
 // completed by epilogue warps take one arrival per warp, after __syncwarp():
 // each lane has already fenced its own writes or tensor-memory accesses.
 enum : int {
-    B_FULLA = 0,     // +3: q, k of a stage landed
-    B_EMPTYA = 3,    // +3: stage of ring A consumed
+    B_FULLQ = 0,     // +3: q of a ring-Q stage landed
+    B_FULLK = 3,     // +3: k of a ring-K stage landed
     B_FULLB = 6,     // +2: v, T landed
     B_EMPTYB = 8,    // +2: stage of ring B consumed
     B_WUFULL = 10,   // W^T of the chunk ready in tensor memory
     B_WTFREE = 11,   // W^T columns read out
-    B_WFULL = 12,    // -W rows of the chunk written to its ring-A stage
+    B_WFULL = 12,    // -W rows of the chunk written to its ring-Q stage
     B_C1 = 13,       // [Z^T | O^T] product complete (bf16 S^T read)
     B_ZFULL = 14,    // bf16 Z^T written
     B_ZFREE = 15,    // fp32 U^T / Z^T columns read out
@@ -118,8 +127,9 @@ enum : int {
     B_UFULL = 28,    // U^T of the chunk ready in tensor memory
     B_DRAIN = 31,    // +2: drain of the chain issuer's / the parallel issuer's products
     B_STALL = 33,    // never completed: the wait of a test stall (Params::stall_chunk)
+    B_EMPTY = 34,    // +6: chunk r's ring-Q and ring-K stages consumed (slot r % 6)
 };
-static_assert(B_STALL < NBAR, "barrier count");
+static_assert(B_EMPTY + NE <= NBAR, "barrier count");
 
 // Optional timeline of CTA 0 (build with -DDN_TRACE): globaltimer stamps per
 // chunk and pipeline event, read back with dn_trace_copy().
@@ -175,54 +185,6 @@ __device__ __forceinline__ void store_token_rows(const RowFrags& f, int q, uint8
                           pack_bf16(scale * __uint_as_float(f.hi[g][2]), scale * __uint_as_float(f.hi[g][3])));
 }
 
-// bf16 pair * f, rounded to nearest-even.
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t w, float f) {
-    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
-    return pack_bf16(lo * f, hi * f);
-}
-// Gated DeltaNet: token rows 16 q .. 16 q + 15 of a chunk tile (two 64-column boxes of
-// 128-byte rows, at box0 and box0 + box_stride) multiplied in place by one factor per
-// row: lane l holds the factor of row 16 q + (l & 15).  A whole warp; the caller fences
-// the writes for the tensor cores.
-__device__ __forceinline__ void scale_token_rows(uint8_t* box0, uint32_t box_stride, int q, float f) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int id = lane + 32 * i;  // 256 pieces of 16 bytes: 16 rows x 2 boxes x 8
-        const int piece = id & 7, lr = (id >> 3) & 15, box = id >> 7;
-        const float fr = __shfl_sync(0xffffffffu, f, lr);
-        uint4* ptr = reinterpret_cast<uint4*>(box0 + box * box_stride + (16 * q + lr) * 128 + piece * 16);
-        uint4 w = *ptr;
-        w.x = scale_bf16x2(w.x, fr);
-        w.y = scale_bf16x2(w.y, fr);
-        w.z = scale_bf16x2(w.z, fr);
-        w.w = scale_bf16x2(w.w, fr);
-        *ptr = w;
-    }
-}
-// Gated DeltaNet: the log decays of chunk c of a run, two per lane (gate_load), or zeros
-// past the run's last chunk.
-__device__ __forceinline__ float2 chunk_gates(const Params& p, const Item& it, int c, int nch) {
-    if (c >= nch) return make_float2(0.f, 0.f);
-    return gate_load(p.g + it.b * p.g_sb + it.head * p.g_sh, p.g_st, it.tok0 + c * kChunk, it.tok1);
-}
-// Gated DeltaNet: lambda[1:C] = exp(c_C) of chunk c of a run (a whole warp).
-__device__ __forceinline__ float chunk_decay(const Params& p, const Item& it, int c) {
-    return expf(gate_sum(chunk_gates(p, it, c, c + 1)));
-}
-// Gated DeltaNet, a whole warp: from the chunk's log decays (gate_load), the factors of its
-// token row 16 q + (lane & 15): lambda[1:l] = exp(c_l) (-> .x) and lambda[l+1:C] =
-// exp(c_C - c_l) (-> .y).
-__device__ __forceinline__ float2 row_decays(float2 g, int q) {
-    const int lane = threadIdx.x & 31;
-    const float2 c = gate_scan(g);
-    const int t = 16 * q + (lane & 15);
-    const float cx = __shfl_sync(0xffffffffu, c.x, t >> 1), cy = __shfl_sync(0xffffffffu, c.y, t >> 1);
-    const float cC = __shfl_sync(0xffffffffu, c.y, 31);
-    const float ct = (t & 1) ? cy : cx;
-    return make_float2(expf(ct), expf(cC - ct));
-}
-
 template <bool GATED>
 static __global__ void __launch_bounds__(kThreadsTc, 1)
     k_tc_chain(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -245,10 +207,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < L::NA; ++s) {
-            mbar_init(&bars[B_FULLA + s], 1);
-            mbar_init(&bars[B_EMPTYA + s], 1);
-        }
+        for (int s = 0; s < L::NQ; ++s) mbar_init(&bars[B_FULLQ + s], 1);
+        for (int s = 0; s < NK; ++s) mbar_init(&bars[B_FULLK + s], 1);
+        for (int s = 0; s < NE; ++s) mbar_init(&bars[B_EMPTY + s], 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars[B_FULLB + s], 1);
             mbar_init(&bars[B_EMPTYB + s], 1);
@@ -297,28 +258,46 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
     if (it.g == 0 && it.G >= 2 && !p.sched.list && p.sched.e_in_c) x_out = p.wsH + (int64_t)it.slot * D * D;
 
     if (warp == kTmaWarp) {
-        // ------------------------------------------------------------ ring A: q, k
+        // ------------------------------------------------------------ rings K and Q
+        // k of chunk r before its q: W^T(r) reads K a chunk before the first product
+        // reads Q
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = 32768u;
-            int issued = 0;
+            int issued_k = 0, issued_q = 0;
             for (int r = 0; r < nch; ++r) {
-                const int s = r % L::NA;
-                if (r >= L::NA && !mbar_wait(&bars[B_EMPTYA + s], ((r / L::NA) - 1) & 1, abort_flag)) break;
-                mbar_expect_tx(&bars[B_FULLA + s], bytes);
-                uint8_t* st = smem + s * A_STAGE;
                 const int t0 = it.tok0 + r * kChunk;
+                const int sk = r % NK;
+                if (r >= NK && !mbar_wait(&bars[B_EMPTY + (r - NK) % NE], ((r - NK) / NE) & 1, abort_flag)) break;
+                mbar_expect_tx(&bars[B_FULLK + sk], 16384u);
+                uint8_t* stk = smem + L::OFF_K + sk * K_STAGE;
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    tma_load_4d(st + a_q(r) + a * 16384, &tq, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
-                    tma_load_4d(st + A_K + a * 8192, &tk, &bars[B_FULLA + s], a * 64, it.head, t0, it.b);
+                for (int a = 0; a < 2; ++a)
+                    tma_load_4d(stk + a * 8192, &tk, &bars[B_FULLK + sk], a * 64, it.head, t0, it.b);
+                issued_k = r + 1;
+                const int sq = r % L::NQ;
+                if (L::NQ < NK && r >= L::NQ &&
+                    !mbar_wait(&bars[B_EMPTY + (r - L::NQ) % NE], ((r - L::NQ) / NE) & 1, abort_flag))
+                    break;
+                mbar_expect_tx(&bars[B_FULLQ + sq], 16384u);
+                uint8_t* stq = smem + sq * Q_STAGE;
+                if constexpr (GATED) {
+                    // Q<- of the chunk, from the pre-pass (two 8 KB boxes)
+                    const uint8_t* ql = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit + kUnitQL;
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) bulk_load(stq + a_q(r) + a * 16384, ql + a * 8192, 8192, &bars[B_FULLQ + sq]);
+                } else {
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_4d(stq + a_q(r) + a * 16384, &tq, &bars[B_FULLQ + sq], a * 64, it.head, t0, it.b);
                 }
-                issued = r + 1;
+                issued_q = r + 1;
                 DN_TR(true, r, 24);
             }
             // the last loads issued must have landed before the CTA may exit (even after an abort)
             volatile int drain = 0;
-            for (int r = issued - L::NA < 0 ? 0 : issued - L::NA; r < issued; ++r)
-                mbar_wait(&bars[B_FULLA + (r % L::NA)], (r / L::NA) & 1, &drain, kDrainWaitNs);
+            for (int r = issued_k - NK < 0 ? 0 : issued_k - NK; r < issued_k; ++r)
+                mbar_wait(&bars[B_FULLK + (r % NK)], (r / NK) & 1, &drain, kDrainWaitNs);
+            for (int r = issued_q - L::NQ < 0 ? 0 : issued_q - L::NQ; r < issued_q; ++r)
+                mbar_wait(&bars[B_FULLQ + (r % L::NQ)], (r / L::NQ) & 1, &drain, kDrainWaitNs);
         }
     } else if (warp == kTmaBWarp) {
         // ------------------------------------------------------------ ring B: v, T
@@ -336,7 +315,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                     tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
                 const uint8_t* unit = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit;
                 bulk_load(st + B_T, unit, 8192, &bars[B_FULLB + s]);
-                if constexpr (GATED) bulk_load(st + B_T2, unit + 16384, 8192, &bars[B_FULLB + s]);
+                if constexpr (GATED) bulk_load(st + B_T2, unit + kUnitT2, 8192, &bars[B_FULLB + s]);
                 issued = r + 1;
             }
             volatile int drain = 0;
@@ -354,11 +333,15 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t i_c3 = idesc_bf16(128, 128, false, true);
             const uint32_t i_o = idesc_bf16(128, 64, false, false);
             const uint64_t dWQ = sdesc(sb, 16, 1024);           // [-W; Q] / [Q; -W] token rows, K-major
-            const uint64_t dK = sdesc(sb + A_K, 8192, 1024);    // K, MN-major
+            const uint64_t dK = sdesc(sb + L::OFF_K, 8192, 1024);  // K, MN-major
+            // the state update's A operand: Z^T, or for Gated DeltaNet Z^T diag(lambda[l+1:C])
+            // (so that the update adds K->^T Z)
+            constexpr uint32_t tm_zs = GATED ? TM_ZBF2 : TM_ZBF;
             const uint64_t dP = sdesc(sb + L::OFF_PB, 16, 1024);   // P^T, K-major (+ 8 KB for odd chunks)
             for (int r = 0; r < nch; ++r) {
-                const int sa = r % L::NA, s = r & 1;
-                const uint64_t sta = (uint64_t)((sa * A_STAGE) >> 4);
+                const int s = r & 1;
+                const uint64_t stq = (uint64_t)(((r % L::NQ) * Q_STAGE) >> 4);
+                const uint64_t stk = (uint64_t)(((r % NK) * K_STAGE) >> 4);
                 DN_TR(true, r, 0);
                 if (r + 1 == p.stall_chunk && !mbar_wait(&bars[B_STALL], 0, abort_flag)) break;
                 const bool ready = mbar_wait4(&bars[B_WFULL], r & 1, &bars[B_SBF], r & 1, &bars[B_UFULL], r & 1,
@@ -371,7 +354,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint64_t o = (uint64_t)(((j >> 2) * 16384 + (j & 3) * 32) >> 4);
-                    umma_bf16_ts(tmem + d1, tmem + TM_SBF + 8 * j, dWQ + sta + o, i_c1, 1u);
+                    umma_bf16_ts(tmem + d1, tmem + TM_SBF + 8 * j, dWQ + stq + o, i_c1, 1u);
                 }
                 umma_commit(&bars[B_C1]);
                 mbar_arrive(&bars[B_GAP1 + s]);
@@ -382,24 +365,24 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 // S^T += Z^T K
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    umma_bf16_ts(tmem + TM_S, tmem + TM_ZBF + 8 * j, dK + sta + (uint64_t)((j * 2048) >> 4), i_c3,
+                    umma_bf16_ts(tmem + TM_S, tmem + tm_zs + 8 * j, dK + stk + (uint64_t)((j * 2048) >> 4), i_c3,
                                  1u);
                 umma_commit(&bars[B_SFULL]);
+                // the chunk's -W, q and k are read by the products above (and k by W^T of
+                // the chunk, complete before its -W rows were written)
+                umma_commit(&bars[B_EMPTY + r % NE]);
                 mbar_arrive(&bars[B_GAP2 + s]);
                 {
                     // O^T += Z^T P^T
                     if (!mbar_wait(&bars[B_PFULL + s], (r >> 1) & 1, abort_flag)) break;
                     tc_fence_after();
-                    const uint64_t pofs = (uint64_t)((s * 8192) >> 4);
+                    const uint64_t pofs = (uint64_t)((s * L::PB_STRIDE) >> 4);
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         umma_bf16_ts(tmem + tm_o(r), tmem + TM_ZBF + 8 * j, dP + pofs + (uint64_t)((j * 32) >> 4),
                                      i_o, 1u);
                     umma_commit(&bars[B_OFULL]);
                 }
-                // the stage's -W, q and k are read by the products above (and k by W^T of
-                // the chunk, complete before its -W rows were written)
-                umma_commit(&bars[B_EMPTYA + sa]);
                 DN_TR(true, r, 11);
             }
             umma_drain(&bars[B_DRAIN]);
@@ -414,17 +397,17 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         if (lane == 0 && nch > 0) {
             const uint32_t sb = saddr(smem);
             const uint32_t i_tt = idesc_bf16(128, 64, true, false);
-            const uint64_t dKT = sdesc(sb + A_K, 8192, 1024);          // K^T, MN-major
+            const uint64_t dKT = sdesc(sb + L::OFF_K, 8192, 1024);     // K^T, MN-major
             const uint64_t dVT = sdesc(sb + L::OFF_B, 8192, 1024);        // V^T, MN-major
             const uint64_t dT = sdesc(sb + L::OFF_B + B_T, 16, 1024);     // T^T, K-major
             // W = T K, or for Gated DeltaNet W<- = T' K with T' = T diag(lambda[1:l])
             const uint64_t dTw = GATED ? sdesc(sb + L::OFF_B + B_T2, 16, 1024) : dT;
             auto issue_w = [&](int c) {
-                const uint64_t sta = (uint64_t)(((c % L::NA) * A_STAGE) >> 4);
+                const uint64_t stk = (uint64_t)(((c % NK) * K_STAGE) >> 4);
                 const uint64_t stb = (uint64_t)(((c & 1) * L::B_STAGE) >> 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    umma_bf16(tmem + TM_WT, dKT + sta + (uint64_t)((j * 2048) >> 4),
+                    umma_bf16(tmem + TM_WT, dKT + stk + (uint64_t)((j * 2048) >> 4),
                               dTw + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 umma_commit(&bars[B_WUFULL]);
             };
@@ -440,7 +423,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 umma_commit(&bars[B_EMPTYB + s]);
             };
             auto wait_data = [&](int c) -> bool {
-                return mbar_wait2(&bars[B_FULLA + c % L::NA], (c / L::NA) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
+                return mbar_wait2(&bars[B_FULLK + c % NK], (c / NK) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
                                   abort_flag);
             };
             bool ok = wait_data(0);
@@ -473,13 +456,15 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         const int q = warp - 8;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         int p_issued = 0;
-        // P tile of chunk c into buffer c % 2 (one thread)
+        // P tile of chunk c into buffer c % 2 (one thread); Gated DeltaNet: followed by the
+        // chunk's row factors
         auto issue_p = [&](int c) {
             ++p_issued;
-            mbar_expect_tx(&bars[B_PFULL + (c & 1)], 8192u);
-            bulk_load(smem + L::OFF_PB + (c & 1) * 8192,
-                      p.wsT + ((size_t)(it.cbase + c) * p.sched.H + it.head) * kUnit + 8192, 8192,
-                      &bars[B_PFULL + (c & 1)]);
+            const uint8_t* unit = p.wsT + ((size_t)(it.cbase + c) * p.sched.H + it.head) * kUnit;
+            uint8_t* buf = smem + L::OFF_PB + (c & 1) * L::PB_STRIDE;
+            mbar_expect_tx(&bars[B_PFULL + (c & 1)], 8192u + (GATED ? (uint32_t)kUnitFBytes : 0u));
+            bulk_load(buf, unit + 8192, 8192, &bars[B_PFULL + (c & 1)]);
+            if constexpr (GATED) bulk_load(buf + 8192, unit + kUnitF, kUnitFBytes, &bars[B_PFULL + (c & 1)]);
         };
         // O^T of chunk c -> out: read out of tensor memory (and zeroed for the next
         // chunk's first product, which accumulates into it), staged as token rows (the
@@ -543,16 +528,12 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 mbar_arrive(&bars[B_OFREE + 1]);
             }
         }
-        // Gated DeltaNet: the chunk's log decays are loaded one chunk ahead
-        float2 g_next = GATED ? chunk_gates(p, it, 0, nch) : make_float2(0.f, 0.f);
         for (int r = 0; r < nch; ++r) {
-            uint8_t* stage = smem + (r % L::NA) * A_STAGE;
-            const float2 g_cur = g_next;
-            if constexpr (GATED) g_next = chunk_gates(p, it, r + 1, nch);
-            // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's q/k stage,
+            uint8_t* stage = smem + (r % L::NQ) * Q_STAGE;
+            // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's ring-Q stage,
             // once the stage holds the chunk (its previous chunk's products are done)
-            if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % L::NA], (r / L::NA) & 1,
-                                                    abort_flag)))
+            if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLQ + r % L::NQ],
+                                                    (r / L::NQ) & 1, abort_flag)))
                 break;
             DN_TR(q == 0, r, 13);
             tc_fence_after();
@@ -563,14 +544,6 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars[B_WTFREE]);
                 store_token_rows(f, q, stage + a_w(r), 16384, -1.f);
-            }
-            if constexpr (GATED) {
-                // W^T has read K: the chunk's Q rows become Q<- (lambda[1:l] q_l, read by the
-                // output product) and its K rows K-> (lambda[l+1:C] k_l, read by the state
-                // update), with lambda[1:l] = exp(c_l) and lambda[l+1:C] = exp(c_C - c_l)
-                const float2 f = row_decays(g_cur, q);
-                scale_token_rows(stage + a_q(r), 16384, q, f.x);
-                scale_token_rows(stage + A_K, 8192, q, f.y);
             }
             fence_async_smem();
             __syncwarp();
@@ -609,6 +582,12 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         // the state entering chunk c of the run (for a backward pass): row = global chunk
         // index; this thread's column d of key rows 64 h .. + 63 (a warp writes 128
         // contiguous bytes of each row)
+        // Gated DeltaNet: the row factors of chunk c (lambda[l+1:C] for rows l = 0..63, then
+        // lambda[1:C]), in its P buffer from B_PFULL until the chunk's output product is
+        // complete
+        auto pfac = [&](int c) {
+            return reinterpret_cast<const float*>(smem + L::OFF_PB + (c & 1) * L::PB_STRIDE + 8192);
+        };
         auto store_chunk_state = [&](int c, const uint32_t(&v)[64]) {
             const int64_t row = (int64_t)it.cbase + c;
             if (!p.cs || row >= p.cs_rows) return;
@@ -616,6 +595,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
             for (int cc = 0; cc < 64; ++cc) dst[(int64_t)(64 * h + cc) * D] = __uint_as_float(v[cc]);
         };
+        bool live = true;
         {
             uint32_t v[64];
 #pragma unroll
@@ -634,8 +614,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 pack_pairs<64>(v, pk);
                 tmem_st32(tmem + lane_base + TM_SBF + 32 * h, pk);
                 if constexpr (GATED) {
-                    // Gated DeltaNet: the update of chunk 0 adds K->^T Z to lambda[1:C] S
-                    const float lam = chunk_decay(p, it, 0);
+                    // Gated DeltaNet: the update of chunk 0 adds K->^T Z to lambda[1:C] S (the
+                    // chunk's factors arrive with its P tile)
+                    live = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL], 0, abort_flag));
+                    const float lam = live ? pfac(0)[kChunk] : 1.f;
 #pragma unroll
                     for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
                 }
@@ -645,16 +627,8 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_SBF]);
-        // Gated DeltaNet: the log decays of the chunk after next, loaded one iteration early
-        float2 g_pre = GATED ? chunk_gates(p, it, 1, nch) : make_float2(0.f, 0.f);
-        for (int r = 0; r < nch; ++r) {
-            // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
-            float lam_next = 1.f;
-            if constexpr (GATED) {
-                lam_next = expf(gate_sum(g_pre));
-                g_pre = chunk_gates(p, it, r + 2, nch);
-            }
+        if (lane == 0 && live) mbar_arrive(&bars[B_SBF]);
+        for (int r = 0; live && r < nch; ++r) {
             // Z^T -> bf16 (A operand of the S^T update and of O^T += Z^T P^T), once the
             // previous chunk's O^T += Z^T P^T has read the previous one
             DN_TR(warp == 0, r, 27);
@@ -669,6 +643,20 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_ld32(tmem + lane_base + TM_ZU + 32 * h, v);
                 pack_pairs<32>(v, pk);
                 tmem_st16(tmem + lane_base + TM_ZBF + 16 * h, pk);
+                if constexpr (GATED) {
+                    // Z^T diag(lambda[l+1:C]) for the state update (this half's 32 tokens)
+                    const float4* f4 = reinterpret_cast<const float4*>(pfac(r) + 32 * h);
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 f = f4[c4];
+                        v[4 * c4 + 0] = __float_as_uint(f.x * __uint_as_float(v[4 * c4 + 0]));
+                        v[4 * c4 + 1] = __float_as_uint(f.y * __uint_as_float(v[4 * c4 + 1]));
+                        v[4 * c4 + 2] = __float_as_uint(f.z * __uint_as_float(v[4 * c4 + 2]));
+                        v[4 * c4 + 3] = __float_as_uint(f.w * __uint_as_float(v[4 * c4 + 3]));
+                    }
+                    pack_pairs<32>(v, pk);
+                    tmem_st16(tmem + lane_base + TM_ZBF2 + 16 * h, pk);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -698,9 +686,13 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 }
                 if (r + 1 < nch) store_chunk_state(r + 1, v);
                 if (GATED && r + 1 < nch) {
-                    // S^T <- lambda[1:C] S^T before the next chunk's update accumulates into
-                    // it (complete before this warp's next Z^T arrival, which that update
-                    // waits for); the bf16 copy above stays unscaled
+                    // S^T <- lambda[1:C] S^T of the next chunk before that chunk's update
+                    // accumulates into it (complete before this warp's next Z^T arrival, which
+                    // the update waits for); the bf16 copy above stays unscaled
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + ((r + 1) & 1)], ((r + 1) >> 1) & 1,
+                                                           abort_flag)))
+                        break;
+                    const float lam_next = pfac(r + 1)[kChunk];
 #pragma unroll
                     for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
                     tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));

@@ -61,20 +61,24 @@ constexpr int kTmaBWarp = 15;
 //   ring B: 2 stages of [V d0-63 | V d64-127 | T]
 //   Z^T bf16 of chain H and of chain P: d_v rows x 64 tokens, 128-byte swizzled
 //   S_P^T bf16: d_v rows x [d_k 0-63 | d_k 64-127], 128-byte swizzled
-//   (Gated DeltaNet: ring B stages also hold T' = T diag(lambda[1:l]), the W<- factor)
+//   (Gated DeltaNet: ring B stages also hold T' = T diag(lambda[1:l]), the W<- factor, and a
+//   2-slot ring holds each chunk's row factors from the pre-pass: lambda[l+1:C] per row,
+//   which scales Z^T's token columns (Z^T diag(lambda[l+1:C]) K = Z^T K->), and lambda[1:C])
 constexpr int NA = 3, NB = 2;
 constexpr int A_STAGE = 32768;
 constexpr int A_K = 16384;
 constexpr int OFF_B = NA * A_STAGE;
 constexpr int B_T = 16384, B_T2 = 24576;
 constexpr int Z_BYTES = 16384;
-constexpr int NBAR = 27;
+constexpr int NF = 2;  // Gated DeltaNet: slots of the row-factor ring
+constexpr int NBAR = 31;
 template <bool GATED>
 struct SumLay {
     static constexpr int B_STAGE = GATED ? 32768 : 24576;
     static constexpr int OFF_Z = OFF_B + NB * B_STAGE;
     static constexpr int OFF_SP = OFF_Z + 2 * Z_BYTES;
-    static constexpr int OFF_BAR = OFF_SP + 32768;
+    static constexpr int OFF_F = OFF_SP + 32768;  // row-factor ring (gated)
+    static constexpr int OFF_BAR = OFF_F + (GATED ? NF * kUnitFBytes : 0);
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_USED = OFF_MISC + 64;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
@@ -119,8 +123,10 @@ enum : int {
     B_GAP1 = 21,    // +2: the chunk's first products are issued (one per chunk parity)
     B_GAP2 = 23,    // +2: chain H's state update is issued (one per chunk parity)
     B_DRAIN = 25,   // +2: drain of the chain issuer's / the parallel issuer's products
+    B_FULLF = 27,   // +2: row factors of a chunk landed (gated)
+    B_EMPTYF = 29,  // +2: row-factor slot read by every chain-epilogue warp (gated)
 };
-static_assert(B_DRAIN + 2 <= NBAR, "barrier count");
+static_assert(B_EMPTYF + NF <= NBAR, "barrier count");
 
 // Optional timeline of CTA 1 (the first two-chain item of a split chain; build
 // with -DDN_TRACE): globaltimer stamps per chunk and pipeline event.
@@ -178,6 +184,10 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
         mbar_init(&bars[B_UFULL], 1);
         mbar_init(&bars[B_DRAIN], 1);
         mbar_init(&bars[B_DRAIN + 1], 1);
+        for (int s = 0; s < NF; ++s) {
+            mbar_init(&bars[B_FULLF + s], 1);
+            mbar_init(&bars[B_EMPTYF + s], mode == kModeHP ? 8 : 4);
+        }
         wait_ctl_init(ctl, p.wait_ns);
         mbar_fence_init();
     }
@@ -220,7 +230,7 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
         } else if (warp == kTmaBWarp) {
             // ------------------------------------------------------------ ring B: v, T
             if (lane == 0 && nch > 0) {
-                int issued = 0;
+                int issued = 0, f_issued = 0;
                 for (int r = 0; r < nch; ++r) {
                     const int s = r & 1;
                     if (r >= 2 && !mbar_wait(&bars[B_EMPTYB + s], ((r >> 1) - 1) & 1, abort_flag)) break;
@@ -231,12 +241,23 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     for (int a = 0; a < 2; ++a) tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
                     const uint8_t* unit = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit;
                     bulk_load(st + B_T, unit, 8192, &bars[B_FULLB + s]);
-                    if constexpr (GATED) bulk_load(st + B_T2, unit + 16384, 8192, &bars[B_FULLB + s]);
                     issued = r + 1;
+                    if constexpr (GATED) {
+                        bulk_load(st + B_T2, unit + kUnitT2, 8192, &bars[B_FULLB + s]);
+                        // the chunk's row factors, once the chain epilogues are done with
+                        // chunk r - 2's
+                        const int sf = r % NF;
+                        if (r >= NF && !mbar_wait(&bars[B_EMPTYF + sf], ((r / NF) - 1) & 1, abort_flag)) break;
+                        mbar_expect_tx(&bars[B_FULLF + sf], (uint32_t)kUnitFBytes);
+                        bulk_load(smem + L::OFF_F + sf * kUnitFBytes, unit + kUnitF, kUnitFBytes, &bars[B_FULLF + sf]);
+                        f_issued = r + 1;
+                    }
                 }
                 volatile int drain = 0;
                 for (int r = issued - 2 < 0 ? 0 : issued - 2; r < issued; ++r)
                     mbar_wait(&bars[B_FULLB + (r & 1)], (r >> 1) & 1, &drain, kDrainWaitNs);
+                for (int r = f_issued - NF < 0 ? 0 : f_issued - NF; r < f_issued; ++r)
+                    mbar_wait(&bars[B_FULLF + (r % NF)], (r / NF) & 1, &drain, kDrainWaitNs);
             }
         } else if (warp == kMmaWarp) {
             // ------------------------------------------------------------ chain products
@@ -378,13 +399,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
             // ------------------------------------------------------------ -W rows
             const int q = warp - 8;
             const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-            // Gated DeltaNet: the chunk's log decays are loaded one chunk ahead
-            float2 g_next = GATED ? tc::chunk_gates(p, it, 0, nch) : make_float2(0.f, 0.f);
             for (int r = 0; r < nch; ++r) {
                 uint8_t* stage = smem + (r % NA) * A_STAGE;
-                const float2 g_cur = g_next;
-                (void)g_cur;
-                if constexpr (GATED) g_next = tc::chunk_gates(p, it, r + 1, nch);
                 // W^T (tensor memory, d_k lanes) -> -W token rows in the chunk's k stage,
                 // once the stage holds the chunk (its previous chunk's products are done)
                 if (!__all_sync(0xffffffffu, mbar_wait2(&bars[B_WUFULL], r & 1, &bars[B_FULLA + r % NA], (r / NA) & 1,
@@ -397,11 +413,6 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     tmem_load_rows(tmem + lane_base + TM_WT, f);
                     tc_fence_before();
                     store_token_rows(f, q, stage, 8192, -1.f);
-                }
-                if constexpr (GATED) {
-                    // W^T has read K: the chunk's K rows become K-> = lambda[l+1:C] k_l
-                    // (exp(c_C - c_l)), read by both state updates
-                    tc::scale_token_rows(stage + A_K, 8192, q, tc::row_decays(g_cur, q).y);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -440,8 +451,20 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                                 make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                     }
                 };
+                // Gated DeltaNet: the row factors of chunk c (lambda[l+1:C] per row, then
+                // lambda[1:C]), held from B_FULLF until this warp's Z^T of the chunk is converted
+                auto ffac = [&](int c) {
+                    return reinterpret_cast<const float*>(smem + L::OFF_F + (c % NF) * kUnitFBytes);
+                };
+                // the update of chunk 0 adds K->^T Z to lambda[1:C] S
+                bool live = true;
+                float lam0 = 1.f;
+                if (GATED && nch > 0) {
+                    live = __all_sync(0xffffffffu, mbar_wait(&bars[B_FULLF], 0, abort_flag));
+                    if (live) lam0 = ffac(0)[kChunk];
+                }
     #pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
+                for (int hh = 0; live && hh < 2; ++hh) {
                     uint32_t v[64];
     #pragma unroll
                     for (int c = 0; c < 64; ++c) {
@@ -458,10 +481,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                         pack_pairs<64>(v, pk);
                         store_sbf(x, hh, pk);
                         if constexpr (GATED) {
-                            // the update of chunk 0 adds K->^T Z to lambda[1:C] S
-                            const float lam = tc::chunk_decay(p, it, 0);
     #pragma unroll
-                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
+                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam0 * __uint_as_float(v[c]));
                         }
                         tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
                         tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
@@ -471,16 +492,8 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                 fence_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
-                // Gated DeltaNet: the log decays of the chunk after next, loaded one iteration early
-                float2 g_pre = GATED ? tc::chunk_gates(p, it, 1, nch) : make_float2(0.f, 0.f);
-                for (int r = 0; r < nch; ++r) {
-                    // Gated DeltaNet: lambda[1:C] of the next chunk, for its state update
-                    float lam_next = 1.f;
-                    if constexpr (GATED) {
-                        lam_next = expf(gate_sum(g_pre));
-                        g_pre = tc::chunk_gates(p, it, r + 2, nch);
-                    }
+                if (lane == 0 && live) mbar_arrive(&bars[B_SBF + x]);
+                for (int r = 0; live && r < nch; ++r) {
                     // Z_x^T -> bf16 token columns of row d in shared memory (the A operand of
                     // the state update)
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_C1 + x], r & 1, abort_flag))) break;
@@ -490,6 +503,18 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     for (int hh = 0; hh < 2; ++hh) {
                         uint32_t v[32], pk[16];
                         tmem_ld32(tmem + lane_base + tm_zu(x) + 32 * hh, v);
+                        if constexpr (GATED) {
+                            // Z^T diag(lambda[l+1:C]): the update then adds K->^T Z
+                            const float4* f4 = reinterpret_cast<const float4*>(ffac(r) + 32 * hh);
+    #pragma unroll
+                            for (int c4 = 0; c4 < 8; ++c4) {
+                                const float4 f = f4[c4];
+                                v[4 * c4 + 0] = __float_as_uint(f.x * __uint_as_float(v[4 * c4 + 0]));
+                                v[4 * c4 + 1] = __float_as_uint(f.y * __uint_as_float(v[4 * c4 + 1]));
+                                v[4 * c4 + 2] = __float_as_uint(f.z * __uint_as_float(v[4 * c4 + 2]));
+                                v[4 * c4 + 3] = __float_as_uint(f.w * __uint_as_float(v[4 * c4 + 3]));
+                            }
+                        }
                         pack_pairs<32>(v, pk);
     #pragma unroll
                         for (int c = 0; c < 4; ++c)
@@ -499,7 +524,10 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     fence_async_smem();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars[B_ZFULL + x]);
+                    if (lane == 0) {
+                        mbar_arrive(&bars[B_ZFULL + x]);
+                        if (GATED) mbar_arrive(&bars[B_EMPTYF + r % NF]);  // done with the chunk's factors
+                    }
                     DN_TS(wq == 0, r, 13 + 4 * x);
                     // S_x^T -> bf16 (and fp32 out after the last chunk); the chunk's first
                     // product (the only reader of the bf16 copy) is complete
@@ -516,15 +544,6 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
     #pragma unroll
                             for (int c = 0; c < 64; ++c) x_out[(int64_t)(64 * hh + c) * D + d] = __uint_as_float(v[c]);
                         }
-                        if (GATED && r + 1 < nch) {
-                            // S_x^T <- lambda[1:C] S_x^T before the next chunk's update accumulates
-                            // into it (the bf16 copy above stays unscaled)
-    #pragma unroll
-                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
-                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
-                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32,
-                                      *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                        }
                     }
                     tmem_wait_st();  // the bf16 copy's tensor-memory stores
                     fence_async_smem();
@@ -532,6 +551,27 @@ static __global__ void __launch_bounds__(kThreadsSum, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars[B_SBF + x]);
                     DN_TS(wq == 0, r, 15 + 4 * x);
+                    if (GATED && r + 1 < nch) {
+                        // S_x^T <- lambda[1:C] S_x^T of the next chunk before that chunk's update
+                        // accumulates into it, off the chain (the update waits for this warp's
+                        // next Z^T arrival); the bf16 copy above stays unscaled
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_FULLF + (r + 1) % NF], ((r + 1) / NF) & 1,
+                                                               abort_flag)))
+                            break;
+                        const float lam_next = ffac(r + 1)[kChunk];
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t v[64];
+                            tmem_ld64(tmem + lane_base + tm_s(x) + 64 * hh, v);
+    #pragma unroll
+                            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
+                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+                            tmem_st32(tmem + lane_base + tm_s(x) + 64 * hh + 32,
+                                      *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                        }
+                        tc_fence_before();
+                    }
                 }
             }
         }
