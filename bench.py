@@ -337,19 +337,21 @@ def run_b200(args, w: wl.Workload):
     tflops = ws * th * fpt / (ms / 1e3) / 1e12
     hbm_peak, tc_peak, peak_kind = load_peaks()
     alg_bytes = algorithmic_bytes(w)
-    # DeltaNet and Gated DeltaNet (one write per token) at d_k = d_v = 128 run on the
+    # DeltaNet, Gated DeltaNet and the Gated Delta Product at d_k = d_v = 128 run on the
     # tensor-core kernels
-    tc_path = w.nh == 1 and not w.kda and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
-    # the tensor-core boundary kernel moves q, k, v, o and the states (beta is read by the
-    # UT pre-pass); the mma.sync boundary kernel reads beta (and g) itself
-    kernel_bytes = alg_bytes - (4.0 * w.tokens * w.H if tc_path else 0.0)
+    tc_path = (not w.kda and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+               and (w.nh == 1 or w.gated))
+    # the tensor-core boundary kernel moves q, k, v, o and the states (beta and the log
+    # decays are read by the UT pre-pass); the mma.sync boundary kernel reads them itself
+    kernel_bytes = alg_bytes - ((4.0 * w.nh + (4.0 if w.gated else 0.0)) * w.tokens * w.H if tc_path else 0.0)
     if tc_path and w.seqlens is None and G >= 2:
         # split dense chains: run 0 of every chain is computed by its own launch next to
         # the summary pass; the timed launch covers runs 1..G-1 (q, k, v, o of their
-        # tokens and the final state)
+        # tokens, n_h rows of k and v per token, and the final state)
         es = 2
-        th_b = w.B * (w.T - s0 * CHUNK) * w.H
-        kernel_bytes = float(th_b * es * (2 * w.dk + 2 * w.dv) + w.n_seq * w.H * w.dk * w.dv * 4)
+        th_b = w.B * (w.T * w.nh - s0 * CHUNK) / w.nh * w.H
+        kernel_bytes = float(th_b * es * ((1 + w.nh) * w.dk + (w.nh + 1) * w.dv)
+                             + w.n_seq * w.H * w.dk * w.dv * 4)
     achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9
     tc_kernel = tc_path
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",

@@ -250,12 +250,12 @@ struct Dims {
 template <typename E, int DK, int DV, int STAGES, bool GATED, bool KDA = false>
 dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream, int forced_s,
                  const int* cu) {
-    // bf16 DeltaNet and Gated DeltaNet with d_k = d_v = 128 run on the tensor-core (tcgen05)
-    // kernels (with or without the chunk-start states); the Gated Delta Product (several
-    // writes per token) and the other shapes on the mma.sync chain kernels
-    // (Kimi Delta Attention, a decay per key channel, runs on the mma.sync chain kernels)
+    // bf16 DeltaNet, Gated DeltaNet and the Gated Delta Product with d_k = d_v = 128 run on
+    // the tensor-core (tcgen05) kernels (with or without the chunk-start states), the other
+    // shapes on the mma.sync chain kernels (Kimi Delta Attention, a decay per key channel,
+    // runs on the mma.sync chain kernels)
     constexpr bool kTcShape = !KDA && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
-    const bool use_tc = kTcShape && p.nh <= 1;
+    const bool use_tc = kTcShape && (p.nh <= 1 || GATED);
     using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED, KDA>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED, KDA>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED, KDA>;
@@ -291,10 +291,11 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     CUtensorMap tq, tk, tv, to;
     if (use_tc) {
         const int64_t Bq = d.varlen ? 1 : d.B;
-        if ((st = make_token_map(&tq, p.q, Bq, d.T, d.H, p.q_sb, p.q_st, p.q_sh)) != DN_OK) return st;
+        const int64_t Tq = d.T / (p.nh > 1 ? p.nh : 1);  // q and out: one row per token
+        if ((st = make_token_map(&tq, p.q, Bq, Tq, d.H, p.q_sb, p.q_st, p.q_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tk, p.k, Bq, d.T, d.H, p.k_sb, p.k_st, p.k_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tv, p.v, Bq, d.T, d.H, p.v_sb, p.v_st, p.v_sh)) != DN_OK) return st;
-        if ((st = make_token_map(&to, p.o, Bq, d.T, d.H, p.o_sb, p.o_st, p.o_sh)) != DN_OK) return st;
+        if ((st = make_token_map(&to, p.o, Bq, Tq, d.H, p.o_sb, p.o_st, p.o_sh)) != DN_OK) return st;
     }
 
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
@@ -388,6 +389,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         sc.counts = reinterpret_cast<const int*>(base);
         sc.cumchunks = reinterpret_cast<const int*>(base + off_cum);
         sc.cu = cu;
+        sc.cu_mul = p.nh > 1 ? p.nh : 1;
         sc.N = (int)d.N;
         k_schedule<<<1, 1024, 0, stream>>>(
             cu, p.nh > 1 ? p.nh : 1, (int)d.N, (int)d.T, (int)d.H, forced_s, forced_s > 0 ? kMaxSlots : kAutoMaxSlots,

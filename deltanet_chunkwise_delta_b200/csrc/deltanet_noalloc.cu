@@ -194,6 +194,7 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
 
     dn::Params p;
     std::memset(&p, 0, sizeof p);
+    p.nh = 1;
     p.q = q->data; p.k = k->data; p.v = v->data; p.o = out->data;
     p.beta = static_cast<const float*>(beta->data);
     p.s0 = initial_state ? static_cast<const float*>(initial_state->data) : nullptr;

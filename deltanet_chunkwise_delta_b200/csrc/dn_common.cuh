@@ -98,6 +98,7 @@ struct Sched {
     const int* cumchunks;   // list: [N + 1] first global chunk index of each sequence
     const int* cu;          // list: cu_seqlens [N + 1]
     int N;                  // list: number of sequences
+    int cu_mul;             // list: rows per token of cu_seqlens (Gated Delta Product: n_h)
 };
 
 struct Params {
@@ -218,8 +219,8 @@ __device__ __forceinline__ void chunk_range(const Sched& s, int id, int& b, int&
         else hi = mid;
     }
     b = 0;
-    t0 = s.cu[lo] + (id - s.cumchunks[lo]) * kChunk;
-    t1 = min(s.cu[lo + 1], t0 + kChunk);
+    t0 = s.cu[lo] * s.cu_mul + (id - s.cumchunks[lo]) * kChunk;
+    t1 = min(s.cu[lo + 1] * s.cu_mul, t0 + kChunk);
 }
 
 __device__ __forceinline__ Item item_scan(const Sched& s, int i) {

@@ -30,6 +30,12 @@
 // row, in the layout the tensor cores read), and the row factors lambda[l+1:C] =
 // exp(c_C - c_l) and lambda[1:C] = exp(c_C) (K-> = diag(lambda[l+1:C]) K enters the
 // state update as diag(lambda[l+1:C]) Z, the state's decay as lambda[1:C]).
+// Gated Delta Product (same page, "GDP as GDN over a virtual sequence"): a chunk is 64
+// virtual steps m (write j of token t is m = n_h t + j; k, v and beta hold one row per
+// step); the step's query is that of token m / n_h (read only on a token's last step, the
+// others' outputs are not stored) and its log decay that of the token on its first step,
+// 0 on the others.  The unit's q box is loaded from token (first step) / n_h and expanded
+// to one row per step in shared memory before the Gram product.
 // One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM (five when
 // gated), so the latency of the solve is hidden by parallelism across chunks.  A CTA's shared
 // memory is one 32 KB region that holds the unit's q/k tile until the product
@@ -167,6 +173,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.sched.H;
+    const int nh = p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
     const int units = count_chunks(p.sched) * H;
     if ((int)blockIdx.x >= units) return;
 
@@ -196,22 +203,26 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         const int id = u / H, head = u % H;
         int b, t0, t1;
         chunk_range(p.sched, id, b, t0, t1);
+        const int tq0 = nh > 1 ? t0 / nh : t0;  // token of the chunk's first step (q is per token)
         if (tid == 0) {
             sm100::mbar_expect_tx(&bars[0], 32768u);
             sm100::tma_load_4d(smem + L::OFF_QK + 8192, &tk, &bars[0], 0, head, t0, b);
-            sm100::tma_load_4d(smem + L::OFF_QK + 16384, &tq, &bars[0], 64, head, t0, b);
+            sm100::tma_load_4d(smem + L::OFF_QK + 16384, &tq, &bars[0], 64, head, tq0, b);
             sm100::tma_load_4d(smem + L::OFF_QK + 16384 + 8192, &tk, &bars[0], 64, head, t0, b);
             if (t_staged) sm100::bulk_wait_read0();
-            sm100::tma_load_4d(smem + L::OFF_QK, &tq, &bars[0], 0, head, t0, b);
+            sm100::tma_load_4d(smem + L::OFF_QK, &tq, &bars[0], 0, head, tq0, b);
         }
         if (tid < kChunk) {
             const bool ok = tid < t1 - t0;
             const float* src = p.beta + b * p.b_sb + (int64_t)(t0 + (ok ? tid : 0)) * p.b_st + head * p.b_sh;
             cp_async4(smem_addr(smem + L::OFF_BETA + (bb * kChunk + tid) * 4), src, ok ? 4 : 0);
             if constexpr (GATED) {
-                // log decays of the chunk (0 past its end: the pad rows are identity steps)
-                const float* gsrc = p.g + b * p.g_sb + (int64_t)(t0 + (ok ? tid : 0)) * p.g_st + head * p.g_sh;
-                cp_async4(smem_addr(smem + L::OFF_G + (bb * kChunk + tid) * 4), gsrc, ok ? 4 : 0);
+                // log decays of the chunk (0 past its end: the pad rows are identity steps;
+                // Gated Delta Product: the token's on its first step, 0 on the others)
+                const int m = t0 + (ok ? tid : 0);
+                const bool gok = ok && (nh == 1 || m % nh == 0);
+                const float* gsrc = p.g + b * p.g_sb + (int64_t)(nh > 1 ? m / nh : m) * p.g_st + head * p.g_sh;
+                cp_async4(smem_addr(smem + L::OFF_G + (bb * kChunk + tid) * 4), gsrc, gok ? 4 : 0);
             }
         }
         cp_async_commit();
@@ -230,6 +241,28 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         if (__syncthreads_or(!got)) break;
         in_flight = false;
         DN_TRP(it_, 1);
+        if (GATED && nh > 1) {
+            // Gated Delta Product: step row m of the q boxes takes token row (t0 + m) / n_h - tq0
+            // of the loaded boxes (128-byte rows whose 16-byte pieces are swizzled by row % 8)
+            int b_, t0_, t1_;
+            chunk_range(p.sched, u / H, b_, t0_, t1_);
+            const int tq0 = t0_ / nh;
+            uint4 w[8];
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const int id = tid + kPrepThreads * k8, a = id >> 9, m = (id >> 3) & 63, j = id & 7;
+                const int sr = (t0_ + m) / nh - tq0;
+                w[k8] = *reinterpret_cast<const uint4*>(smem + L::OFF_QK + a * 16384 + sr * 128 + ((j ^ (sr & 7)) * 16));
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const int id = tid + kPrepThreads * k8, a = id >> 9, m = (id >> 3) & 63, j = id & 7;
+                *reinterpret_cast<uint4*>(smem + L::OFF_QK + a * 16384 + m * 128 + ((j ^ (m & 7)) * 16)) = w[k8];
+            }
+            sm100::fence_async_smem();
+            __syncthreads();
+        }
         if constexpr (GATED) {
             // running sums c_l of the chunk's log decays (read after the next barrier)
             if (warp == 1) {

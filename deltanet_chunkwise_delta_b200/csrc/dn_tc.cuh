@@ -470,7 +470,10 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         // chunk's first product, which accumulates into it), staged as token rows (the
         // TMA box layout of out) and written by one TMA store per box; a chunk that
         // ends inside the run's last 64 tokens is written with bounded 16-byte stores.
+        // Gated Delta Product: rows are steps, and only a token's last step is written,
+        // to its token row (bounded stores).
         __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
+        const int nh = p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
         uint8_t* ob = smem + L::OFF_OB;
         auto store_o = [&](int c) -> bool {
             // read out and zero the columns first: the next chunk's first product waits
@@ -494,7 +497,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             DN_TR(q == 0, c, 28);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_OSTAGED], c & 1, abort_flag))) return false;
             const int t0 = it.tok0 + c * kChunk;
-            if (t0 + kChunk <= it.tok1) {
+            if (t0 + kChunk <= it.tok1 && nh == 1) {
                 if (q == 0 && lane == 0) {
                     tma_store_4d(&to, ob, 0, it.head, t0, it.b);
                     tma_store_4d(&to, ob + 8192, 64, it.head, t0, it.b);
@@ -506,7 +509,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 for (int k = 0; k < 8; ++k) {
                     const int id = 32 * q + lane + 128 * k, t = id >> 4, dc = id & 15;
                     const uint4 row = *reinterpret_cast<const uint4*>(ob + (dc >> 3) * 8192 + swz128(t, (dc & 7) * 8));
-                    if (t0 + t < it.tok1) *reinterpret_cast<uint4*>(og + (int64_t)(t0 + t) * p.o_st + 8 * dc) = row;
+                    const int m = t0 + t;
+                    if (m < it.tok1 && (m + 1) % nh == 0)
+                        *reinterpret_cast<uint4*>(og + (int64_t)(m / nh) * p.o_st + 8 * dc) = row;
                 }
             }
             __syncwarp();
