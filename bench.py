@@ -74,7 +74,7 @@ def algorithmic_bytes(w: wl.Workload, with_final: bool = True) -> float:
 
 # Sources that define the tensor-core boundary kernel's code (its parameter struct lives
 # in dn_common.cuh, whose fields do not change what the kernel reads or writes).
-BOUNDARY_KERNEL_SOURCES = ("dn_sm100.cuh", "dn_tc.cuh")
+BOUNDARY_KERNEL_SOURCES = ("dn_common.cuh", "dn_sm100.cuh", "dn_tc.cuh")
 
 
 def kernel_source_digest() -> str:
