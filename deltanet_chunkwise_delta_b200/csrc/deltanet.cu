@@ -210,14 +210,14 @@ EncodeTiledFn encode_fn() {
 // TMA map of a bf16 [B, T, H, 128] tensor (element strides sb, st, sh): boxes of
 // 64 tokens x 64 channels of one head, 128-byte swizzle, zero fill past T.
 dn_status make_token_map(CUtensorMap* m, const void* base, int64_t B, int64_t T, int64_t H,
-                         int64_t sb, int64_t st, int64_t sh) {
+                         int64_t sb, int64_t st, int64_t sh, int rows = 64) {
     std::memset(m, 0, sizeof *m);
     if (B * T == 0) return DN_OK;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return DN_ERR_CUDA;
     cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)sh * 2, (cuuint64_t)st * 2, (cuuint64_t)(sb > 0 ? sb : T * st) * 2};
-    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -268,9 +268,11 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kA = k_summary<E, DK, DV, STAGES, GATED, KDA>;
     auto* kS8 = k_scan<DK, DV, 8>;
     auto* kS16 = k_scan<DK, DV, 16>;
-    auto* kCt = tc::k_tc_chain<GATED>;
+    // the Gated Delta Product runs the instances that handle several steps per token
+    const bool multi = GATED && p.nh > 1;
+    auto* kCt = multi ? tc::k_tc_chain<GATED, GATED> : tc::k_tc_chain<GATED, false>;
     auto* kAt = tcs::k_tc_summary<GATED>;
-    auto* kPrep = k_ut_prep<GATED>;
+    auto* kPrep = multi ? k_ut_prep<GATED, GATED> : k_ut_prep<GATED, false>;
     constexpr int smemPrep = PrepSmemT<GATED>::TOTAL;
     constexpr int smemCt = tc::TcLay<GATED>::SMEM_BYTES, smemAt = tcs::SumLay<GATED>::SMEM_BYTES;
     dn_status st;
@@ -288,7 +290,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     }
     if ((st = set_smem(kS8, dev, smemS8)) != DN_OK) return st;
     if ((st = set_smem(kS16, dev, smemS16)) != DN_OK) return st;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv, to, toc;
     if (use_tc) {
         const int64_t Bq = d.varlen ? 1 : d.B;
         const int64_t Tq = d.T / (p.nh > 1 ? p.nh : 1);  // q and out: one row per token
@@ -296,6 +298,11 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
         if ((st = make_token_map(&tk, p.k, Bq, d.T, d.H, p.k_sb, p.k_st, p.k_sh)) != DN_OK) return st;
         if ((st = make_token_map(&tv, p.v, Bq, d.T, d.H, p.v_sb, p.v_st, p.v_sh)) != DN_OK) return st;
         if ((st = make_token_map(&to, p.o, Bq, Tq, d.H, p.o_sb, p.o_st, p.o_sh)) != DN_OK) return st;
+        // Gated Delta Product: a chunk's outputs are 64 / n_h token rows
+        toc = to;
+        if (p.nh > 1 && kChunk % p.nh == 0 &&
+            (st = make_token_map(&toc, p.o, Bq, Tq, d.H, p.o_sb, p.o_st, p.o_sh, kChunk / p.nh)) != DN_OK)
+            return st;
     }
 
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
@@ -429,7 +436,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             if (cudaEventRecord(aux.fork, stream) != cudaSuccess ||
                 cudaStreamWaitEvent(aux.stream, aux.fork, 0) != cudaSuccess)
                 return DN_ERR_CUDA;
-            kCt<<<(unsigned)chains, tc::kThreadsTc, smemCt, aux.stream>>>(tq, tk, tv, to, p0);
+            kCt<<<(unsigned)chains, tc::kThreadsTc, smemCt, aux.stream>>>(tq, tk, tv, to, toc, p0);
             ++launches;
             if (cudaEventRecord(aux.join, aux.stream) != cudaSuccess) return DN_ERR_CUDA;
             if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, smemAt, stream>>>(tk, tv, p); ++launches; }
@@ -438,14 +445,14 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             Params p1 = p;
             p1.sched.c_part = 2;
             if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-            kCt<<<(unsigned)(chains * (G - 1)), tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, p1);
+            kCt<<<(unsigned)(chains * (G - 1)), tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, toc, p1);
             ++launches;
             if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
         } else {
             if (nA > 0) { kAt<<<(unsigned)nA, tcs::kThreadsSum, smemAt, stream>>>(tk, tv, p); ++launches; }
             if (nScan > 0) { launch_scan(); ++launches; }
             if (g_ev_start) cudaEventRecord(g_ev_start, stream);
-            if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, p); ++launches; }
+            if (nC > 0) { kCt<<<(unsigned)nC, tc::kThreadsTc, smemCt, stream>>>(tq, tk, tv, to, toc, p); ++launches; }
             if (g_ev_stop) cudaEventRecord(g_ev_stop, stream);
         }
     } else {

@@ -231,7 +231,7 @@ extern "C" dn_status deltanet_fwd_noalloc(const dn_tensor* q, const dn_tensor* k
     const int grid = (int)(units < cap ? units : cap);
     dn::k_ut_prep<false><<<grid, dn::kPrepThreads, dn::PrepSmem::TOTAL, stream>>>(tq, tk, p);
     dn::tc::k_tc_chain<false><<<(unsigned)(B * H), dn::tc::kThreadsTc, dn::tc::SMEM_BYTES, stream>>>(
-        tq, tk, tv, to, p);
+        tq, tk, tv, to, to, p);
     return cudaGetLastError() == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

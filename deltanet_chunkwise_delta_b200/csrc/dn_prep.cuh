@@ -155,7 +155,9 @@ __device__ __forceinline__ void ld_blk(float (&acc)[2][4], const float* C) {
     }
 }
 
-template <bool GATED>
+// MULTI: the Gated Delta Product's instance (several steps per token); the others are
+// compiled with one step per token.
+template <bool GATED, bool MULTI = false>
 static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>())
     k_ut_prep(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk, Params p) {
     using L = PrepSmemT<GATED>;
@@ -173,7 +175,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.sched.H;
-    const int nh = p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
+    const int nh = MULTI && p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
     const int units = count_chunks(p.sched) * H;
     if ((int)blockIdx.x >= units) return;
 

@@ -185,10 +185,30 @@ __device__ __forceinline__ void store_token_rows(const RowFrags& f, int q, uint8
                           pack_bf16(scale * __uint_as_float(f.hi[g][2]), scale * __uint_as_float(f.hi[g][3])));
 }
 
-template <bool GATED>
+// As store_token_rows (scale 1), with token row 8 g + (lane & 7) written to staging row
+// prow[g] of this lane.
+__device__ __forceinline__ void store_token_rows_mapped(const RowFrags& f, int q, uint8_t* box0, uint32_t box_stride,
+                                                        const int (&prow)[8]) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t obox = saddr(box0) + (uint32_t)(q >> 1) * box_stride;
+    const int dcol = 32 * (q & 1) + 8 * (lane >> 3);
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+        stmatrix_x4_trans(obox + swz128(prow[g], dcol), pack_bf16(__uint_as_float(f.lo[g][0]), __uint_as_float(f.lo[g][1])),
+                          pack_bf16(__uint_as_float(f.lo[g][2]), __uint_as_float(f.lo[g][3])),
+                          pack_bf16(__uint_as_float(f.hi[g][0]), __uint_as_float(f.hi[g][1])),
+                          pack_bf16(__uint_as_float(f.hi[g][2]), __uint_as_float(f.hi[g][3])));
+}
+
+// toc: Gated Delta Product with n_h dividing 64, a map over out with boxes of 64 / n_h
+// token rows (a chunk's outputs); otherwise the same as to.
+// MULTI: the Gated Delta Product's instance (several steps per token); the others are
+// compiled with one step per token.
+template <bool GATED, bool MULTI = false>
 static __global__ void __launch_bounds__(kThreadsTc, 1)
     k_tc_chain(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
+               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+               const __grid_constant__ CUtensorMap toc, Params p) {
     using L = TcLay<GATED>;
     constexpr int kUnit = unit_bytes(GATED);
     extern __shared__ uint8_t smem_raw[];
@@ -473,7 +493,17 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         // Gated Delta Product: rows are steps, and only a token's last step is written,
         // to its token row (bounded stores).
         __nv_bfloat16* og = static_cast<__nv_bfloat16*>(p.o) + it.b * p.o_sb + it.head * p.o_sh;
-        const int nh = p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
+        const int nh = MULTI && p.nh > 1 ? p.nh : 1;  // steps per token (Gated Delta Product)
+        // Gated Delta Product with n_h dividing 64: a full chunk's outputs (a token's last
+        // step) are packed into staging rows 0 .. 64 / n_h - 1 and written with one TMA store
+        // per box; the other steps' rows go to distinct rows past them
+        const bool packed_o = MULTI && nh > 1 && kChunk % nh == 0;
+        int prow[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const int t = 8 * g + (lane & 7), kept = kChunk / nh;
+            prow[g] = !MULTI ? t : (t + 1) % nh == 0 ? t / nh : kept + t % (kChunk - kept);
+        }
         uint8_t* ob = smem + L::OFF_OB;
         auto store_o = [&](int c) -> bool {
             // read out and zero the columns first: the next chunk's first product waits
@@ -490,17 +520,21 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             // the staging buffer is released by chunk c - 1's store
             if (c >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_OBFREE], (c - 1) & 1, abort_flag)))
                 return false;
-            store_token_rows(f, q, ob, 8192, 1.f);
+            const int t0 = it.tok0 + c * kChunk;
+            const bool full = t0 + kChunk <= it.tok1;
+            if (MULTI && packed_o && full) store_token_rows_mapped(f, q, ob, 8192, prow);
+            else store_token_rows(f, q, ob, 8192, 1.f);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[B_OSTAGED]);
             DN_TR(q == 0, c, 28);
             if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_OSTAGED], c & 1, abort_flag))) return false;
-            const int t0 = it.tok0 + c * kChunk;
-            if (t0 + kChunk <= it.tok1 && nh == 1) {
+            if (full && (nh == 1 || packed_o)) {
                 if (q == 0 && lane == 0) {
-                    tma_store_4d(&to, ob, 0, it.head, t0, it.b);
-                    tma_store_4d(&to, ob + 8192, 64, it.head, t0, it.b);
+                    const CUtensorMap* om = MULTI && nh > 1 ? &toc : &to;
+                    const int r0 = MULTI && nh > 1 ? t0 / nh : t0;
+                    tma_store_4d(om, ob, 0, it.head, r0, it.b);
+                    tma_store_4d(om, ob + 8192, 64, it.head, r0, it.b);
                     bulk_commit();
                     bulk_wait_read0();
                 }
