@@ -295,26 +295,31 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         sm100::tc_fence_after();
         if constexpr (GATED) {
             // Q<- = diag(lambda[1:l]) Q: the unit's two q boxes (128-byte rows, swizzled
-            // within the row) scaled per token row and written out unchanged in layout,
-            // before the solve's blocks overwrite them
+            // within the row) scaled per token row in place and copied out unchanged in
+            // layout by two bulk stores, whose reads complete before the solve's blocks
+            // overwrite the region (asynchronous copies: no ordinary global store is left in
+            // flight ahead of the tensor-memory reads below)
             const float* lam = reinterpret_cast<const float*>(smem + L::OFF_LAM);
-            uint8_t* dst = p.wsT + (size_t)u * kUnit + kUnitQL;
-            uint4 w[8];
 #pragma unroll
             for (int k8 = 0; k8 < 8; ++k8) {
                 const int id = tid + kPrepThreads * k8, a = id >> 9, row = (id >> 3) & 63, pc = id & 7;
-                w[k8] = *reinterpret_cast<const uint4*>(smem + L::OFF_QK + a * 16384 + row * 128 + pc * 16);
-            }
-#pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) {
-                const int id = tid + kPrepThreads * k8, a = id >> 9, row = (id >> 3) & 63, pc = id & 7;
+                uint4* ptr = reinterpret_cast<uint4*>(smem + L::OFF_QK + a * 16384 + row * 128 + pc * 16);
                 const float f = lam[row];
-                uint4 v = w[k8];
+                uint4 v = *ptr;
                 v.x = scale_pair(v.x, f);
                 v.y = scale_pair(v.y, f);
                 v.z = scale_pair(v.z, f);
                 v.w = scale_pair(v.w, f);
-                *reinterpret_cast<uint4*>(dst + a * 8192 + row * 128 + pc * 16) = v;
+                *ptr = v;
+            }
+            sm100::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                uint8_t* dst = p.wsT + (size_t)u * kUnit + kUnitQL;
+                sm100::bulk_store(dst, smem + L::OFF_QK, 8192);
+                sm100::bulk_store(dst + 8192, smem + L::OFF_QK + 16384, 8192);
+                sm100::bulk_commit();
+                sm100::bulk_wait_read0();
             }
             __syncthreads();
         }
