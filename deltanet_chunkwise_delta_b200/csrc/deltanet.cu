@@ -252,10 +252,22 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
                  const int* cu) {
     // bf16 DeltaNet, Gated DeltaNet and the Gated Delta Product with d_k = d_v = 128 run on
     // the tensor-core (tcgen05) kernels (with or without the chunk-start states), the other
-    // shapes on the mma.sync chain kernels (Kimi Delta Attention, a decay per key channel,
-    // runs on the mma.sync chain kernels)
-    constexpr bool kTcShape = !KDA && std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
-    const bool use_tc = kTcShape && (p.nh <= 1 || GATED);
+    // shapes on the mma.sync chain kernels.  Kimi Delta Attention (a decay per key channel)
+    // with d_k = d_v = 128 runs on its tensor-core pre-pass and boundary kernel when a dense
+    // batch's chains are not split (one run per chain; there is no KDA summary pass on the
+    // tensor cores), otherwise on the mma.sync chain kernels.
+    constexpr bool kBf16x128 = std::is_same<E, __nv_bfloat16>::value && DK == 128 && DV == 128;
+    constexpr bool kTcShape = !KDA && kBf16x128;
+    bool use_tc = kTcShape && (p.nh <= 1 || GATED);
+    if constexpr (KDA && kBf16x128) {
+        if (!d.varlen) {
+            const int64_t n_c = (d.T + kChunk - 1) / kChunk;
+            const int s1 = forced_s > 0 ? (forced_s & 0xffff)
+                                        : choose_dense(CostModel{}, (int)(d.N * d.H), (int)n_c, sms,
+                                                       kAutoMaxSlots, false).s;
+            use_tc = s1 >= n_c;
+        }
+    }
     using LC = ChainSmem<E, DK, DV, true, true, STAGES, GATED, KDA>;
     using LH = ChainSmem<E, DK, DV, true, false, STAGES, GATED, KDA>;
     using LP = ChainSmem<E, DK, DK, false, false, STAGES, GATED, KDA>;
@@ -270,20 +282,32 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     auto* kS16 = k_scan<DK, DV, 16>;
     // the Gated Delta Product runs the instances that handle several steps per token
     const bool multi = GATED && p.nh > 1;
-    auto* kCt = multi ? tc::k_tc_chain<GATED, GATED> : tc::k_tc_chain<GATED, false>;
+    // KDA's tensor-core instances: the gated layout with K<- and K-> from its own pre-pass
+    constexpr bool kKdaTc = KDA && kBf16x128;
+    auto* kCt = kKdaTc ? tc::k_tc_chain<true, false, kKdaTc>
+                       : (multi ? tc::k_tc_chain<GATED, GATED> : tc::k_tc_chain<GATED, false>);
     auto* kAt = tcs::k_tc_summary<GATED>;
     auto* kPrep = multi ? k_ut_prep<GATED, GATED> : k_ut_prep<GATED, false>;
-    constexpr int smemPrep = PrepSmemT<GATED>::TOTAL;
-    constexpr int smemCt = tc::TcLay<GATED>::SMEM_BYTES, smemAt = tcs::SumLay<GATED>::SMEM_BYTES;
+    constexpr int smemPrep = kKdaTc ? KdaPrepLay::TOTAL : PrepSmemT<GATED>::TOTAL;
+    constexpr int smemCt = kKdaTc ? tc::TcLay<true, true>::SMEM_BYTES : tc::TcLay<GATED>::SMEM_BYTES;
+    constexpr int smemAt = tcs::SumLay<GATED>::SMEM_BYTES;
     dn_status st;
     if (use_tc) {
         if ((st = set_smem(kCt, dev, smemCt)) != DN_OK) return st;
         if ((st = set_smem(kAt, dev, smemAt)) != DN_OK) return st;
-        if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
-        // several pre-pass CTAs share an SM: ask for the largest shared-memory carveout
-        if (cudaFuncSetAttribute(kPrep, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-            return DN_ERR_CUDA;
+        if constexpr (kKdaTc) {
+            auto* kKp = k_kda_prep<DK>;
+            if ((st = set_smem(kKp, dev, smemPrep)) != DN_OK) return st;
+            if (cudaFuncSetAttribute(kKp, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+                return DN_ERR_CUDA;
+        } else {
+            if ((st = set_smem(kPrep, dev, smemPrep)) != DN_OK) return st;
+            // several pre-pass CTAs share an SM: ask for the largest shared-memory carveout
+            if (cudaFuncSetAttribute(kPrep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+                return DN_ERR_CUDA;
+        }
     } else {
         if ((st = set_smem(kC, dev, smemC)) != DN_OK) return st;
         if ((st = set_smem(kA, dev, smemA)) != DN_OK) return st;
@@ -308,7 +332,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     const int64_t n_c_max = (d.T + kChunk - 1) / kChunk;
     const int64_t chains = d.N * d.H;
     CostModel model;
-    if (use_tc) model.a = kTcSummaryCost;
+    if (use_tc && !KDA) model.a = kTcSummaryCost;
     size_t bytes = 0;
     int64_t slots = 0, nC = 0, nA = 0, nScan = 0;
     int G = 1, s = 1, s0 = 0;
@@ -319,7 +343,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
             s0 = (forced_s >> 16) & 0x7fff;
             if (s < 1 || s0 > s) return DN_ERR_INVALID_ARG;
         } else {
-            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, use_tc);
+            SegChoice ch = choose_dense(model, (int)chains, (int)n_c_max, sms, kAutoMaxSlots, use_tc && !KDA);
             s = ch.s;
             s0 = ch.s0;
         }
@@ -361,7 +385,7 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     // UT factors of every (chunk, head): chunks <= ceil(T / C) per row (+1 per sequence)
     const int64_t chunk_ub = d.varlen ? n_c_max + d.N : d.B * n_c_max;
     const size_t off_T = off_SS + up256((size_t)slots * DK * DV * 4);
-    bytes = off_T + (use_tc ? (size_t)chunk_ub * d.H * unit_bytes(GATED) : 0);
+    bytes = off_T + (use_tc ? (size_t)chunk_ub * d.H * (KDA ? kKdaUnitBytes : unit_bytes(GATED)) : 0);
     StreamWs ws;
     if ((st = get_ws(dev, stream, bytes, ws)) != DN_OK) return st;
     char* base = ws.buf;
@@ -422,8 +446,13 @@ dn_status launch(Params p, const Dims& d, int dev, int sms, cudaStream_t stream,
     if (use_tc) {
         const int64_t units = chunk_ub * d.H;
         if (units > 0) {
-            const int grid = (int)std::min<int64_t>(units, (int64_t)sms * prep_ctas_per_sm<GATED>());
-            kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
+            if constexpr (kKdaTc) {
+                const int grid = (int)std::min<int64_t>(units, (int64_t)sms * 2);
+                k_kda_prep<DK><<<grid, kThreads, smemPrep, stream>>>(p);
+            } else {
+                const int grid = (int)std::min<int64_t>(units, (int64_t)sms * prep_ctas_per_sm<GATED>());
+                kPrep<<<grid, kPrepThreads, smemPrep, stream>>>(tq, tk, p);
+            }
             ++launches;
         }
         if (e_in_c) {

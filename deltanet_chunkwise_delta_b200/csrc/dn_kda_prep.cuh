@@ -1,0 +1,211 @@
+// Kimi Delta Attention: the chunk-parallel pre-pass of the tensor-core path
+// (bf16, d_k = d_v = 128).
+//
+// "Linear Attention, Visualized", section "Kimi Delta Attention (KDA)", complete
+// per-chunk algorithm: every key channel c decays by its own a_t[c] = exp(g_t[c]).
+// With G_l = g_1 + ... + g_l per channel (within the chunk) the chunk's factors are
+//   L[l][m] = sum_c k_l[c] k_m[c] exp(G_l[c] - G_m[c])   (m < l)
+//   P[l][m] = sum_c q_l[c] k_m[c] exp(G_l[c] - G_m[c])   (m <= l)
+//   T = (I + B L)^{-1} B,  Q<- = exp(G) o Q,  K<- = exp(G) o K,  K-> = exp(G_C - G) o K,
+//   lambda[1:C] = exp(G_C) per channel.
+// The chain kernels then need no gate arithmetic: W = T K<-, U = T V,
+// Z = U - W S, O = Q<- S + P Z, S' = Diag(lambda[1:C]) S + K->^T Z.
+// Like "Context Parallelism for DeltaNet", section 2, step 1, all of it depends only on
+// the chunk's own inputs, so one CTA forms one (chunk, head) unit at a time and the
+// units run in parallel.  L and P are formed block by block of 16 rows against the
+// block's first row s (exp(G_l - G_m) = exp(G_l - G_s) exp(G_s - G_m)), which keeps
+// every factor in range for |g| < 5.8 per token and channel (see dn_chain.cuh).
+//
+// Unit layout in the workspace (66,560 bytes per (chunk, head)): T and P (bf16 64 x 64,
+// 128-byte rows, 16-byte pieces swizzled by row % 8: the tensor cores' operand layout),
+// Q<-, K<-, K-> (each two boxes of 64 channels x 64 rows in the same layout, the layout a
+// TMA load of the tile would give), lambda[1:C] per channel (fp32).
+#pragma once
+
+#include "dn_chain.cuh"
+#include "dn_common.cuh"
+#include "dn_warp_gemm.cuh"
+
+namespace dn {
+
+constexpr int kKdaUnitT = 0, kKdaUnitP = 8192, kKdaUnitQL = 16384, kKdaUnitKL = 32768, kKdaUnitKR = 49152,
+              kKdaUnitF = 65536, kKdaUnitFBytes = 512;
+constexpr int kKdaUnitBytes = 66560;
+
+// Shared memory of the KDA pre-pass (byte offsets).  [0, OFF_AF) holds the chunk's k, q,
+// log decays and the block operands until the scaled tiles are written out; the solve's
+// N, X and T tiles then reuse it.
+struct KdaPrepLay {
+    static constexpr int DK = 128;
+    static constexpr int OFF_K = 0;          // 64 x 128 bf16 (Swz): K, later K->
+    static constexpr int OFF_Q = 16384;      // 64 x 128 bf16 (Swz): Q, later Q<-
+    static constexpr int OFF_G = 32768;      // 64 x 128 fp32: log decays, later running sums
+    static constexpr int OFF_R = 65536;      // 64 x 128 bf16 (Swz): a block's right operand, later K<-
+    static constexpr int OFF_LQ = 81920;     // 32 x 128 bf16 (Swz): a block's left operands [K; Q]
+    static constexpr int OFF_N = 0;          // after the tiles: N, 64 x 65 fp32
+    static constexpr int OFF_X = 16640;      //   the solve's staging, 3 x 256 fp32
+    static constexpr int OFF_T = 19712;      //   T, 64 x 64 bf16 (Swz)
+    static constexpr int OFF_AF = 90112;     // A = B L, 64 x 65 fp32
+    static constexpr int OFF_P = 106752;     // P, 64 x 64 bf16 (Swz)
+    static constexpr int OFF_BETA = 114944;  // 64 fp32
+    static constexpr int OFF_LAMC = 115200;  // lambda[1:C], 128 fp32
+    static constexpr int TOTAL = 115712;     // two CTAs per SM
+};
+static_assert(KdaPrepLay::OFF_T + 8192 <= KdaPrepLay::OFF_AF, "solve tiles fit the freed region");
+
+// One 64-row bf16 tile of width W (Swz layout) -> global, as W / 64 boxes of 64 channels
+// x 64 rows with 128-byte rows: row r's bytes [128 a, 128 a + 128) are row r of box a
+// (the 16-byte pieces keep their order: both layouts swizzle them by row % 8 within 128
+// bytes).  All threads.
+template <int W>
+__device__ __forceinline__ void tile_to_boxes(uint8_t* dst, const __nv_bfloat16* src) {
+    constexpr int PR = W / 8;  // 16-byte pieces per row
+    for (int idx = threadIdx.x; idx < kChunk * PR; idx += kThreads) {
+        const int r = idx / PR, pc = idx % PR;
+        const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(src) + r * (W * 2) + pc * 16);
+        *reinterpret_cast<uint4*>(dst + (pc >> 3) * 8192 + r * 128 + (pc & 7) * 16) = v;
+    }
+}
+
+template <int DK>
+static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
+    static_assert(DK == KdaPrepLay::DK, "the tensor-core path has d_k = 128");
+    using E = __nv_bfloat16;
+    using SW = Swz<E>;
+    using L = KdaPrepLay;
+    constexpr int LD = 65;  // fp32 solve tiles
+    extern __shared__ __align__(128) char kda_smem[];
+    E* Kc = reinterpret_cast<E*>(kda_smem + L::OFF_K);
+    E* Qc = reinterpret_cast<E*>(kda_smem + L::OFF_Q);
+    float* G = reinterpret_cast<float*>(kda_smem + L::OFF_G);
+    E* Rs = reinterpret_cast<E*>(kda_smem + L::OFF_R);
+    E* LQs = reinterpret_cast<E*>(kda_smem + L::OFF_LQ);
+    float* Nf = reinterpret_cast<float*>(kda_smem + L::OFF_N);
+    float* Xt = reinterpret_cast<float*>(kda_smem + L::OFF_X);
+    E* Ts = reinterpret_cast<E*>(kda_smem + L::OFF_T);
+    float* Af = reinterpret_cast<float*>(kda_smem + L::OFF_AF);
+    E* Ps = reinterpret_cast<E*>(kda_smem + L::OFF_P);
+    float* bc = reinterpret_cast<float*>(kda_smem + L::OFF_BETA);
+    float* lamc = reinterpret_cast<float*>(kda_smem + L::OFF_LAMC);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const int H = p.sched.H;
+    const int units = count_chunks(p.sched) * H;
+
+#pragma unroll 1
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int head = u % H;
+        int b, t0, t1;
+        chunk_range(p.sched, u / H, b, t0, t1);
+        const int rows = t1 - t0;
+        uint8_t* unit = p.wsT + (size_t)u * kKdaUnitBytes;
+
+        // the chunk's k, q, beta and log decays (rows past the chunk: zeros, identity steps)
+        const E* kg = static_cast<const E*>(p.k) + b * p.k_sb + head * p.k_sh;
+        const E* qg = static_cast<const E*>(p.q) + b * p.q_sb + head * p.q_sh;
+        const float* bg = p.beta + b * p.b_sb + head * p.b_sh;
+        const float* gg = p.g + b * p.g_sb + head * p.g_sh;
+        load_tile<E, DK>(Kc, kg + (int64_t)t0 * p.k_st, p.k_st, rows);
+        load_tile<E, DK>(Qc, qg + (int64_t)t0 * p.q_st, p.q_st, rows);
+        if (tid < kChunk) {
+            const bool ok = tid < rows;
+            cp_async4(smem_addr(bc + tid), ok ? bg + (int64_t)(t0 + tid) * p.b_st : bg, ok ? 4 : 0);
+        }
+        for (int idx = tid; idx < kChunk * (DK / 4); idx += kThreads) {
+            const int rr = idx / (DK / 4), c = idx % (DK / 4);
+            const bool ok = rr < rows;
+            const float* src = ok ? gg + (int64_t)(t0 + rr) * p.g_st + 4 * c : gg;
+            cp_async16(smem_addr(G + rr * DK + 4 * c), src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+
+        // running sums per key channel, in place, and lambda[1:C]
+        if (tid < DK) {
+            float acc = 0.f;
+            for (int l = 0; l < kChunk; ++l) {
+                acc += G[l * DK + tid];
+                G[l * DK + tid] = acc;
+            }
+            lamc[tid] = expf(acc);
+        }
+        __syncthreads();
+
+        // rows 16 b .. 16 b + 15 of A = B L (fp32, strict lower) and of P (inclusive),
+        // against reference row s = 16 b
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+            const int s = 16 * blk, ncol = s + 16;
+            for (int idx = tid; idx < ncol * DK; idx += kThreads) {
+                const int m = idx / DK, c = idx % DK;
+                const int o = SW::template off<DK>(m, c);
+                Rs[o] = __float2bfloat16_rn(__bfloat162float(Kc[o]) * expf(G[s * DK + c] - G[m * DK + c]));
+            }
+            for (int idx = tid; idx < 16 * DK; idx += kThreads) {
+                const int lr = idx / DK, c = idx % DK, l = s + lr;
+                const float f = expf(G[l * DK + c] - G[s * DK + c]);
+                const int o = SW::template off<DK>(l, c), ol = SW::template off<DK>(lr, c);
+                LQs[ol] = __float2bfloat16_rn(__bfloat162float(Kc[o]) * f);
+                LQs[16 * DK + ol] = __float2bfloat16_rn(__bfloat162float(Qc[o]) * f);
+            }
+            // the block's rows right of its last column are zero in both
+            for (int idx = tid; idx < 16 * (kChunk - ncol); idx += kThreads) {
+                const int row = s + idx / (kChunk - ncol), col = ncol + idx % (kChunk - ncol);
+                Af[row * LD + col] = 0.f;
+                Ps[SW::template off<kChunk>(row, col)] = __float2bfloat16_rn(0.f);
+            }
+            __syncthreads();
+            const int ntile = blk + 1;
+            if (warp < 2 * ntile) {
+                const int mat = warp / ntile, j = warp % ntile;
+                float acc[2][4];
+                zero_frag(acc);
+                warp_gemm<DK, 2, DK, false, DK, false>(acc, LQs + mat * 16 * DK, 0, Rs, 16 * j);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int row = s + g8 + 8 * (e >> 1);
+                        const int col = 16 * j + 8 * nt + 2 * t4 + (e & 1);
+                        if (mat == 0) Af[row * LD + col] = col < row ? bc[row] * acc[nt][e] : 0.f;
+                        else acc[nt][e] = col > row ? 0.f : acc[nt][e];
+                    }
+                if (mat == 1) store_frag<2, kChunk>(Ps, s, 16 * j, acc, 1.f);
+            }
+            __syncthreads();
+        }
+
+        // K<- = exp(G) o K, K-> = exp(G_C - G) o K, Q<- = exp(G) o Q, then out to the unit
+        for (int idx = tid; idx < kChunk * DK; idx += kThreads) {
+            const int l = idx / DK, c = idx % DK;
+            const int o = SW::template off<DK>(l, c);
+            const float gl = G[l * DK + c], gC = G[(kChunk - 1) * DK + c];
+            const float kv = __bfloat162float(Kc[o]);
+            Rs[o] = __float2bfloat16_rn(kv * expf(gl));
+            Kc[o] = __float2bfloat16_rn(kv * expf(gC - gl));
+            Qc[o] = __float2bfloat16_rn(__bfloat162float(Qc[o]) * expf(gl));
+        }
+        __syncthreads();
+        tile_to_boxes<DK>(unit + kKdaUnitQL, Qc);
+        tile_to_boxes<DK>(unit + kKdaUnitKL, Rs);
+        tile_to_boxes<DK>(unit + kKdaUnitKR, Kc);
+        if (tid < DK / 4)
+            reinterpret_cast<float4*>(unit + kKdaUnitF)[tid] = reinterpret_cast<const float4*>(lamc)[tid];
+        __syncthreads();  // the region is taken by the solve's tiles next
+
+        // T = (I + B L)^{-1} B
+        ut_solve<E>(Af, Nf, Xt, bc, Ts);
+        __syncthreads();
+        for (int idx = tid; idx < 2 * 512; idx += kThreads) {
+            const int t = idx >> 9, pc = idx & 511;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(t == 0 ? Ts : Ps);
+            *reinterpret_cast<uint4*>(unit + (t == 0 ? kKdaUnitT : kKdaUnitP) + pc * 16) =
+                *reinterpret_cast<const uint4*>(src + pc * 16);
+        }
+        __syncthreads();  // the next unit's loads overwrite the tiles
+    }
+}
+
+}  // namespace dn

@@ -39,6 +39,7 @@
 #pragma once
 
 #include "dn_common.cuh"
+#include "dn_kda_prep.cuh"
 #include "dn_sm100.cuh"
 
 namespace dn {
@@ -68,18 +69,24 @@ constexpr int kTmaBWarp = 15;
 // Gated DeltaNet: ring Q holds Q<- = diag(lambda[1:l]) Q from the pre-pass and has two
 // stages, ring B stages also hold T' = T diag(lambda[1:l]) (the W<- factor), and each P
 // buffer is followed by the chunk's row factors (lambda[l+1:C] per row, lambda[1:C]).
-constexpr int NB = 2, NK = 3, NE = 6;
+// Kimi Delta Attention (KDA, built on the gated layout): ring B stages hold K<- (the W
+// factor, with T) in place of T', ring K holds K-> (the state update's operand, 2 stages),
+// both from the KDA pre-pass, and the factors after each P tile are lambda[1:C] per key
+// channel.
+constexpr int NB = 2, NE = 6;
 constexpr int Q_STAGE = 32768, K_STAGE = 16384;
 __host__ __device__ constexpr int a_w(int c) { return (c & 1) ? 8192 : 0; }  // -W rows of chunk c
 __host__ __device__ constexpr int a_q(int c) { return (c & 1) ? 0 : 8192; }  // Q rows of chunk c
 constexpr int B_T = 16384, B_T2 = 24576;
 constexpr int NBAR = 42;
-template <bool GATED>
+constexpr int B_KL = 24576;  // KDA: K<- in a ring-B stage (two 64-channel boxes)
+template <bool GATED, bool KDA = false>
 struct TcLay {
     static constexpr int NQ = GATED ? 2 : 3;
+    static constexpr int NK = KDA ? 2 : 3;
     static constexpr int OFF_K = NQ * Q_STAGE;
     static constexpr int OFF_B = OFF_K + NK * K_STAGE;
-    static constexpr int B_STAGE = GATED ? 32768 : 24576;  // V, T (, T')
+    static constexpr int B_STAGE = KDA ? 40960 : (GATED ? 32768 : 24576);  // V, T (, T' | K<-)
     static constexpr int PB_STRIDE = GATED ? 9216 : 8192;  // P tile (+ row factors)
     static constexpr int OFF_PB = OFF_B + NB * B_STAGE;
     static constexpr int OFF_OB = OFF_PB + 2 * PB_STRIDE;  // O staging
@@ -88,7 +95,9 @@ struct TcLay {
     static constexpr int SMEM_USED = OFF_MISC + 64;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 };
-static_assert(TcLay<false>::SMEM_BYTES <= 232448 && TcLay<true>::SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(TcLay<false>::SMEM_BYTES <= 232448 && TcLay<true>::SMEM_BYTES <= 232448 &&
+                  TcLay<true, true>::SMEM_BYTES <= 232448,
+              "shared memory budget");
 constexpr int SMEM_BYTES = TcLay<false>::SMEM_BYTES;
 
 // tensor-memory columns (512 allocated): S^T fp32, [O^T (odd chunks) | U^T/Z^T |
@@ -203,14 +212,18 @@ __device__ __forceinline__ void store_token_rows_mapped(const RowFrags& f, int q
 // toc: Gated Delta Product with n_h dividing 64, a map over out with boxes of 64 / n_h
 // token rows (a chunk's outputs); otherwise the same as to.
 // MULTI: the Gated Delta Product's instance (several steps per token); the others are
-// compiled with one step per token.
-template <bool GATED, bool MULTI = false>
+// compiled with one step per token.  KDA: Kimi Delta Attention's instance (with GATED).
+template <bool GATED, bool MULTI = false, bool KDA = false>
 static __global__ void __launch_bounds__(kThreadsTc, 1)
     k_tc_chain(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
                const __grid_constant__ CUtensorMap toc, Params p) {
-    using L = TcLay<GATED>;
-    constexpr int kUnit = unit_bytes(GATED);
+    static_assert(!KDA || (GATED && !MULTI), "KDA runs on the gated layout, one step per token");
+    using L = TcLay<GATED, KDA>;
+    constexpr int NK = L::NK;
+    constexpr int kUnit = KDA ? kKdaUnitBytes : unit_bytes(GATED);
+    constexpr int kUnitQ = KDA ? kKdaUnitQL : kUnitQL;
+    constexpr int kUnitFac = KDA ? kKdaUnitF : kUnitF;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -289,9 +302,17 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 if (r >= NK && !mbar_wait(&bars[B_EMPTY + (r - NK) % NE], ((r - NK) / NE) & 1, abort_flag)) break;
                 mbar_expect_tx(&bars[B_FULLK + sk], 16384u);
                 uint8_t* stk = smem + L::OFF_K + sk * K_STAGE;
+                if constexpr (KDA) {
+                    // K-> of the chunk, from the KDA pre-pass (two 8 KB boxes)
+                    const uint8_t* kr =
+                        p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit + kKdaUnitKR;
 #pragma unroll
-                for (int a = 0; a < 2; ++a)
-                    tma_load_4d(stk + a * 8192, &tk, &bars[B_FULLK + sk], a * 64, it.head, t0, it.b);
+                    for (int a = 0; a < 2; ++a) bulk_load(stk + a * 8192, kr + a * 8192, 8192, &bars[B_FULLK + sk]);
+                } else {
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+                        tma_load_4d(stk + a * 8192, &tk, &bars[B_FULLK + sk], a * 64, it.head, t0, it.b);
+                }
                 issued_k = r + 1;
                 const int sq = r % L::NQ;
                 if (L::NQ < NK && r >= L::NQ &&
@@ -301,7 +322,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 uint8_t* stq = smem + sq * Q_STAGE;
                 if constexpr (GATED) {
                     // Q<- of the chunk, from the pre-pass (two 8 KB boxes)
-                    const uint8_t* ql = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit + kUnitQL;
+                    const uint8_t* ql = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit + kUnitQ;
 #pragma unroll
                     for (int a = 0; a < 2; ++a) bulk_load(stq + a_q(r) + a * 16384, ql + a * 8192, 8192, &bars[B_FULLQ + sq]);
                 } else {
@@ -322,7 +343,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
     } else if (warp == kTmaBWarp) {
         // ------------------------------------------------------------ ring B: v, T
         if (lane == 0 && nch > 0) {
-            const uint32_t bytes = 16384u + 8192u + (GATED ? 8192u : 0u);
+            const uint32_t bytes = 16384u + 8192u + (KDA ? 16384u : (GATED ? 8192u : 0u));
             int issued = 0;
             for (int r = 0; r < nch; ++r) {
                 const int s = r & 1;
@@ -335,7 +356,12 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                     tma_load_4d(st + a * 8192, &tv, &bars[B_FULLB + s], a * 64, it.head, t0, it.b);
                 const uint8_t* unit = p.wsT + ((size_t)(it.cbase + r) * p.sched.H + it.head) * kUnit;
                 bulk_load(st + B_T, unit, 8192, &bars[B_FULLB + s]);
-                if constexpr (GATED) bulk_load(st + B_T2, unit + kUnitT2, 8192, &bars[B_FULLB + s]);
+                if constexpr (KDA) {
+                    bulk_load(st + B_KL, unit + kKdaUnitKL, 8192, &bars[B_FULLB + s]);
+                    bulk_load(st + B_KL + 8192, unit + kKdaUnitKL + 8192, 8192, &bars[B_FULLB + s]);
+                } else if constexpr (GATED) {
+                    bulk_load(st + B_T2, unit + kUnitT2, 8192, &bars[B_FULLB + s]);
+                }
                 issued = r + 1;
             }
             volatile int drain = 0;
@@ -356,7 +382,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint64_t dK = sdesc(sb + L::OFF_K, 8192, 1024);  // K, MN-major
             // the state update's A operand: Z^T, or for Gated DeltaNet Z^T diag(lambda[l+1:C])
             // (so that the update adds K->^T Z)
-            constexpr uint32_t tm_zs = GATED ? TM_ZBF2 : TM_ZBF;
+            constexpr uint32_t tm_zs = GATED && !KDA ? TM_ZBF2 : TM_ZBF;  // KDA: K-> in ring K
             const uint64_t dP = sdesc(sb + L::OFF_PB, 16, 1024);   // P^T, K-major (+ 8 KB for odd chunks)
             for (int r = 0; r < nch; ++r) {
                 const int s = r & 1;
@@ -379,7 +405,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 umma_commit(&bars[B_C1]);
                 mbar_arrive(&bars[B_GAP1 + s]);
                 DN_TR(true, r, 1);
-                if (!mbar_wait(&bars[B_ZFULL], r & 1, abort_flag)) break;
+                if (!(KDA ? mbar_wait2(&bars[B_ZFULL], r & 1, &bars[B_FULLK + r % NK], (r / NK) & 1, abort_flag)
+                          : mbar_wait(&bars[B_ZFULL], r & 1, abort_flag)))
+                    break;
                 DN_TR(true, r, 10);
                 tc_fence_after();
                 // S^T += Z^T K
@@ -421,13 +449,16 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint64_t dVT = sdesc(sb + L::OFF_B, 8192, 1024);        // V^T, MN-major
             const uint64_t dT = sdesc(sb + L::OFF_B + B_T, 16, 1024);     // T^T, K-major
             // W = T K, or for Gated DeltaNet W<- = T' K with T' = T diag(lambda[1:l])
-            const uint64_t dTw = GATED ? sdesc(sb + L::OFF_B + B_T2, 16, 1024) : dT;
+            const uint64_t dTw = GATED && !KDA ? sdesc(sb + L::OFF_B + B_T2, 16, 1024) : dT;
+            // KDA: W = T K<- with K<- in ring B
+            const uint64_t dKLT = sdesc(sb + L::OFF_B + B_KL, 8192, 1024);
             auto issue_w = [&](int c) {
-                const uint64_t stk = (uint64_t)(((c % NK) * K_STAGE) >> 4);
+                const uint64_t stk = KDA ? (uint64_t)(((c & 1) * L::B_STAGE) >> 4)
+                                         : (uint64_t)(((c % NK) * K_STAGE) >> 4);
                 const uint64_t stb = (uint64_t)(((c & 1) * L::B_STAGE) >> 4);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    umma_bf16(tmem + TM_WT, dKT + stk + (uint64_t)((j * 2048) >> 4),
+                    umma_bf16(tmem + TM_WT, (KDA ? dKLT : dKT) + stk + (uint64_t)((j * 2048) >> 4),
                               dTw + stb + (uint64_t)((j * 32) >> 4), i_tt, j > 0);
                 umma_commit(&bars[B_WUFULL]);
             };
@@ -442,7 +473,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 umma_commit(&bars[B_UFULL]);
                 umma_commit(&bars[B_EMPTYB + s]);
             };
+            // (KDA: W^T reads K<- from ring B; ring K's K-> is the state update's alone)
             auto wait_data = [&](int c) -> bool {
+                if constexpr (KDA) return mbar_wait(&bars[B_FULLB + (c & 1)], (c >> 1) & 1, abort_flag);
                 return mbar_wait2(&bars[B_FULLK + c % NK], (c / NK) & 1, &bars[B_FULLB + (c & 1)], (c >> 1) & 1,
                                   abort_flag);
             };
@@ -483,8 +516,9 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint8_t* unit = p.wsT + ((size_t)(it.cbase + c) * p.sched.H + it.head) * kUnit;
             uint8_t* buf = smem + L::OFF_PB + (c & 1) * L::PB_STRIDE;
             mbar_expect_tx(&bars[B_PFULL + (c & 1)], 8192u + (GATED ? (uint32_t)kUnitFBytes : 0u));
+            static_assert(kKdaUnitFBytes == kUnitFBytes, "row factors of one size");
             bulk_load(buf, unit + 8192, 8192, &bars[B_PFULL + (c & 1)]);
-            if constexpr (GATED) bulk_load(buf + 8192, unit + kUnitF, kUnitFBytes, &bars[B_PFULL + (c & 1)]);
+            if constexpr (GATED) bulk_load(buf + 8192, unit + kUnitFac, kUnitFBytes, &bars[B_PFULL + (c & 1)]);
         };
         // O^T of chunk c -> out: read out of tensor memory (and zeroed for the next
         // chunk's first product, which accumulates into it), staged as token rows (the
@@ -627,6 +661,26 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
         auto pfac = [&](int c) {
             return reinterpret_cast<const float*>(smem + L::OFF_PB + (c & 1) * L::PB_STRIDE + 8192);
         };
+        // Gated DeltaNet: this thread's 64 values of S^T times lambda[1:C] (f[64]), in
+        // registers.  KDA: its columns (key channels 64 h .. 64 h + 63) of S^T in tensor memory
+        // times lambda[1:C] of their channel, 32 columns at a time (the caller has written them)
+        auto rescale_state = [&](uint32_t(&v)[64], const float* f) {
+            const float lam = f[kChunk];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
+        };
+        auto rescale_state_tm = [&](const float* f) {
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t w[32];
+                const uint32_t ta = tmem + lane_base + TM_S + 64 * h + 32 * hf;
+                tmem_ld32(ta, w);
+                const float* fh = f + 64 * h + 32 * hf;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(fh[c] * __uint_as_float(w[c]));
+                tmem_st32(ta, w);
+            }
+        };
         auto store_chunk_state = [&](int c, const uint32_t(&v)[64]) {
             const int64_t row = (int64_t)it.cbase + c;
             if (!p.cs || row >= p.cs_rows) return;
@@ -654,14 +708,14 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_st32(tmem + lane_base + TM_SBF + 32 * h, pk);
                 if constexpr (GATED) {
                     // Gated DeltaNet: the update of chunk 0 adds K->^T Z to lambda[1:C] S (the
-                    // chunk's factors arrive with its P tile)
+                    // chunk's factors arrive with its P tile); KDA: Diag(lambda[1:C]) S, this
+                    // thread's key channels 64 h .. 64 h + 63
                     live = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL], 0, abort_flag));
-                    const float lam = live ? pfac(0)[kChunk] : 1.f;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam * __uint_as_float(v[c]));
+                    if (!KDA && live) rescale_state(v, pfac(0));
                 }
                 tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
                 tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                if (KDA && live) rescale_state_tm(pfac(0));
             }
         }
         tc_fence_before();
@@ -682,7 +736,7 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_ld32(tmem + lane_base + TM_ZU + 32 * h, v);
                 pack_pairs<32>(v, pk);
                 tmem_st16(tmem + lane_base + TM_ZBF + 16 * h, pk);
-                if constexpr (GATED) {
+                if constexpr (GATED && !KDA) {
                     // Z^T diag(lambda[l+1:C]) for the state update (this half's 32 tokens)
                     const float4* f4 = reinterpret_cast<const float4*>(pfac(r) + 32 * h);
 #pragma unroll
@@ -731,11 +785,13 @@ static __global__ void __launch_bounds__(kThreadsTc, 1)
                     if (!__all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + ((r + 1) & 1)], ((r + 1) >> 1) & 1,
                                                            abort_flag)))
                         break;
-                    const float lam_next = pfac(r + 1)[kChunk];
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = __float_as_uint(lam_next * __uint_as_float(v[c]));
-                    tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                    if constexpr (KDA) {
+                        rescale_state_tm(pfac(r + 1));
+                    } else {
+                        rescale_state(v, pfac(r + 1));
+                        tmem_st32(tmem + lane_base + TM_S + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+                        tmem_st32(tmem + lane_base + TM_S + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                    }
                 }
             }
         }

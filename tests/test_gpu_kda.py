@@ -1,6 +1,7 @@
 """GPU parity of Kimi Delta Attention ("Linear Attention, Visualized", section
-"Kimi Delta Attention (KDA)"): kda_fwd through the C ABI against the float64
-oracle (a decay per key channel, S_t = (I - beta k^T k) Diag(a_t) S_{t-1} +
+"Kimi Delta Attention (KDA)"): kda_fwd through the C ABI, on the tensor-core path
+(d_k = d_v = 128, chains not split) and on the mma.sync chain kernels, against the
+float64 oracle (a decay per key channel, S_t = (I - beta k^T k) Diag(a_t) S_{t-1} +
 beta k^T v, o_t = q_t S_t) on the same seeded inputs.
 
 Bar: max|x - x_ref| / max|x_ref| <= 1e-2 (bf16 inputs) on out and final_state.
@@ -135,7 +136,46 @@ def test_kda_chained_calls_equal_one_call():
     assert torch.equal(s2, s_full)
 
 
+# One run per chain (seg_chunks past the chain length): d_k = d_v = 128 then runs on the
+# tensor-core path, its pre-pass and boundary kernel (two launches), instead of the
+# mma.sync chain kernel (one launch).
+ONE_RUN = 1 << 14
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 200, 333])
+def test_kda_tensor_core_path_shapes(T):
+    w = wl.custom(2, T, 3, 128, 128, torch.bfloat16, init_state=True, kda=True)
+    x = wl.generate(w, seed=80 + T)
+    check(w, x, seg_chunks=ONE_RUN)
+    assert dn.last_launches() == 2
+
+
+def test_kda_tensor_core_path_strong_decays_no_initial_state():
+    """Log decays down to -2 per channel and token, no initial state: the channel-decayed
+    Gram blocks, K<-, K-> and the per-channel state decay of the tensor-core path."""
+    w = wl.custom(2, 300, 2, 128, 128, torch.bfloat16, init_state=False, kda=True)
+    x = wl.generate(w, seed=90)
+    gen = torch.Generator().manual_seed(91)
+    x["g"] = -2.0 * torch.rand(x["g"].shape, generator=gen)
+    check(w, x, seg_chunks=ONE_RUN)
+    assert dn.last_launches() == 2
+
+
+def test_kda_tensor_core_path_equals_gdn_on_equal_channel_gates():
+    """Equal gates on every channel: the KDA tensor-core path and Gated DeltaNet's agree
+    within the bar."""
+    w = wl.custom(2, 200, 2, 128, 128, torch.bfloat16, init_state=True, gated=True)
+    x = wl.generate(w, seed=92)
+    g = to_dev(x)
+    o_gdn, s_gdn = dn.gated_deltanet_fwd(g["q"], g["k"], g["v"], g["beta"], g["g"], g["initial_state"])
+    gk = g["g"].unsqueeze(-1).expand(-1, -1, -1, 128).contiguous()
+    o_kda, s_kda = dn.kda_fwd(g["q"], g["k"], g["v"], g["beta"], gk, g["initial_state"], seg_chunks=ONE_RUN)
+    assert dn.get_error() == 0
+    assert rel_err(o_kda, o_gdn) <= TOL and rel_err(s_kda, s_gdn) <= TOL
+
+
 @pytest.mark.slow
 def test_config_kda_1p3b(margins):
     w = wl.WORKLOADS["kda_1p3b"]
     check(w, wl.generate(w, 0), heads=(0, 2), log=margins, name="kda_1p3b (heads 0-1)")
+    assert dn.last_launches() == 2  # unsplit chains: the tensor-core pre-pass and boundary kernel
