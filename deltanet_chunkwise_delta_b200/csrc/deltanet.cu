@@ -819,6 +819,9 @@ int dn_trace_copy_prep(unsigned long long* host) {
 int dn_trace_copy_sum(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, tcs::g_dn_trace_sum, sizeof(tcs::g_dn_trace_sum)) == cudaSuccess ? 0 : 1;
 }
+int dn_trace_copy_kda(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_dn_trace_kda, sizeof(g_dn_trace_kda)) == cudaSuccess ? 0 : 1;
+}
 int dn_trace_copy_scan(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_dn_trace_scan, sizeof(g_dn_trace_scan)) == cudaSuccess ? 0 : 1;
 }

@@ -28,6 +28,22 @@
 
 namespace dn {
 
+#ifdef DN_TRACE
+static __device__ unsigned long long g_dn_trace_kda[16 * 8];
+#define DN_TRK(k, slot)                                                               \
+    do {                                                                              \
+        if (blockIdx.x == 0 && (k) < 16 && threadIdx.x == 0) {                         \
+            unsigned long long t_;                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                    \
+            g_dn_trace_kda[(k) * 8 + (slot)] = t_;                                    \
+        }                                                                             \
+    } while (0)
+#else
+#define DN_TRK(k, slot) \
+    do {                \
+    } while (0)
+#endif
+
 constexpr int kKdaUnitT = 0, kKdaUnitP = 8192, kKdaUnitQL = 16384, kKdaUnitKL = 32768, kKdaUnitKR = 49152,
               kKdaUnitF = 65536, kKdaUnitFBytes = 512;
 constexpr int kKdaUnitBytes = 66560;
@@ -67,6 +83,21 @@ __device__ __forceinline__ void tile_to_boxes(uint8_t* dst, const __nv_bfloat16*
     }
 }
 
+// bf16 pair (lo, hi) times (fa, fb), rounded to nearest-even.
+__device__ __forceinline__ uint32_t kda_scale2(uint32_t w, float fa, float fb) {
+    return sm100::pack_bf16(__uint_as_float(w << 16) * fa, __uint_as_float(w & 0xffff0000u) * fb);
+}
+__device__ __forceinline__ uint4 kda_scale8(uint4 v, const float (&f)[8]) {
+    return make_uint4(kda_scale2(v.x, f[0], f[1]), kda_scale2(v.y, f[2], f[3]), kda_scale2(v.z, f[4], f[5]),
+                      kda_scale2(v.w, f[6], f[7]));
+}
+// the 8 running sums of row r, channels 8 c8 .. 8 c8 + 7
+__device__ __forceinline__ void kda_row8(const float* G, int r, int c8, float (&g)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(G + r * KdaPrepLay::DK + 8 * c8);
+    const float4 b = *reinterpret_cast<const float4*>(G + r * KdaPrepLay::DK + 8 * c8 + 4);
+    g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w; g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
+}
+
 template <int DK>
 static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
     static_assert(DK == KdaPrepLay::DK, "the tensor-core path has d_k = 128");
@@ -92,9 +123,20 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
     const int g8 = lane >> 2, t4 = lane & 3;
     const int H = p.sched.H;
     const int units = count_chunks(p.sched) * H;
+    // the scaled-operand passes work on 16-byte pieces of 8 channels: thread tid always
+    // takes piece c8 of rows tid / 16, tid / 16 + 16, ... (a Swz tile row r keeps piece c8
+    // at byte r * 256 + ((c8 ^ (r % 8)) * 16))
+    const int c8 = tid & 15, r16 = tid >> 4;
+    auto piece = [](int r, int c) { return r * 256 + ((c ^ (r & 7)) << 4); };
+    uint8_t* Kb = reinterpret_cast<uint8_t*>(Kc);
+    uint8_t* Qb = reinterpret_cast<uint8_t*>(Qc);
+    uint8_t* Rb = reinterpret_cast<uint8_t*>(Rs);
+    uint8_t* LQb = reinterpret_cast<uint8_t*>(LQs);
 
+    int it_ = 0;
 #pragma unroll 1
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it_) {
+        DN_TRK(it_, 0);
         const int head = u % H;
         int b, t0, t1;
         chunk_range(p.sched, u / H, b, t0, t1);
@@ -121,6 +163,7 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
+        DN_TRK(it_, 1);
 
         // running sums per key channel, in place, and lambda[1:C]
         if (tid < DK) {
@@ -132,23 +175,35 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             lamc[tid] = expf(acc);
         }
         __syncthreads();
+        DN_TRK(it_, 2);
 
         // rows 16 b .. 16 b + 15 of A = B L (fp32, strict lower) and of P (inclusive),
         // against reference row s = 16 b
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
             const int s = 16 * blk, ncol = s + 16;
-            for (int idx = tid; idx < ncol * DK; idx += kThreads) {
-                const int m = idx / DK, c = idx % DK;
-                const int o = SW::template off<DK>(m, c);
-                Rs[o] = __float2bfloat16_rn(__bfloat162float(Kc[o]) * expf(G[s * DK + c] - G[m * DK + c]));
+            float gs[8];
+            kda_row8(G, s, c8, gs);
+            // right operand rows m < ncol: k_m o exp(G_s - G_m)
+            for (int m = r16; m < ncol; m += kThreads / 16) {
+                float gm[8], f[8];
+                kda_row8(G, m, c8, gm);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __expf(gs[e] - gm[e]);
+                *reinterpret_cast<uint4*>(Rb + piece(m, c8)) =
+                    kda_scale8(*reinterpret_cast<const uint4*>(Kb + piece(m, c8)), f);
             }
-            for (int idx = tid; idx < 16 * DK; idx += kThreads) {
-                const int lr = idx / DK, c = idx % DK, l = s + lr;
-                const float f = expf(G[l * DK + c] - G[s * DK + c]);
-                const int o = SW::template off<DK>(l, c), ol = SW::template off<DK>(lr, c);
-                LQs[ol] = __float2bfloat16_rn(__bfloat162float(Kc[o]) * f);
-                LQs[16 * DK + ol] = __float2bfloat16_rn(__bfloat162float(Qc[o]) * f);
+            // left operands, rows l = s + r16 of the block: k_l and q_l o exp(G_l - G_s)
+            {
+                const int l = s + r16;
+                float gl[8], f[8];
+                kda_row8(G, l, c8, gl);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __expf(gl[e] - gs[e]);
+                *reinterpret_cast<uint4*>(LQb + piece(r16, c8)) =
+                    kda_scale8(*reinterpret_cast<const uint4*>(Kb + piece(l, c8)), f);
+                *reinterpret_cast<uint4*>(LQb + piece(16 + r16, c8)) =
+                    kda_scale8(*reinterpret_cast<const uint4*>(Qb + piece(l, c8)), f);
             }
             // the block's rows right of its last column are zero in both
             for (int idx = tid; idx < 16 * (kChunk - ncol); idx += kThreads) {
@@ -177,15 +232,25 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             __syncthreads();
         }
 
+        DN_TRK(it_, 3);
         // K<- = exp(G) o K, K-> = exp(G_C - G) o K, Q<- = exp(G) o Q, then out to the unit
-        for (int idx = tid; idx < kChunk * DK; idx += kThreads) {
-            const int l = idx / DK, c = idx % DK;
-            const int o = SW::template off<DK>(l, c);
-            const float gl = G[l * DK + c], gC = G[(kChunk - 1) * DK + c];
-            const float kv = __bfloat162float(Kc[o]);
-            Rs[o] = __float2bfloat16_rn(kv * expf(gl));
-            Kc[o] = __float2bfloat16_rn(kv * expf(gC - gl));
-            Qc[o] = __float2bfloat16_rn(__bfloat162float(Qc[o]) * expf(gl));
+        {
+            float gC[8];
+            kda_row8(G, kChunk - 1, c8, gC);
+            for (int l = r16; l < kChunk; l += kThreads / 16) {
+                float gl[8], fl[8], fr[8];
+                kda_row8(G, l, c8, gl);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    fl[e] = __expf(gl[e]);
+                    fr[e] = __expf(gC[e] - gl[e]);
+                }
+                const int o = piece(l, c8);
+                const uint4 kv = *reinterpret_cast<const uint4*>(Kb + o);
+                *reinterpret_cast<uint4*>(Rb + o) = kda_scale8(kv, fl);
+                *reinterpret_cast<uint4*>(Kb + o) = kda_scale8(kv, fr);
+                *reinterpret_cast<uint4*>(Qb + o) = kda_scale8(*reinterpret_cast<const uint4*>(Qb + o), fl);
+            }
         }
         __syncthreads();
         tile_to_boxes<DK>(unit + kKdaUnitQL, Qc);
@@ -194,10 +259,12 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
         if (tid < DK / 4)
             reinterpret_cast<float4*>(unit + kKdaUnitF)[tid] = reinterpret_cast<const float4*>(lamc)[tid];
         __syncthreads();  // the region is taken by the solve's tiles next
+        DN_TRK(it_, 4);
 
         // T = (I + B L)^{-1} B
         ut_solve<E>(Af, Nf, Xt, bc, Ts);
         __syncthreads();
+        DN_TRK(it_, 5);
         for (int idx = tid; idx < 2 * 512; idx += kThreads) {
             const int t = idx >> 9, pc = idx & 511;
             const uint8_t* src = reinterpret_cast<const uint8_t*>(t == 0 ? Ts : Ps);
@@ -205,6 +272,7 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
                 *reinterpret_cast<const uint4*>(src + pc * 16);
         }
         __syncthreads();  // the next unit's loads overwrite the tiles
+        DN_TRK(it_, 6);
     }
 }
 
