@@ -339,11 +339,14 @@ def run_b200(args, w: wl.Workload):
     alg_bytes = algorithmic_bytes(w)
     # DeltaNet, Gated DeltaNet and the Gated Delta Product at d_k = d_v = 128 run on the
     # tensor-core kernels
-    tc_path = (not w.kda and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
-               and (w.nh == 1 or w.gated))
+    # (Kimi Delta Attention: on a dense batch whose chains are not split)
+    tc_path = (w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+               and (w.nh == 1 or w.gated)
+               and (not w.kda or (w.seqlens is None and G == 1)))
     # the tensor-core boundary kernel moves q, k, v, o and the states (beta and the log
-    # decays are read by the UT pre-pass); the mma.sync boundary kernel reads them itself
-    kernel_bytes = alg_bytes - ((4.0 * w.nh + (4.0 if w.gated else 0.0)) * w.tokens * w.H if tc_path else 0.0)
+    # decays are read by the pre-pass); the mma.sync boundary kernel reads them itself
+    gate_bytes = 4.0 * w.dk if w.kda else (4.0 if w.gated else 0.0)
+    kernel_bytes = alg_bytes - ((4.0 * w.nh + gate_bytes) * w.tokens * w.H if tc_path else 0.0)
     if tc_path and w.seqlens is None and G >= 2:
         # split dense chains: run 0 of every chain is computed by its own launch next to
         # the summary pass; the timed launch covers runs 1..G-1 (q, k, v, o of their
