@@ -131,11 +131,65 @@ __device__ __forceinline__ float to_e<float>(float x) {
     return x;
 }
 
+// 16 x 16 fp32 blocks of row stride LD as tf32 warp products (one warp):
+// acc (16 x 16, two n8 tiles in the m16n8 accumulator layout) += A * B.
+template <int LD>
+__device__ __forceinline__ void blk16_tf32(float (&acc)[2][4], const float* A, const float* B) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = sm100::to_tf32(A[g * LD + 8 * ks + t]);
+        const uint32_t a1 = sm100::to_tf32(A[(g + 8) * LD + 8 * ks + t]);
+        const uint32_t a2 = sm100::to_tf32(A[g * LD + 8 * ks + t + 4]);
+        const uint32_t a3 = sm100::to_tf32(A[(g + 8) * LD + 8 * ks + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = sm100::to_tf32(B[(8 * ks + t) * LD + 8 * nt + g]);
+            const uint32_t b1 = sm100::to_tf32(B[(8 * ks + t + 4) * LD + 8 * nt + g]);
+            sm100::mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
+        }
+    }
+}
+template <int LD>
+__device__ __forceinline__ void blk16_store(float* C, const float (&acc)[2][4], float scale) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        C[g * LD + 8 * nt + 2 * t] = scale * acc[nt][0];
+        C[g * LD + 8 * nt + 2 * t + 1] = scale * acc[nt][1];
+        C[(g + 8) * LD + 8 * nt + 2 * t] = scale * acc[nt][2];
+        C[(g + 8) * LD + 8 * nt + 2 * t + 1] = scale * acc[nt][3];
+    }
+}
+template <int LD>
+__device__ __forceinline__ void blk16_load(float (&acc)[2][4], const float* C) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        acc[nt][0] = C[g * LD + 8 * nt + 2 * t];
+        acc[nt][1] = C[g * LD + 8 * nt + 2 * t + 1];
+        acc[nt][2] = C[(g + 8) * LD + 8 * nt + 2 * t];
+        acc[nt][3] = C[(g + 8) * LD + 8 * nt + 2 * t + 1];
+    }
+}
+// N_ij = -N_ii Y for a finished sum Y held in acc, through the staging block X (one warp).
+template <int LD>
+__device__ __forceinline__ void blk16_finish(float* Nij, const float* Nii, float* X, const float (&acc)[2][4]) {
+    blk16_store<LD>(X, acc, 1.f);
+    __syncwarp();
+    float out[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    blk16_tf32<LD>(out, Nii, X);
+    blk16_store<LD>(Nij, out, -1.f);
+}
+
 // Blocked solve of (I + A) N = I for the strictly lower A (= B L, 64 x 64, fp32,
 // row stride 65), followed by T = N diag(beta) written to a swizzled tile, and,
 // when colscale is given, T diag(colscale) to a second tile T2.
 // Diagonal 16 x 16 blocks by forward substitution, one column per thread;
 // off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order of i - j.
+// For bf16 operands (whose T is rounded to bf16 anyway) the off-diagonal block products
+// take tf32 inputs on the tensor cores, one warp per block, staged in N's strictly upper
+// blocks (never read); fp32 runs them as fp32 FMAs.
 template <typename E, int NT = kThreads>
 __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
                                          const float* beta, E* Ts,
@@ -167,6 +221,49 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
         }
     }
     __syncthreads();
+    if constexpr (std::is_same<E, __nv_bfloat16>::value) {
+        const int warp = tid >> 5;
+        auto A_ = [&](int i, int j) { return Af + (16 * i) * LD + 16 * j; };
+        auto N_ = [&](int i, int j) { return Nf + (16 * i) * LD + 16 * j; };
+        auto U_ = [&](int u) {  // staging: the strictly upper blocks (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+            const int bi = u < 3 ? 0 : (u < 5 ? 1 : 2), bj = u < 3 ? u + 1 : (u < 5 ? u - 1 : 3);
+            return Nf + (16 * bi) * LD + 16 * bj;
+        };
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float y30[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // N_{i+1,i} (warps 0-2); warp 3: the partial sums A20 N00 and A31 N11
+        if (warp < 3) {
+            blk16_tf32<LD>(acc, A_(warp + 1, warp), N_(warp, warp));
+            blk16_finish<LD>(N_(warp + 1, warp), N_(warp + 1, warp + 1), U_(warp), acc);
+        } else if (warp == 3) {
+            blk16_tf32<LD>(acc, A_(2, 0), N_(0, 0));
+            blk16_store<LD>(U_(3), acc, 1.f);
+            float a2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            blk16_tf32<LD>(a2, A_(3, 1), N_(1, 1));
+            blk16_store<LD>(U_(4), a2, 1.f);
+        }
+        __syncthreads();
+        // N20 (warp 0), N31 (warp 1); warp 2: A30 N00 + A31 N10
+        if (warp == 0) {
+            blk16_load<LD>(acc, U_(3));
+            blk16_tf32<LD>(acc, A_(2, 1), N_(1, 0));
+            blk16_finish<LD>(N_(2, 0), N_(2, 2), U_(0), acc);
+        } else if (warp == 1) {
+            blk16_load<LD>(acc, U_(4));
+            blk16_tf32<LD>(acc, A_(3, 2), N_(2, 1));
+            blk16_finish<LD>(N_(3, 1), N_(3, 3), U_(1), acc);
+        } else if (warp == 2) {
+            blk16_tf32<LD>(y30, A_(3, 0), N_(0, 0));
+            blk16_tf32<LD>(y30, A_(3, 1), N_(1, 0));
+        }
+        __syncthreads();
+        // N30 (warp 2)
+        if (warp == 2) {
+            blk16_tf32<LD>(y30, A_(3, 2), N_(2, 0));
+            blk16_finish<LD>(N_(3, 0), N_(3, 3), U_(2), y30);
+        }
+        __syncthreads();
+    } else {
 #pragma unroll 1
     for (int d = 1; d < 4; ++d) {
         const int npairs = 4 - d;
@@ -190,6 +287,7 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
             Nf[(16 * i + ri) * LD + 16 * j + cj] = -acc;
         }
         __syncthreads();
+    }
     }
     for (int e = tid; e < kChunk * kChunk; e += NT) {
         const int i = e >> 6, j = e & 63;

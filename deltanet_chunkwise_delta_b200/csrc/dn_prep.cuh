@@ -109,20 +109,7 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t w, float f) {
 
 // acc (16 x 16, two n8 tiles) += A (16 x 16) * B (16 x 16), tf32 inputs, fp32 accumulate.
 __device__ __forceinline__ void mm16_tf32(float (&acc)[2][4], const float* A, const float* B) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t a0 = sm100::to_tf32(A[g * kBlkLd + 8 * ks + t]);
-        const uint32_t a1 = sm100::to_tf32(A[(g + 8) * kBlkLd + 8 * ks + t]);
-        const uint32_t a2 = sm100::to_tf32(A[g * kBlkLd + 8 * ks + t + 4]);
-        const uint32_t a3 = sm100::to_tf32(A[(g + 8) * kBlkLd + 8 * ks + t + 4]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t b0 = sm100::to_tf32(B[(8 * ks + t) * kBlkLd + 8 * nt + g]);
-            const uint32_t b1 = sm100::to_tf32(B[(8 * ks + t + 4) * kBlkLd + 8 * nt + g]);
-            sm100::mma_tf32(acc[nt], a0, a1, a2, a3, b0, b1);
-        }
-    }
+    blk16_tf32<kBlkLd>(acc, A, B);
 }
 
 __device__ __forceinline__ void st_blk(float* C, const float (&acc)[2][4], float scale) {
