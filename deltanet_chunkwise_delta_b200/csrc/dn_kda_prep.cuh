@@ -49,39 +49,29 @@ constexpr int kKdaUnitT = 0, kKdaUnitP = 8192, kKdaUnitQL = 16384, kKdaUnitKL = 
 constexpr int kKdaUnitBytes = 66560;
 
 // Shared memory of the KDA pre-pass (byte offsets).  [0, OFF_AF) holds the chunk's k, q,
-// log decays and the block operands until the scaled tiles are written out; the solve's
-// N, X and T tiles then reuse it.
+// log decays and the block operands until the scaled tiles are written out.  The solve
+// then keeps N where the right operand was and writes T over A, so that the next unit's
+// k, q, log decays and beta load into [0, OFF_R) and OFF_BNEXT while it runs.
 struct KdaPrepLay {
     static constexpr int DK = 128;
-    static constexpr int OFF_K = 0;          // 64 x 128 bf16 (Swz): K, later K->
-    static constexpr int OFF_Q = 16384;      // 64 x 128 bf16 (Swz): Q, later Q<-
+    static constexpr int OFF_K = 0;          // 64 x 128 bf16 (Swz): K
+    static constexpr int OFF_Q = 16384;      // 64 x 128 bf16 (Swz): Q
     static constexpr int OFF_G = 32768;      // 64 x 128 fp32: log decays, later running sums
-    static constexpr int OFF_R = 65536;      // 64 x 128 bf16 (Swz): a block's right operand, later K<-
+    static constexpr int OFF_R = 65536;      // 64 x 128 bf16 (Swz): a block's right operand
     static constexpr int OFF_LQ = 81920;     // 32 x 128 bf16 (Swz): a block's left operands [K; Q]
-    static constexpr int OFF_N = 0;          // after the tiles: N, 64 x 65 fp32
-    static constexpr int OFF_X = 16640;      //   the solve's staging, 3 x 256 fp32
-    static constexpr int OFF_T = 19712;      //   T, 64 x 64 bf16 (Swz)
-    static constexpr int OFF_AF = 90112;     // A = B L, 64 x 65 fp32
+    static constexpr int OFF_N = 65536;      // after the tiles: N, 64 x 65 fp32
+    static constexpr int OFF_X = 82176;      //   the fp32 solve's staging (the bf16 solve stages in N)
+    static constexpr int OFF_BNEXT = 89856;  //   the next unit's beta, 64 fp32
+    static constexpr int OFF_AF = 90112;     // A = B L, 64 x 65 fp32; T (64 x 64 bf16, Swz) once the solve has read A
+    static constexpr int OFF_T = OFF_AF;
     static constexpr int OFF_P = 106752;     // P, 64 x 64 bf16 (Swz)
     static constexpr int OFF_BETA = 114944;  // 64 fp32
     static constexpr int OFF_LAMC = 115200;  // lambda[1:C], 128 fp32
     static constexpr int TOTAL = 115712;     // two CTAs per SM
 };
-static_assert(KdaPrepLay::OFF_T + 8192 <= KdaPrepLay::OFF_AF, "solve tiles fit the freed region");
-
-// One 64-row bf16 tile of width W (Swz layout) -> global, as W / 64 boxes of 64 channels
-// x 64 rows with 128-byte rows: row r's bytes [128 a, 128 a + 128) are row r of box a
-// (the 16-byte pieces keep their order: both layouts swizzle them by row % 8 within 128
-// bytes).  All threads.
-template <int W>
-__device__ __forceinline__ void tile_to_boxes(uint8_t* dst, const __nv_bfloat16* src) {
-    constexpr int PR = W / 8;  // 16-byte pieces per row
-    for (int idx = threadIdx.x; idx < kChunk * PR; idx += kThreads) {
-        const int r = idx / PR, pc = idx % PR;
-        const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(src) + r * (W * 2) + pc * 16);
-        *reinterpret_cast<uint4*>(dst + (pc >> 3) * 8192 + r * 128 + (pc & 7) * 16) = v;
-    }
-}
+static_assert(KdaPrepLay::OFF_N + 64 * 65 * 4 <= KdaPrepLay::OFF_X && KdaPrepLay::OFF_X + 3 * 256 * 4 <= KdaPrepLay::OFF_BNEXT &&
+                  KdaPrepLay::OFF_BNEXT + 64 * 4 <= KdaPrepLay::OFF_AF && KdaPrepLay::OFF_R == KdaPrepLay::OFF_N,
+              "the solve's tiles stay clear of the next unit's loads");
 
 // bf16 pair (lo, hi) times (fa, fb), rounded to nearest-even.
 __device__ __forceinline__ uint32_t kda_scale2(uint32_t w, float fa, float fb) {
@@ -118,6 +108,7 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
     E* Ps = reinterpret_cast<E*>(kda_smem + L::OFF_P);
     float* bc = reinterpret_cast<float*>(kda_smem + L::OFF_BETA);
     float* lamc = reinterpret_cast<float*>(kda_smem + L::OFF_LAMC);
+    float* bnext = reinterpret_cast<float*>(kda_smem + L::OFF_BNEXT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
@@ -133,17 +124,13 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
     uint8_t* Rb = reinterpret_cast<uint8_t*>(Rs);
     uint8_t* LQb = reinterpret_cast<uint8_t*>(LQs);
 
-    int it_ = 0;
-#pragma unroll 1
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it_) {
-        DN_TRK(it_, 0);
-        const int head = u % H;
+    // unit uu's k, q, beta and log decays (rows past the chunk: zeros, identity steps), as
+    // one group of asynchronous copies
+    auto issue_loads = [&](int uu) {
+        const int head = uu % H;
         int b, t0, t1;
-        chunk_range(p.sched, u / H, b, t0, t1);
+        chunk_range(p.sched, uu / H, b, t0, t1);
         const int rows = t1 - t0;
-        uint8_t* unit = p.wsT + (size_t)u * kKdaUnitBytes;
-
-        // the chunk's k, q, beta and log decays (rows past the chunk: zeros, identity steps)
         const E* kg = static_cast<const E*>(p.k) + b * p.k_sb + head * p.k_sh;
         const E* qg = static_cast<const E*>(p.q) + b * p.q_sb + head * p.q_sh;
         const float* bg = p.beta + b * p.b_sb + head * p.b_sh;
@@ -152,7 +139,7 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
         load_tile<E, DK>(Qc, qg + (int64_t)t0 * p.q_st, p.q_st, rows);
         if (tid < kChunk) {
             const bool ok = tid < rows;
-            cp_async4(smem_addr(bc + tid), ok ? bg + (int64_t)(t0 + tid) * p.b_st : bg, ok ? 4 : 0);
+            cp_async4(smem_addr(bnext + tid), ok ? bg + (int64_t)(t0 + tid) * p.b_st : bg, ok ? 4 : 0);
         }
         for (int idx = tid; idx < kChunk * (DK / 4); idx += kThreads) {
             const int rr = idx / (DK / 4), c = idx % (DK / 4);
@@ -161,9 +148,18 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             cp_async16(smem_addr(G + rr * DK + 4 * c), src, ok ? 16 : 0);
         }
         cp_async_commit();
+    };
+
+    if (blockIdx.x < units) issue_loads(blockIdx.x);
+    int it_ = 0;
+#pragma unroll 1
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it_) {
+        DN_TRK(it_, 0);
+        uint8_t* unit = p.wsT + (size_t)u * kKdaUnitBytes;
         cp_async_wait<0>();
         __syncthreads();
         DN_TRK(it_, 1);
+        if (tid < kChunk) bc[tid] = bnext[tid];  // before the block operands take OFF_BNEXT
 
         // running sums per key channel, in place, and lambda[1:C]
         if (tid < DK) {
@@ -179,12 +175,13 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
 
         // rows 16 b .. 16 b + 15 of A = B L (fp32, strict lower) and of P (inclusive),
         // against reference row s = 16 b
-#pragma unroll 1
+#pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             const int s = 16 * blk, ncol = s + 16;
             float gs[8];
             kda_row8(G, s, c8, gs);
             // right operand rows m < ncol: k_m o exp(G_s - G_m)
+#pragma unroll
             for (int m = r16; m < ncol; m += kThreads / 16) {
                 float gm[8], f[8];
                 kda_row8(G, m, c8, gm);
@@ -233,10 +230,13 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
         }
 
         DN_TRK(it_, 3);
-        // K<- = exp(G) o K, K-> = exp(G_C - G) o K, Q<- = exp(G) o Q, then out to the unit
+        // K<- = exp(G) o K, K-> = exp(G_C - G) o K, Q<- = exp(G) o Q, stored straight to the
+        // unit's boxes: logical piece c8 of row l sits in box c8 / 8 at row l, piece
+        // (c8 % 8) ^ (l % 8) (a warp writes whole 128-byte box rows)
         {
             float gC[8];
             kda_row8(G, kChunk - 1, c8, gC);
+#pragma unroll
             for (int l = r16; l < kChunk; l += kThreads / 16) {
                 float gl[8], fl[8], fr[8];
                 kda_row8(G, l, c8, gl);
@@ -246,20 +246,19 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
                     fr[e] = __expf(gC[e] - gl[e]);
                 }
                 const int o = piece(l, c8);
+                const int go = (c8 >> 3) * 8192 + l * 128 + (((c8 & 7) ^ (l & 7)) << 4);
                 const uint4 kv = *reinterpret_cast<const uint4*>(Kb + o);
-                *reinterpret_cast<uint4*>(Rb + o) = kda_scale8(kv, fl);
-                *reinterpret_cast<uint4*>(Kb + o) = kda_scale8(kv, fr);
-                *reinterpret_cast<uint4*>(Qb + o) = kda_scale8(*reinterpret_cast<const uint4*>(Qb + o), fl);
+                *reinterpret_cast<uint4*>(unit + kKdaUnitKL + go) = kda_scale8(kv, fl);
+                *reinterpret_cast<uint4*>(unit + kKdaUnitKR + go) = kda_scale8(kv, fr);
+                *reinterpret_cast<uint4*>(unit + kKdaUnitQL + go) =
+                    kda_scale8(*reinterpret_cast<const uint4*>(Qb + o), fl);
             }
         }
-        __syncthreads();
-        tile_to_boxes<DK>(unit + kKdaUnitQL, Qc);
-        tile_to_boxes<DK>(unit + kKdaUnitKL, Rs);
-        tile_to_boxes<DK>(unit + kKdaUnitKR, Kc);
         if (tid < DK / 4)
             reinterpret_cast<float4*>(unit + kKdaUnitF)[tid] = reinterpret_cast<const float4*>(lamc)[tid];
-        __syncthreads();  // the region is taken by the solve's tiles next
+        __syncthreads();  // k, q, the log decays and the right operand are read
         DN_TRK(it_, 4);
+        if (u + (int)gridDim.x < units) issue_loads(u + gridDim.x);
 
         // T = (I + B L)^{-1} B
         ut_solve<E>(Af, Nf, Xt, bc, Ts);
@@ -271,7 +270,7 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             *reinterpret_cast<uint4*>(unit + (t == 0 ? kKdaUnitT : kKdaUnitP) + pc * 16) =
                 *reinterpret_cast<const uint4*>(src + pc * 16);
         }
-        __syncthreads();  // the next unit's loads overwrite the tiles
+        __syncthreads();  // the next unit's block operands overwrite the tiles
         DN_TRK(it_, 6);
     }
 }
