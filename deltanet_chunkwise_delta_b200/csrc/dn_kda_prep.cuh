@@ -173,6 +173,16 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
         __syncthreads();
         DN_TRK(it_, 2);
 
+        // the thread's rows r16 + 16 i (i = 0..3), piece c8: running sums and k, held in
+        // registers through the Gram blocks and the decayed tiles
+        float gr[4][8];
+        uint4 kr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            kda_row8(G, r16 + 16 * i, c8, gr[i]);
+            kr[i] = *reinterpret_cast<const uint4*>(Kb + piece(r16 + 16 * i, c8));
+        }
+
         // rows 16 b .. 16 b + 15 of A = B L (fp32, strict lower) and of P (inclusive),
         // against reference row s = 16 b
 #pragma unroll
@@ -180,25 +190,21 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             const int s = 16 * blk, ncol = s + 16;
             float gs[8];
             kda_row8(G, s, c8, gs);
-            // right operand rows m < ncol: k_m o exp(G_s - G_m)
+            // right operand rows m = r16 + 16 i < ncol: k_m o exp(G_s - G_m)
 #pragma unroll
-            for (int m = r16; m < ncol; m += kThreads / 16) {
-                float gm[8], f[8];
-                kda_row8(G, m, c8, gm);
+            for (int i = 0; i <= blk; ++i) {
+                float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = __expf(gs[e] - gm[e]);
-                *reinterpret_cast<uint4*>(Rb + piece(m, c8)) =
-                    kda_scale8(*reinterpret_cast<const uint4*>(Kb + piece(m, c8)), f);
+                for (int e = 0; e < 8; ++e) f[e] = __expf(gs[e] - gr[i][e]);
+                *reinterpret_cast<uint4*>(Rb + piece(r16 + 16 * i, c8)) = kda_scale8(kr[i], f);
             }
             // left operands, rows l = s + r16 of the block: k_l and q_l o exp(G_l - G_s)
             {
                 const int l = s + r16;
-                float gl[8], f[8];
-                kda_row8(G, l, c8, gl);
+                float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = __expf(gl[e] - gs[e]);
-                *reinterpret_cast<uint4*>(LQb + piece(r16, c8)) =
-                    kda_scale8(*reinterpret_cast<const uint4*>(Kb + piece(l, c8)), f);
+                for (int e = 0; e < 8; ++e) f[e] = __expf(gr[blk][e] - gs[e]);
+                *reinterpret_cast<uint4*>(LQb + piece(r16, c8)) = kda_scale8(kr[blk], f);
                 *reinterpret_cast<uint4*>(LQb + piece(16 + r16, c8)) =
                     kda_scale8(*reinterpret_cast<const uint4*>(Qb + piece(l, c8)), f);
             }
@@ -237,21 +243,19 @@ static __global__ void __launch_bounds__(kThreads, 2) k_kda_prep(Params p) {
             float gC[8];
             kda_row8(G, kChunk - 1, c8, gC);
 #pragma unroll
-            for (int l = r16; l < kChunk; l += kThreads / 16) {
-                float gl[8], fl[8], fr[8];
-                kda_row8(G, l, c8, gl);
+            for (int i = 0; i < 4; ++i) {
+                const int l = r16 + 16 * i;
+                float fl[8], fr[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    fl[e] = __expf(gl[e]);
-                    fr[e] = __expf(gC[e] - gl[e]);
+                    fl[e] = __expf(gr[i][e]);
+                    fr[e] = __expf(gC[e] - gr[i][e]);
                 }
-                const int o = piece(l, c8);
                 const int go = (c8 >> 3) * 8192 + l * 128 + (((c8 & 7) ^ (l & 7)) << 4);
-                const uint4 kv = *reinterpret_cast<const uint4*>(Kb + o);
-                *reinterpret_cast<uint4*>(unit + kKdaUnitKL + go) = kda_scale8(kv, fl);
-                *reinterpret_cast<uint4*>(unit + kKdaUnitKR + go) = kda_scale8(kv, fr);
+                *reinterpret_cast<uint4*>(unit + kKdaUnitKL + go) = kda_scale8(kr[i], fl);
+                *reinterpret_cast<uint4*>(unit + kKdaUnitKR + go) = kda_scale8(kr[i], fr);
                 *reinterpret_cast<uint4*>(unit + kKdaUnitQL + go) =
-                    kda_scale8(*reinterpret_cast<const uint4*>(Qb + o), fl);
+                    kda_scale8(*reinterpret_cast<const uint4*>(Qb + piece(l, c8)), fl);
             }
         }
         if (tid < DK / 4)
