@@ -309,6 +309,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                 sm100::bulk_wait_read0();
             }
             __syncthreads();
+            DN_TRP(it_, 6);
         }
         const float* betas = reinterpret_cast<const float*>(smem + L::OFF_BETA) + bb * kChunk;
         const float* cs = reinterpret_cast<const float*>(smem + L::OFF_C);  // gated: running sums
@@ -377,6 +378,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                         *reinterpret_cast<uint4*>(ps + sm100::swz128(i, col)) = w;
                     }
                 }
+                DN_TRP(it_, 7);
                 sm100::fence_async_smem();
             }
         }
