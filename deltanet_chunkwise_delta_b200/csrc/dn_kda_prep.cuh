@@ -81,10 +81,15 @@ __device__ __forceinline__ uint4 kda_scale8(uint4 v, const float (&f)[8]) {
     return make_uint4(kda_scale2(v.x, f[0], f[1]), kda_scale2(v.y, f[2], f[3]), kda_scale2(v.z, f[4], f[5]),
                       kda_scale2(v.w, f[6], f[7]));
 }
-// the 8 running sums of row r, channels 8 c8 .. 8 c8 + 7
+// the 8 running sums of row r, channels 8 c8 .. 8 c8 + 7.  Pieces c8 with bit 2 set read their
+// second half first: a quarter warp's 16-byte reads (pieces 32 bytes apart) then fall in eight
+// distinct groups of four banks.
 __device__ __forceinline__ void kda_row8(const float* G, int r, int c8, float (&g)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(G + r * KdaPrepLay::DK + 8 * c8);
-    const float4 b = *reinterpret_cast<const float4*>(G + r * KdaPrepLay::DK + 8 * c8 + 4);
+    const int sw = (c8 >> 2) & 1;
+    const float4* src = reinterpret_cast<const float4*>(G + r * KdaPrepLay::DK + 8 * c8);
+    const float4 x = src[sw];
+    const float4 y = src[sw ^ 1];
+    const float4 a = sw ? y : x, b = sw ? x : y;
     g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w; g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
 }
 
