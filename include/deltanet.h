@@ -129,8 +129,10 @@ dn_status deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn_tenso
  *   other arguments, layouts, ownership, aliasing (g is an input) and errors
  *   as deltanet_fwd; g == NULL returns DN_ERR_INVALID_ARG.
  *
- * All supported shapes run on the mma.sync chain kernels (the tcgen05 kernels
- * serve deltanet_fwd only).
+ * bf16 with d_k = d_v = 128 runs on the tensor-core (tcgen05) kernels' gated
+ * instances: a pre-pass that also writes T diag(lambda), the decayed queries and
+ * the row factors per (chunk, head), then the summary and boundary passes.  The
+ * other supported shapes run on the mma.sync chain kernels.
  */
 dn_status gated_deltanet_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                              const dn_tensor* beta, const dn_tensor* g,
@@ -164,8 +166,10 @@ dn_status gated_deltanet_fwd_ex(const dn_tensor* q, const dn_tensor* k, const dn
  *   other arguments, layouts, ownership and errors as deltanet_fwd /
  *   gated_deltanet_fwd; chunk_states may not overlap any other tensor.
  *
- * These calls run on the mma.sync chain kernels, which keep the state in
- * registers and store it at every chunk start.
+ * bf16 with d_k = d_v = 128 runs on the tensor-core kernels, whose boundary
+ * pass stores the state from tensor memory at every chunk start; the other
+ * supported shapes run on the mma.sync chain kernels, which keep the state in
+ * registers and store it likewise.
  */
 dn_status deltanet_fwd_states(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                               const dn_tensor* beta, const dn_tensor* g,
@@ -202,6 +206,8 @@ dn_status deltanet_fwd_states(const dn_tensor* q, const dn_tensor* k, const dn_t
  *   out           [B, T, H, d_v]        one row per token
  *   other arguments, layouts, ownership, aliasing and errors as gated_deltanet_fwd;
  *   B * T * n_h must stay below 2^31.
+ * bf16 with d_k = d_v = 128 runs on the tensor-core kernels' gated instances for
+ * several steps per token; the other supported shapes on the mma.sync chain kernels.
  */
 dn_status gated_deltaproduct_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v,
                                  const dn_tensor* beta, const dn_tensor* g,
@@ -232,8 +238,13 @@ dn_status gated_deltaproduct_fwd_ex(const dn_tensor* q, const dn_tensor* k, cons
  *       (within a chunk the kernel forms decay ratios over up to 15 tokens from
  *       running sums of g, which stay in range under that bound).
  * Supported: bf16 q/k/v/out with d_k, d_v in {64, 128}, dense or packed
- * (cu_seqlens), split across SMs like deltanet_fwd.  Runs on the mma.sync chain
- * kernels.  Pad rows of a last partial chunk carry g = 0 (identity steps).
+ * (cu_seqlens), split across SMs like deltanet_fwd.  A dense batch with
+ * d_k = d_v = 128 whose chains the schedule does not split runs on the tensor
+ * cores: a KDA pre-pass writes T, P, the decayed Q<-, K<-, K-> and lambda[1:C]
+ * per (chunk, head) (66,560 bytes of workspace each), then the boundary kernel's
+ * KDA instance runs the chains.  Split chains, packed input and d = 64 run on
+ * the mma.sync chain kernels.  Pad rows of a last partial chunk carry g = 0
+ * (identity steps).
  * Returns DN_ERR_UNSUPPORTED for fp32 inputs or other head sizes.
  */
 dn_status kda_fwd(const dn_tensor* q, const dn_tensor* k, const dn_tensor* v, const dn_tensor* beta,
