@@ -185,19 +185,21 @@ __device__ __forceinline__ void blk16_finish(float* Nij, const float* Nii, float
 // Blocked solve of (I + A) N = I for the strictly lower A (= B L, 64 x 64, fp32,
 // row stride 65), followed by T = N diag(beta) written to a swizzled tile, and,
 // when colscale is given, T diag(colscale) to a second tile T2.
-// Diagonal 16 x 16 blocks by forward substitution, one column per thread;
-// off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order of i - j.
-// For bf16 operands (whose T is rounded to bf16 anyway) the off-diagonal block products
-// take tf32 inputs on the tensor cores, one warp per block, staged in N's strictly upper
-// blocks (never read); fp32 runs them as fp32 FMAs.
+// Diagonal 16 x 16 blocks by forward substitution, one warp per block and one column per
+// lane (lanes 16-31 repeat 0-15: two blocks in one warp would sit 16 * 65 + 16 floats apart,
+// in the same banks); off-diagonal blocks by N_ij = -N_ii sum_{k=j}^{i-1} A_ik N_kj, in order
+// of i - j.  N's strictly upper blocks are never read as N.  For bf16 operands (whose T is
+// rounded to bf16 anyway) the off-diagonal block products take tf32 inputs on the tensor
+// cores, one warp per block, staged in those upper blocks; fp32 runs them as fp32 FMAs.
 template <typename E, int NT = kThreads>
 __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
                                          const float* beta, E* Ts,
                                          const float* colscale = nullptr, E* T2 = nullptr) {
+    static_assert(NT >= 128, "one warp per diagonal block");
     constexpr int LD = 65;
     const int tid = threadIdx.x;
-    if (tid < 64) {
-        const int blk = tid >> 4, c = tid & 15;
+    if (tid < 128) {
+        const int blk = tid >> 5, c = tid & 15;
         const float* Ab = Af + (16 * blk) * LD + 16 * blk;
         float x[16];
 #pragma unroll
@@ -207,17 +209,10 @@ __device__ __forceinline__ void ut_solve(const float* Af, float* Nf, float* Xt,
             for (int j = 0; j < i; ++j) a = fmaf(-Ab[i * LD + j], x[j], a);
             x[i] = a;
         }
-        float* Nb = Nf + (16 * blk) * LD + 16 * blk;
+        if ((tid & 31) < 16) {
+            float* Nb = Nf + (16 * blk) * LD + 16 * blk;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Nb[i * LD + c] = x[i];
-    } else {
-        // zero the strictly upper blocks: (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
-            const int p = e >> 8;
-            const int bi = p < 3 ? 0 : (p < 5 ? 1 : 2);
-            const int bj = p < 3 ? p + 1 : (p < 5 ? p - 1 : 3);
-            const int ri = (e >> 4) & 15, cj = e & 15;
-            Nf[(16 * bi + ri) * LD + 16 * bj + cj] = 0.f;
+            for (int i = 0; i < 16; ++i) Nb[i * LD + c] = x[i];
         }
     }
     __syncthreads();
