@@ -16,6 +16,13 @@
 // block's first row s (exp(G_l - G_m) = exp(G_l - G_s) exp(G_s - G_m)), which keeps
 // every factor in range for |g| < 5.8 per token and channel (see dn_chain.cuh).
 //
+// Per unit a CTA (8 warps, two per SM) waits for the chunk's k, q, beta and log decays
+// (copies issued while the previous unit's solve ran), forms the running sums, loads each
+// thread's four rows of running sums and k (piece c8 = tid % 16 of rows tid / 16 + 16 i)
+// into registers, builds the four Gram blocks (operand rows scaled 8 channels at a time,
+// one fast exponential per element, then mma.sync warp products), stores Q<-, K<- and K->
+// straight from registers into the unit, solves for T and copies T and P out.
+//
 // Unit layout in the workspace (66,560 bytes per (chunk, head)): T and P (bf16 64 x 64,
 // 128-byte rows, 16-byte pieces swizzled by row % 8: the tensor cores' operand layout),
 // Q<-, K<-, K-> (each two boxes of 64 channels x 64 rows in the same layout, the layout a
