@@ -70,7 +70,7 @@ static __device__ unsigned long long g_dn_trace_prep[16 * 8];
 
 constexpr int kPrepThreads = 128;
 template <bool GATED>
-constexpr int prep_ctas_per_sm() { return GATED ? 5 : 6; }
+constexpr int prep_ctas_per_sm() { return 6; }
 constexpr int kPrepCtasPerSm = prep_ctas_per_sm<false>();
 constexpr int kBlkLd = 20;  // fp32 16 x 16 blocks, 16-byte aligned rows
 constexpr int kBlkFloats = 16 * kBlkLd;
@@ -84,8 +84,8 @@ struct PrepSmemT {
     static constexpr int OFF_A = 0;                               // 10 blocks of A = B L; later the T tile
     static constexpr int OFF_N = OFF_A + 10 * kBlkFloats * 4;     // 10 blocks of N; before them the P tile
     static constexpr int OFF_X = OFF_N + 10 * kBlkFloats * 4;     // 5 staging blocks of the off-diagonal solve
-    static constexpr int OFF_T2 = 32768;                          // gated: the T' tile
-    static constexpr int OFF_BETA = GATED ? 40960 : 32768;        // 2 x 64 step sizes
+    static constexpr int OFF_T2 = 8192;                           // gated: the T' tile, once N is read
+    static constexpr int OFF_BETA = 32768;                        // 2 x 64 step sizes
     static constexpr int OFF_G = OFF_BETA + 2 * kChunk * 4;       // gated: 2 x 64 log decays
     static constexpr int OFF_C = OFF_G + (GATED ? 2 * kChunk * 4 : 0);  // gated: 64 running sums
     static constexpr int OFF_LAM = OFF_C + (GATED ? kChunk * 4 : 0);    // gated: exp of those
@@ -186,8 +186,8 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
     // (cp.async, zero past the chunk's last token, which zeroes T's rows and
     // columns there; one group)
     // With t_staged, the T tile of the previous unit is being copied out of the first
-    // 8 KB of the region: the three other boxes go first, the Q box that overwrites the
-    // staging once the copy has read it.
+    // 8 KB of the region (gated: and T' out of the next 8 KB): the other boxes go first,
+    // the boxes that overwrite the staging once the copies have read it.
     auto issue = [&](int u, int bb, bool t_staged) {
         const int id = u / H, head = u % H;
         int b, t0, t1;
@@ -195,11 +195,12 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         const int tq0 = nh > 1 ? t0 / nh : t0;  // token of the chunk's first step (q is per token)
         if (tid == 0) {
             sm100::mbar_expect_tx(&bars[0], 32768u);
-            sm100::tma_load_4d(smem + L::OFF_QK + 8192, &tk, &bars[0], 0, head, t0, b);
+            if (!GATED) sm100::tma_load_4d(smem + L::OFF_QK + 8192, &tk, &bars[0], 0, head, t0, b);
             sm100::tma_load_4d(smem + L::OFF_QK + 16384, &tq, &bars[0], 64, head, tq0, b);
             sm100::tma_load_4d(smem + L::OFF_QK + 16384 + 8192, &tk, &bars[0], 64, head, t0, b);
             if (t_staged) sm100::bulk_wait_read0();
             sm100::tma_load_4d(smem + L::OFF_QK, &tq, &bars[0], 0, head, tq0, b);
+            if (GATED) sm100::tma_load_4d(smem + L::OFF_QK + 8192, &tk, &bars[0], 0, head, t0, b);
         }
         if (tid < kChunk) {
             const bool ok = tid < t1 - t0;
@@ -482,6 +483,7 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
         {
             const int i = 32 * (warp & 1) + lane, hh = warp >> 1, bi = i >> 4;
             uint8_t* tg = smem + L::OFF_A;
+            uint4 t2w[4];  // gated: this thread's pieces of T', written once N is read
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int j0 = 32 * hh + 8 * cc, bj = j0 >> 4;
@@ -513,13 +515,17 @@ static __global__ void __launch_bounds__(kPrepThreads, prep_ctas_per_sm<GATED>()
                     float l8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) l8[e] = vals[e] * lam[j0 + e];
-                    uint4 w2;
-                    w2.x = sm100::pack_bf16(l8[0], l8[1]);
-                    w2.y = sm100::pack_bf16(l8[2], l8[3]);
-                    w2.z = sm100::pack_bf16(l8[4], l8[5]);
-                    w2.w = sm100::pack_bf16(l8[6], l8[7]);
-                    *reinterpret_cast<uint4*>(smem + L::OFF_T2 + sm100::swz128(i, j0)) = w2;
+                    t2w[cc].x = sm100::pack_bf16(l8[0], l8[1]);
+                    t2w[cc].y = sm100::pack_bf16(l8[2], l8[3]);
+                    t2w[cc].z = sm100::pack_bf16(l8[4], l8[5]);
+                    t2w[cc].w = sm100::pack_bf16(l8[6], l8[7]);
                 }
+            }
+            if constexpr (GATED) {
+                __syncthreads();  // N is read: T' takes the region's second 8 KB
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    *reinterpret_cast<uint4*>(smem + L::OFF_T2 + sm100::swz128(i, 32 * hh + 8 * cc)) = t2w[cc];
             }
             sm100::fence_async_smem();
         }
