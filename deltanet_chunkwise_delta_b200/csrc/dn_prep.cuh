@@ -36,13 +36,13 @@
 // others' outputs are not stored) and its log decay that of the token on its first step,
 // 0 on the others.  The unit's q box is loaded from token (first step) / n_h and expanded
 // to one row per step in shared memory before the Gram product.
-// One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM (five when
-// gated), so the latency of the solve is hidden by parallelism across chunks.  A CTA's shared
-// memory is one 32 KB region that holds the unit's q/k tile until the product
-// has read it, and then the solve's blocks, the P tile (staged where N is
-// written later) and the T tile (staged where A was); the next unit's tile is
-// loaded as soon as the T tile is built, its first box once the T copy has read
-// the staging.
+// One CTA of 4 warps per (chunk, head) at a time, six CTAs per SM, so the latency of
+// the solve is hidden by parallelism across chunks.  A CTA's shared memory is one 32 KB
+// region that holds the unit's q/k tile until the product has read it, and then the
+// solve's blocks, the P tile (staged where N is written later), the T tile (staged where
+// A was) and, gated, the T' tile (staged in the next 8 KB once N is read); the next
+// unit's tile is loaded as soon as the T tile is built, the boxes over the T (and T')
+// staging once the copies have read it.
 #pragma once
 
 #include "dn_chain.cuh"
